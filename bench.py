@@ -1,0 +1,366 @@
+"""Benchmark of the two-stage DDIM denoiser on B200.
+
+One bench step = one full generation of the throughput workload: 100 DDIM steps,
+B=16 prompts x 150 frames, CFG 2.0, cond and uncond batched (32 sequences of 151
+tokens per network forward), bf16 tensor-core path, random-init weights and
+seeded synthetic inputs.  Metric: clips/min (whole job), higher is better.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+N > 1 runs one process per GPU (torchrun); every rank generates its own 16
+prompts (weak scaling, no collective on the data path); time = max over ranks.
+--impl reference times the plain CPU oracle on the host cores on a bounded
+sample of the same workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+WORKLOAD = dict(batch=16, frames=150, steps=100, cfg_scale=2.0)
+METRIC = "clips/min (150-frame, 100-step DDIM, B=16) + denoiser % of roofline"
+UNIT = "clips/min"
+L2_FLUSH_BYTES = 256 << 20
+GEMM_FLOP_PER_TOKEN = 268_435_456      # 2 * 16 * (3d^2 + d^2 + 2 d F), per network forward
+
+
+def workload_config(n_gpus):
+    w = WORKLOAD
+    return {"workload": f"100-step DDIM two-stage generation, B={w['batch']} prompts x {w['frames']} frames, "
+                        f"CFG {w['cfg_scale']}, cond+uncond batched (32 x 151 tokens per forward)",
+            "batch_per_gpu": w["batch"], "frames": w["frames"], "ddim_steps": w["steps"],
+            "cfg_scale": w["cfg_scale"], "global_batch": w["batch"] * n_gpus,
+            "parallelism": f"replicas x{n_gpus} (independent prompts per GPU)",
+            "l2": "flushed between timed iterations (256 MiB write)"}
+
+
+def rank_inputs(rank: int):
+    """Seeded inputs of one rank: distinct prompts and noise per rank."""
+    import synth
+    w = WORKLOAD
+    emb = synth.text_embeddings(w["batch"], seed=synth.SEED_TEXT + 1000 * rank)
+    noise = synth.noise(w["batch"], w["frames"], seed=synth.SEED_NOISE + 1000 * rank)
+    null = synth.null_embeddings(1)[0]
+    lengths = np.full(w["batch"], w["frames"], np.int32)
+    return emb, null, noise, lengths
+
+
+def clips_per_min(n_gpus: int, steps: int, seconds: float) -> float:
+    return n_gpus * WORKLOAD["batch"] * steps * 60.0 / seconds
+
+
+def tokens_per_s(n_gpus: int, steps: int, seconds: float) -> float:
+    w = WORKLOAD
+    toks = 2 * 2 * w["batch"] * (w["frames"] + 1) * w["steps"]   # 2 nets x (cond, uncond)
+    return n_gpus * toks * steps / seconds
+
+
+# --------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{device_index}.csv")
+
+    def __enter__(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        rows = []
+        for line in open(self.path):
+            p = [x.strip() for x in line.split(",")]
+            if len(p) >= 9 and p[1].replace(".", "").isdigit():
+                rows.append(p)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[1]) for r in rows]
+        mx = max(float(r[2]) for r in rows)
+        under = [s for s in sm if s > 0.3 * mx] or sm
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(under), "sm_max_mhz": mx, "reasons": reasons,
+                "samples": len(rows), "power_w_max": max(float(r[3]) for r in rows if r[3].replace(".", "").isdigit())}
+
+
+# --------------------------------------------------------------------------- roofline
+
+def _measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+def _ncu_traffic():
+    """DRAM bytes per tcgen05-GEMM launch from the committed ncu summary, or None
+    if the GEMM source changed since those counters were taken."""
+    path = os.path.join(ROOT, "profiles", "gemm_tc_traffic.txt")
+    src = os.path.join(ROOT, "transformer_denoiser_b200", "csrc", "gemm_tc.cu")
+    if not os.path.exists(path):
+        return None
+    vals = {}
+    for line in open(path):
+        if "=" in line and not line.lstrip().startswith("#"):
+            k, v = line.split("=", 1)
+            vals[k.strip()] = v.strip()
+    sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
+    if vals.get("gemm_tc_source_sha256") != sha:
+        return None
+    try:
+        return float(vals["dram_bytes_per_launch_c4"])
+    except (KeyError, ValueError):
+        return None
+
+
+def roofline(prof):
+    peaks, kind = _measured_peaks()
+    g = prof["gemm_tc"]
+    achieved = g["flops"] / (g["ms"] * 1e-3) / 1e12
+    peak = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))
+    return {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
+            "frac": round(achieved / peak, 4), "traffic": _ncu_traffic(),
+            "kernel": "gemm_tc (tcgen05 bf16 GEMM, all projections)",
+            "launches_per_step": g["launches"], "ms_per_step": round(g["ms"], 3),
+            "peak_source": f"{kind} sustained bf16 GEMM (MEASURED_PEAKS.json)" if kind == "measured" else
+                           "fallback sustained bf16 figure",
+            "other_kernels_ms": {k: round(v["ms"], 3) for k, v in prof.items() if k != "gemm_tc" and v["launches"]}}
+
+
+# --------------------------------------------------------------------------- CPU oracle leg
+
+_ORACLE_PARAMS = None
+
+
+def oracle_sample(target_s: float = 12.0):
+    """Time the CPU oracle on a bounded sample of the workload: DDIM steps of one
+    sequence (cond + uncond chains, 4 transformer forwards per step) until
+    ~target_s of CPU work; returns (clips/min, seconds per sequence-step, desc, threads)."""
+    import synth
+    from oracle import kimodo_oracle as ko
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [os.cpu_count()])
+    except Exception:
+        threads = os.cpu_count()
+    w = WORKLOAD
+    global _ORACLE_PARAMS
+    if _ORACLE_PARAMS is None:
+        _ORACLE_PARAMS = ko.unpack_weights(synth.weight_blob())
+    params = _ORACLE_PARAMS
+    emb, null, noise, lengths = rank_inputs(0)
+    ab = ko.alphabar_linear()
+    ts = ko.ddim_timesteps(w["steps"])
+    x = noise[0].astype(np.float64)
+    n = 0
+    t0 = time.perf_counter()
+    while True:
+        t, tp = ts[n % len(ts)]
+        x, _ = ko.ddim_step(params, x, emb[0], null, w["frames"], t, tp, w["cfg_scale"], ab)
+        n += 1
+        el = time.perf_counter() - t0
+        if el >= target_s or n >= len(ts):
+            break
+    per_step = el / n
+    clips = 60.0 / (per_step * w["steps"])
+    desc = (f"{n} DDIM steps of 1 sequence (150 frames, cond+uncond = 4 forwards/step), fp64 numpy, "
+            f"extrapolated x100 steps per clip")
+    return clips, per_step, desc, threads
+
+
+# --------------------------------------------------------------------------- our arm
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    import synth
+    import transformer_denoiser_b200 as kb
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    model = kb.Kimodo(synth.weight_blob(), kb.BF16, local_rank)
+    emb, null, noise, lengths = rank_inputs(rank)
+    d_emb = torch.from_numpy(emb).to(dev)
+    d_null = torch.from_numpy(null).to(dev)
+    d_noise = torch.from_numpy(noise).to(dev)
+    d_len = torch.from_numpy(lengths).to(dev)
+    d_out = torch.empty_like(d_noise)
+    w = WORKLOAD
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(out=d_out):
+        model.ddim_sample(d_emb, d_null, d_noise, d_len, w["steps"], w["cfg_scale"], out=out)
+
+    for _ in range(max(args.warmup, 3) if args.warmup > 0 else 3):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    model.sync_status()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local_rank) as clk:
+        barrier()
+        torch.cuda.synchronize()
+        ev0.record(stream)
+        for _ in range(args.steps):
+            flush.zero_()
+            step()
+        ev1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+    ms = ev0.elapsed_time(ev1)
+    launches_per_step = model.last_launch_count()
+    model.sync_status()
+
+    # end-to-end: HOST (pinned) inputs and output through the same C-ABI call
+    h_emb = torch.from_numpy(emb).pin_memory()
+    h_null = torch.from_numpy(null).pin_memory()
+    h_noise = torch.from_numpy(noise).pin_memory()
+    h_len = torch.from_numpy(lengths).pin_memory()
+    h_out = torch.empty(h_noise.shape, dtype=torch.float32).pin_memory()
+    model.ddim_sample(h_emb, h_null, h_noise, h_len, w["steps"], w["cfg_scale"], out=h_out)
+    e2e_steps = max(1, min(args.steps, 5))
+    barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        flush.zero_()
+        model.ddim_sample(h_emb, h_null, h_noise, h_len, w["steps"], w["cfg_scale"], out=h_out)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = e0.elapsed_time(e1)
+    h2d = h_emb.numel() * 4 + h_null.numel() * 4 + h_noise.numel() * 4 + h_len.numel() * 4
+    d2h = h_out.numel() * 4
+
+    # per-kernel live timing of one generation (CUDA events around every launch)
+    model.profile_enable(True)
+    flush.zero_()
+    step()
+    prof = model.profile_read(6)
+    model.profile_enable(False)
+    model.sync_status()
+
+    t = torch.tensor([ms, e2e_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_max, e2e_max = float(t[0]), float(t[1])
+    model.close()
+    if rank != 0:
+        return None
+    sec = ms_max / 1e3
+    line = {
+        "metric": METRIC, "value": round(clips_per_min(world, args.steps, sec), 3), "unit": UNIT,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(ms_max / args.steps, 3), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) embeddings and noise; "
+                                                         "random-init N(0,0.02) weights)",
+        "config": workload_config(world),
+        "denoiser_tokens_per_s": round(tokens_per_s(world, args.steps, sec), 1),
+        "e2e": {"value": round(clips_per_min(world, e2e_steps, e2e_max / 1e3), 3), "unit": UNIT,
+                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
+        "gpu_launches": int(launches_per_step * args.steps),
+        "roofline": roofline(prof),
+        "clocks": clk.summary(),
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        clips, per_step, desc, threads = oracle_sample()
+        line["cpu_baseline"] = {"value": round(clips, 6), "unit": UNIT, "cores": threads, "kind": "oracle",
+                                "sample": desc}
+    return line
+
+
+def run_reference(args, rank):
+    if rank != 0:
+        return None
+    t0 = time.perf_counter()
+    vals = []
+    desc, threads = "", 1
+    for _ in range(max(1, args.steps)):
+        clips, per_step, desc, threads = oracle_sample(target_s=min(12.0, 120.0 / max(1, args.steps)))
+        vals.append(clips)
+    v = float(statistics.median(vals))
+    return {"impl": "reference", "metric": METRIC, "value": round(v, 6), "unit": UNIT,
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(60e3 * WORKLOAD["batch"] / v, 1), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": workload_config(1),
+            "cpu_baseline": {"kind": "oracle", "cores": threads, "sample": desc, "value": round(v, 6)},
+            "e2e": {"value": round(v, 6), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+            "wall_s": round(time.perf_counter() - t0, 1)}
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    local_rank = int(os.environ.get("LOCAL_RANK", 0))
+    if args.impl == "reference":
+        line = run_reference(args, rank)
+    else:
+        if world > 1:
+            import torch
+            import torch.distributed as dist
+            torch.cuda.set_device(local_rank)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
+                                    device_id=torch.device("cuda", local_rank))
+        try:
+            line = run_ours(args, rank, world, local_rank)
+        finally:
+            if world > 1:
+                import torch.distributed as dist
+                dist.destroy_process_group()
+    if line is not None:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,161 @@
+/*
+ * kimodo.h -- C ABI of the B200 (sm_100a) two-stage DDIM motion denoiser.
+ *
+ * The library runs the denoising loop of a Kimodo-style text-to-motion model on
+ * one GPU: per DDIM step a root transformer, the global-to-local root transform,
+ * a body transformer, classifier-free guidance and the DDIM x(t-1) update
+ * ("Kimodo WebGPU" page, "Architecture" figure and "Model details" table).
+ * The text encoder is not part of the library: 4096-float embeddings are inputs.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * Return value: KIMODO_OK (0) or a negative KIMODO_E* status; the message of the
+ *   last failure on the calling thread is available from kimodo_last_error().
+ *   No exception or abort crosses this boundary.
+ * Pointers: every tensor argument may be HOST memory (pageable or pinned) or
+ *   DEVICE memory of the context's GPU; the library detects which.  Host inputs
+ *   are copied to device staging on `stream`; when any output is host memory the
+ *   call synchronises `stream` before returning, otherwise it returns once the
+ *   work is enqueued (asynchronous).  The caller keeps ownership of all tensors.
+ * Layouts: row-major float32, C order.  Motion features per frame are
+ *   [root 5 | body 274] = 279 floats; root 5 = (x, z, sin heading,
+ *   cos heading, height); body 274 = 30 joints x (3 position + 6D rotation) +
+ *   4 foot contacts.
+ * Masking: frames at index >= lengths[b] are padding.  Their input values,
+ *   whatever they are (NaN included), never reach a valid output, and every
+ *   output writes 0 there.
+ * stream: a cudaStream_t cast to void*; NULL means the legacy default stream.
+ * Device-side failures (a bounded wait in a kernel that ran out) are reported
+ *   by kimodo_sync_status() and by the next call on the context.
+ */
+#ifndef KIMODO_H
+#define KIMODO_H
+
+#include <stddef.h>
+
+#if defined(__GNUC__)
+#define KIMODO_API __attribute__((visibility("default")))
+#else
+#define KIMODO_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct kimodo_ctx kimodo_ctx;
+
+enum {
+  KIMODO_OK = 0,
+  KIMODO_EINVAL = -1,       /* bad argument (message says which) */
+  KIMODO_ENOMEM = -2,       /* device or host allocation failed */
+  KIMODO_ECUDA = -3,        /* a CUDA runtime/driver call failed */
+  KIMODO_EUNSUPPORTED = -4, /* no sm_100 device, or the kernels are missing */
+  KIMODO_ETIMEOUT = -5      /* a kernel's bounded wait gave up */
+};
+
+enum { KIMODO_FP32 = 0, KIMODO_BF16 = 1 };
+enum { KIMODO_NET_ROOT = 0, KIMODO_NET_BODY = 1 };
+
+/* Model constants ("Kimodo WebGPU", "Model details": 16-layer post-norm encoders,
+ * 1024 hidden, 8 heads x 128, 2048 FFN; 282M parameters in all). */
+#define KIMODO_N_PARAMS 281963799u
+#define KIMODO_TEXT_DIM 4096
+#define KIMODO_MOTION_DIM 279
+#define KIMODO_ROOT_DIM 5
+#define KIMODO_BODY_DIM 274
+#define KIMODO_MAX_FRAMES 300
+
+/*
+ * Create a context on CUDA device `device` and upload the weights.
+ *
+ * host_blob: n_floats float32 values in the canonical order (root network, then
+ *   body network; per network: text projection W[1024x4096], b[1024]; timestep
+ *   MLP W1[1024x1024], b1, W2[1024x1024], b2; input projection W[1024xDin], b;
+ *   16 x (qkv W[3072x1024] with rows Q,K,V, qkv b[3072], out-proj W[1024x1024],
+ *   b, LayerNorm-1 gamma, beta, FFN-1 W[2048x1024], b[2048], FFN-2 W[1024x2048],
+ *   b, LayerNorm-2 gamma, beta); output projection W[Doutx1024], b[Dout]).
+ *   Din/Dout = 5/5 (root) and 279/274 (body).  Matrices are [out x in].
+ *   Read during the call only; host or device memory.
+ * n_floats: must equal KIMODO_N_PARAMS, else KIMODO_EINVAL.
+ * precision: KIMODO_BF16 (tensor-core path: bf16 operands, fp32 accumulation,
+ *   fp32 LayerNorm/softmax/DDIM) or KIMODO_FP32 (fp32 everywhere).
+ * On success *ctx receives a context owned by the caller (kimodo_free).
+ */
+KIMODO_API int kimodo_load_weights(kimodo_ctx** ctx, const float* host_blob, size_t n_floats,
+                        int precision, int device);
+
+/*
+ * One sub-network forward ("Kimodo WebGPU", "Model details": one 16-layer
+ * TransformerEncoder).  Sequence = [condition token | T frame tokens]; the
+ * condition token is TextProj(emb) + TimestepMLP(sinusoid(t)).
+ *
+ * net: KIMODO_NET_ROOT (Din=5, Dout=5) or KIMODO_NET_BODY (Din=279, Dout=274).
+ * x: [batch, frames, Din] input features.  emb: [batch, 4096] text embeddings.
+ * t: diffusion timestep in [0, 999].  lengths: int32 [batch], 1..frames.
+ * out: [batch, frames, Dout] network output (padded frames written as 0).
+ * 1 <= batch, 1 <= frames <= 300.
+ */
+KIMODO_API int kimodo_denoiser_forward(kimodo_ctx* ctx, int net, const float* x, const float* emb, int t,
+                            const int* lengths, int batch, int frames, float* out, void* stream);
+
+/*
+ * One two-stage DDIM step with classifier-free guidance, cond and uncond
+ * batched in one pass per network:
+ *   per branch: root = Root(x_t[..., :5]); local = G2L(root);
+ *               body = Body([x_t[..., 5:] | local]); x0_branch = [root | body]
+ *   x0 = x0_u + cfg_scale (x0_c - x0_u)
+ *   x_prev = sqrt(ab_prev) x0 + sqrt(1 - ab_prev) (x_t - sqrt(ab_t) x0) / sqrt(1 - ab_t)
+ * with ab the linear-beta (1e-4..0.02, 1000 steps) cumulative product, ab(-1) = 1.
+ *
+ * x_t: [batch, frames, 279].  text_emb: [batch, 4096].  null_emb: [4096]
+ *   (broadcast) or [batch, 4096], pass null_batch = 1 or batch.
+ * t in [0, 999], t_prev in [-1, t).  cfg_scale finite.
+ * x_prev: [batch, frames, 279]; may alias x_t.
+ */
+KIMODO_API int kimodo_ddim_step(kimodo_ctx* ctx, const float* x_t, const float* text_emb,
+                     const float* null_emb, int null_batch, const int* lengths, int batch,
+                     int frames, int t, int t_prev, float cfg_scale, float* x_prev, void* stream);
+
+/*
+ * Full DDIM sampling loop: `steps` two-stage steps (as kimodo_ddim_step) on the
+ * trailing timesteps t_k = 999 - k (1000/steps), t_prev = t_k - 1000/steps,
+ * starting from `noise`.  steps must divide 1000.  The loop runs as one CUDA
+ * graph captured per (batch, frames, steps, cfg_scale) and cached in the context;
+ * no host synchronisation happens between steps.
+ *
+ * noise: [batch, frames, 279].  out: [batch, frames, 279] final sample; may alias noise.
+ */
+KIMODO_API int kimodo_ddim_sample(kimodo_ctx* ctx, const float* text_emb, const float* null_emb,
+                       int null_batch, const float* noise, const int* lengths, int batch,
+                       int frames, int steps, float cfg_scale, float* out, void* stream);
+
+/* Synchronise `stream` and report any device-side failure recorded since the
+ * last check (KIMODO_ETIMEOUT with the kernel named in kimodo_last_error()). */
+KIMODO_API int kimodo_sync_status(kimodo_ctx* ctx, void* stream);
+
+/* Per-kernel-class timing of the next calls (instrumentation, off by default).
+ * With enable != 0, kimodo_ddim_sample runs eagerly (no graph) and brackets every
+ * launch with CUDA events; kimodo_profile_read() returns, for each of
+ * n_classes <= 8 classes (0 tensor-core GEMM, 1 attention, 2 LayerNorm,
+ * 3 elementwise/motion, 4 fp32 GEMM, 5 setup), the summed milliseconds, the
+ * number of launches and the algorithmic FLOPs and bytes since the last reset. */
+KIMODO_API int kimodo_profile_enable(kimodo_ctx* ctx, int enable);
+KIMODO_API int kimodo_profile_read(kimodo_ctx* ctx, int n_classes, double* ms, long long* launches,
+                        double* flops, double* bytes);
+
+/* Number of this library's kernel launches enqueued by the last completed
+ * sample/step/forward call (graph nodes included). */
+KIMODO_API long long kimodo_last_launch_count(kimodo_ctx* ctx);
+
+/* Release the context and all device memory it owns.  NULL is accepted. */
+KIMODO_API void kimodo_free(kimodo_ctx* ctx);
+
+/* Message of the last failure on the calling thread ("" if none). */
+KIMODO_API const char* kimodo_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KIMODO_H */

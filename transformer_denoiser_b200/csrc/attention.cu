@@ -1,0 +1,251 @@
+// Masked multi-head self-attention ("Kimodo WebGPU", "WGSL compute shaders"
+// table: multi-head self-attention with optional key masking).
+//
+// Per (sequence, head) the keys 0..n_valid-1 take part, n_valid = 1 + length
+// (the condition token is always valid).  Keys at or beyond n_valid are never
+// loaded: their shared-memory rows are zero-filled and their scores are set to
+// -inf by selection, so padded content (even NaN) cannot reach an output.
+//
+// bf16 kernel: one CTA per (64-query block, head, sequence), 4 warps of 16 query
+// rows.  K and V of the valid keys are staged in shared memory (row stride 136
+// bf16 to keep ldmatrix conflict-free); Q K^T and P V run on mma.sync
+// m16n8k16 (bf16 in, fp32 accumulate) with an online softmax over 64-key blocks
+// whose row max / sum are reduced across the 4-thread quads by warp shuffles.
+//
+// fp32 kernel (fp32 path): one warp per query row, scores by warp-shuffle dot
+// products, online softmax in fp32.
+#include <cuda_runtime.h>
+#include <math.h>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "ptx.cuh"
+
+namespace kd {
+namespace {
+
+constexpr int QB = 64;
+constexpr int KBLK = 64;
+constexpr int LDS = DH + 8;   // smem row stride in bf16 elements
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(addr));
+}
+__device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+__global__ void __launch_bounds__(128) attn_bf16_kernel(const bf16* __restrict__ qkv, bf16* __restrict__ out,
+                                                        const int* __restrict__ lengths, int len_mod, int S) {
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  bf16* sQ = reinterpret_cast<bf16*>(smem_raw);
+  const int q0 = blockIdx.x * QB, h = blockIdx.y, seq = blockIdx.z;
+  int n_valid = 1 + lengths[seq % len_mod];
+  n_valid = n_valid < 1 ? 1 : (n_valid > S ? S : n_valid);
+  const int nkb = (n_valid + KBLK - 1) / KBLK;
+  bf16* sK = sQ + QB * LDS;
+  bf16* sV = sK + nkb * KBLK * LDS;
+
+  const long rs = 3L * D;
+  const bf16* base = qkv + (long)seq * S * rs + h * DH;
+  const int tid = threadIdx.x;
+  for (int c = tid; c < QB * 16; c += 128) {
+    const int r = c >> 4, ch = c & 15, q = q0 + r;
+    const bool v = q < S;
+    ptx::cp_async_16_zfill(ptx::smem_u32(sQ + r * LDS + ch * 8), base + (long)(v ? q : 0) * rs + ch * 8, v);
+  }
+  for (int c = tid; c < nkb * KBLK * 16; c += 128) {
+    const int r = c >> 4, ch = c & 15;
+    const bool v = r < n_valid;
+    const bf16* src = base + (long)(v ? r : 0) * rs + ch * 8;
+    ptx::cp_async_16_zfill(ptx::smem_u32(sK + r * LDS + ch * 8), src + D, v);
+    ptx::cp_async_16_zfill(ptx::smem_u32(sV + r * LDS + ch * 8), src + 2 * D, v);
+  }
+  ptx::cp_async_commit();
+  ptx::cp_async_wait_all();
+  __syncthreads();
+
+  const int warp = tid >> 5, lane = tid & 31;
+  const int qw = q0 + warp * 16;
+  if (qw >= S) return;
+  const int g = lane >> 2, c4 = lane & 3;
+
+  // Q fragments for the 8 k-steps of the 128-wide head
+  uint32_t qf[8][4];
+  {
+    const int r = warp * 16 + (lane & 15);
+    const int cb = (lane >> 4) * 8;
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk)
+      ldsm_x4(ptx::smem_u32(sQ + r * LDS + kk * 16 + cb), qf[kk][0], qf[kk][1], qf[kk][2], qf[kk][3]);
+  }
+
+  const float scale = 0.08838834764831845f * 1.4426950408889634f;  // 1/sqrt(128) * log2(e)
+  float o[16][4];
+#pragma unroll
+  for (int n = 0; n < 16; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
+  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+
+  for (int kb = 0; kb < nkb; ++kb) {
+    float s[8][4];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      s[j][0] = s[j][1] = s[j][2] = s[j][3] = 0.f;
+      const int key = kb * KBLK + j * 8 + (lane & 7);
+#pragma unroll
+      for (int kk2 = 0; kk2 < 4; ++kk2) {
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4(ptx::smem_u32(sK + key * LDS + kk2 * 32 + (lane >> 3) * 8), b0, b1, b2, b3);
+        mma_bf16(s[j], qf[2 * kk2], b0, b1);
+        mma_bf16(s[j], qf[2 * kk2 + 1], b2, b3);
+      }
+    }
+    float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int key = kb * KBLK + j * 8 + 2 * c4;
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const bool ok = key + e < n_valid;
+        s[j][e] = ok ? s[j][e] * scale : -INFINITY;
+        s[j][e + 2] = ok ? s[j][e + 2] * scale : -INFINITY;
+        mx0 = fmaxf(mx0, s[j][e]);
+        mx1 = fmaxf(mx1, s[j][e + 2]);
+      }
+    }
+    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
+    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
+    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
+    const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
+    const float a0 = exp2f(m0 - mn0), a1 = exp2f(m1 - mn1);
+    m0 = mn0;
+    m1 = mn1;
+    float rs0 = 0.f, rs1 = 0.f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      s[j][0] = exp2f(s[j][0] - mn0);
+      s[j][1] = exp2f(s[j][1] - mn0);
+      s[j][2] = exp2f(s[j][2] - mn1);
+      s[j][3] = exp2f(s[j][3] - mn1);
+      rs0 += s[j][0] + s[j][1];
+      rs1 += s[j][2] + s[j][3];
+    }
+    l0 = l0 * a0 + rs0;
+    l1 = l1 * a1 + rs1;
+#pragma unroll
+    for (int n = 0; n < 16; ++n) {
+      o[n][0] *= a0; o[n][1] *= a0;
+      o[n][2] *= a1; o[n][3] *= a1;
+    }
+    // O += P V over the 4 sixteen-key slices of this block
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk) {
+      uint32_t pf[4];
+      pf[0] = pack_bf16(s[2 * kk][0], s[2 * kk][1]);
+      pf[1] = pack_bf16(s[2 * kk][2], s[2 * kk][3]);
+      pf[2] = pack_bf16(s[2 * kk + 1][0], s[2 * kk + 1][1]);
+      pf[3] = pack_bf16(s[2 * kk + 1][2], s[2 * kk + 1][3]);
+      const int key = kb * KBLK + kk * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+#pragma unroll
+      for (int dp = 0; dp < 8; ++dp) {
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4_t(ptx::smem_u32(sV + key * LDS + dp * 16 + (lane >> 4) * 8), b0, b1, b2, b3);
+        mma_bf16(o[2 * dp], pf, b0, b1);
+        mma_bf16(o[2 * dp + 1], pf, b2, b3);
+      }
+    }
+  }
+  l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
+  l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
+  l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
+  l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
+  const float i0 = 1.f / l0, i1 = 1.f / l1;
+  const int r0 = qw + g, r1 = qw + g + 8;
+  bf16* ob = out + (long)seq * S * D + h * DH + 2 * c4;
+#pragma unroll
+  for (int n = 0; n < 16; ++n) {
+    if (r0 < S)
+      *reinterpret_cast<__nv_bfloat162*>(ob + (long)r0 * D + n * 8) = __floats2bfloat162_rn(o[n][0] * i0, o[n][1] * i0);
+    if (r1 < S)
+      *reinterpret_cast<__nv_bfloat162*>(ob + (long)r1 * D + n * 8) = __floats2bfloat162_rn(o[n][2] * i1, o[n][3] * i1);
+  }
+}
+
+__global__ void __launch_bounds__(128) attn_f32_kernel(const float* __restrict__ qkv, float* __restrict__ out,
+                                                       const int* __restrict__ lengths, int len_mod, int S) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int q = blockIdx.x * 4 + warp, h = blockIdx.y, seq = blockIdx.z;
+  if (q >= S) return;
+  int n_valid = 1 + lengths[seq % len_mod];
+  n_valid = n_valid < 1 ? 1 : (n_valid > S ? S : n_valid);
+  const long rs = 3L * D;
+  const float* base = qkv + (long)seq * S * rs + h * DH + lane * 4;
+  const float4 qv = *reinterpret_cast<const float4*>(base + (long)q * rs);
+  const float scale = 0.08838834764831845f;
+  float m = -INFINITY, l = 0.f;
+  float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int j = 0; j < n_valid; ++j) {
+    const float4 kv = *reinterpret_cast<const float4*>(base + (long)j * rs + D);
+    float d = qv.x * kv.x + qv.y * kv.y + qv.z * kv.z + qv.w * kv.w;
+#pragma unroll
+    for (int off = 16; off; off >>= 1) d += __shfl_xor_sync(0xffffffffu, d, off);
+    const float sc = d * scale;
+    const float mn = fmaxf(m, sc);
+    const float a = expf(m - mn), p = expf(sc - mn);
+    const float4 vv = *reinterpret_cast<const float4*>(base + (long)j * rs + 2 * D);
+    l = l * a + p;
+    o.x = o.x * a + p * vv.x;
+    o.y = o.y * a + p * vv.y;
+    o.z = o.z * a + p * vv.z;
+    o.w = o.w * a + p * vv.w;
+    m = mn;
+  }
+  const float inv = 1.f / l;
+  *reinterpret_cast<float4*>(out + ((long)seq * S + q) * D + h * DH + lane * 4) =
+      make_float4(o.x * inv, o.y * inv, o.z * inv, o.w * inv);
+}
+
+}  // namespace
+
+size_t attention_bf16_smem(int S) {
+  const int nk = ((S + KBLK - 1) / KBLK) * KBLK;
+  return (size_t)(QB + 2 * nk) * LDS * sizeof(bf16);
+}
+
+cudaError_t attention_bf16(const bf16* qkv, bf16* out, const int* lengths, int len_mod, int nseq, int S,
+                           cudaStream_t st) {
+  if (nseq <= 0 || S <= 0) return cudaSuccess;
+  const size_t smem = attention_bf16_smem(S);
+  dim3 grid((S + QB - 1) / QB, H, nseq);
+  attn_bf16_kernel<<<grid, 128, smem, st>>>(qkv, out, lengths, len_mod, S);
+  return cudaGetLastError();
+}
+
+cudaError_t attention_prepare() {
+  return cudaFuncSetAttribute(attn_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              (int)attention_bf16_smem(MAX_FRAMES + 1));
+}
+
+cudaError_t attention_f32(const float* qkv, float* out, const int* lengths, int len_mod, int nseq, int S,
+                          cudaStream_t st) {
+  if (nseq <= 0 || S <= 0) return cudaSuccess;
+  dim3 grid((S + 3) / 4, H, nseq);
+  attn_f32_kernel<<<grid, 128, 0, st>>>(qkv, out, lengths, len_mod, S);
+  return cudaGetLastError();
+}
+
+}  // namespace kd

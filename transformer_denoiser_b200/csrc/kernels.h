@@ -1,0 +1,72 @@
+// Internal launchers of the denoiser kernels (not part of the public C ABI).
+#pragma once
+
+#include <cuda_runtime.h>
+#include "common.cuh"
+#include "epilogue.cuh"
+
+namespace kd {
+
+// D[M, N] = A[M, K] . B[N, K]^T; A, B row-major with leading dimensions lda, ldb.
+struct GemmArgs {
+  const void* A = nullptr;
+  const void* B = nullptr;
+  int M = 0, N = 0, K = 0;
+  int lda = 0, ldb = 0;
+};
+
+// tcgen05 bf16 GEMM.  bn in {16, 128, 256}; returns cudaErrorInvalidValue for an
+// unsupported (bn, kind, output type) combination.
+cudaError_t gemm_tc(const GemmArgs& g, int bn, int kind, bool out_f32, const EpiParams& ep, DevError* err,
+                    cudaStream_t st, int num_sms);
+bool gemm_tc_available();
+// Set the dynamic shared-memory limits of every kernel instantiation (call once
+// per device before any launch or graph capture).
+cudaError_t gemm_tc_prepare();
+cudaError_t attention_prepare();
+size_t attention_bf16_smem(int S);
+
+// fp32 SIMT GEMM with the same epilogues (fp32 everywhere).  K % 16 == 0.
+cudaError_t gemm_f32(const GemmArgs& g, int kind, const EpiParams& ep, cudaStream_t st);
+
+// Masked multi-head self-attention over the fused QKV matrix [nseq*S, 3*D]
+// (columns Q | K | V, head h at h*DH).  Keys at token index >= 1 + lengths[seq %
+// len_mod] are excluded.  out [nseq*S, D].
+cudaError_t attention_bf16(const bf16* qkv, bf16* out, const int* lengths, int len_mod, int nseq, int S,
+                           cudaStream_t st);
+cudaError_t attention_f32(const float* qkv, float* out, const int* lengths, int len_mod, int nseq, int S,
+                          cudaStream_t st);
+
+// Row LayerNorm over D features: y fp32 [M, D] -> out (bf16 or fp32) [M, D], and
+// optionally an fp32 copy into out32 (which may be y itself).
+cudaError_t layernorm(const float* y, void* out, bool out_bf16, const float* gamma, const float* beta, int M,
+                      cudaStream_t st, float* out32 = nullptr);
+
+// ---- motion / sampler kernels (element type of the activation matrices: bf16 or fp32)
+
+// A[(seq*S + 1 + i) * lda + col0 + f] = src[((seq % nsrc) * T + i) * ld_src + f0 + f], f < nf, i < T.
+cudaError_t pack_frames(const float* src, int nsrc, int ld_src, int f0, int nf, void* A, bool a_bf16, int lda,
+                        int col0, int nseq, int T, int S, cudaStream_t st);
+
+// Body-network input of the two-stage step: for seq in [0, nseq), frame i < T:
+//   A[.., 0:274] = x[seq % B, i, 5:279];  A[.., 274:279] = G2L(root_hat[seq])[i]  (0 for padded frames)
+cudaError_t g2l_body_input(const float* root_hat, const float* x, const int* lengths, int B, int nseq, int T,
+                           int S, void* A, bool a_bf16, int lda, cudaStream_t st);
+
+// CFG + DDIM update in place on x [B, T, 279]: x0 = u + w (c - u) from the root /
+// body predictions of sequences b (cond) and B + b (uncond); x = c0 x0 + c1 x;
+// padded frames 0.  If A_next != nullptr the new root features are also packed
+// into the root network's input matrix for sequences b and B + b.
+cudaError_t cfg_ddim(const float* root_hat, const float* body_hat, float* x, const int* lengths, int B, int T,
+                     float w, float c0, float c1, void* A_next, bool a_bf16, int lda, int S, cudaStream_t st);
+
+// Condition inputs: rows [0, B) = text_emb, rows [B, B + nnull_rows) = null_emb
+// (row (r - B) % null_batch).  out (bf16 or fp32) [rows, DTXT].
+cudaError_t pack_embeddings(const float* text_emb, int B, const float* null_emb, int null_batch, int null_rows,
+                            void* out, bool out_bf16, cudaStream_t st);
+
+// out[k, :] = pe[t0 - k * stride, :] for k < n (sinusoid rows of the timesteps).
+cudaError_t gather_timestep_rows(const float* pe, int t0, int stride, int n, void* out, bool out_bf16,
+                                 cudaStream_t st);
+
+}  // namespace kd
