@@ -100,6 +100,32 @@ KIMODO_API int kimodo_denoiser_forward(kimodo_ctx* ctx, int net, const float* x,
                             const int* lengths, int batch, int frames, float* out, void* stream);
 
 /*
+ * Allocation-free variant of kimodo_denoiser_forward (the pages describe no
+ * counterpart: it serves callers of this library that must not allocate device
+ * memory).  Some callers cannot call cudaMalloc: an engine or runtime that owns
+ * every byte of device memory through its own allocator or a fixed budget, and
+ * latency-sensitive callers that cannot afford the device-wide synchronisation a
+ * cudaMalloc or cudaFree may cause.  kimodo_denoiser_forward allocates its
+ * activation workspace on first use; this call instead uses a static device array
+ * of the library (about 19 MiB, held by every GPU that loads the library until
+ * the process exits) and calls no cudaMalloc, cudaFree or other allocating
+ * routine.  The context itself is created, with its weights, by
+ * kimodo_load_weights.
+ *
+ * Arguments, layouts and results are those of kimodo_denoiser_forward, within
+ * these limits: batch <= 16 and batch * (frames + 1) <= 512 tokens, else
+ * KIMODO_EINVAL (use kimodo_denoiser_forward for larger calls).
+ * The first call on a device looks up the array's device address (set-up); make
+ * that first call before any stream capture.  Every call on a device shares the
+ * one array and overwrites the previous call's contents: calls whose work can
+ * overlap on the GPU (other streams, other contexts, other threads) race and
+ * must be ordered by the caller.
+ */
+KIMODO_API int kimodo_denoiser_forward_noalloc(kimodo_ctx* ctx, int net, const float* x, const float* emb,
+                                               int t, const int* lengths, int batch, int frames,
+                                               float* out, void* stream);
+
+/*
  * One two-stage DDIM step with classifier-free guidance, cond and uncond
  * batched in one pass per network:
  *   per branch: root = Root(x_t[..., :5]); local = G2L(root);

@@ -28,6 +28,7 @@ _P, _I, _F, _SZ, _LL, _D = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes
 SIGNATURES = [
     ("kimodo_load_weights", _I, [ctypes.POINTER(_P), _P, _SZ, _I, _I]),
     ("kimodo_denoiser_forward", _I, [_P, _I, _P, _P, _I, _P, _I, _I, _P, _P]),
+    ("kimodo_denoiser_forward_noalloc", _I, [_P, _I, _P, _P, _I, _P, _I, _I, _P, _P]),
     ("kimodo_ddim_step", _I, [_P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _F, _P, _P]),
     ("kimodo_ddim_sample", _I, [_P, _P, _P, _I, _P, _P, _I, _I, _I, _F, _P, _P]),
     ("kimodo_sync_status", _I, [_P, _P]),
@@ -206,6 +207,16 @@ class Kimodo:
         out = _like(x, (B, T, dout)) if out is None else out
         _check(self._lib.kimodo_denoiser_forward(self._ctx, int(net), _ptr(x), _ptr(emb), int(t), _ptr(lengths),
                                                  B, T, _ptr(out), _stream(stream, x, out)))
+        return out
+
+    def denoiser_forward_noalloc(self, net, x, emb, t, lengths, out=None, stream=None):
+        """kimodo_denoiser_forward_noalloc: same result, no device allocation (size limits apply)."""
+        x, emb, lengths = _f32(x), _f32(emb), _i32(lengths)
+        B, T = x.shape[0], x.shape[1]
+        dout = ROOT_DIM if net == NET_ROOT else BODY_DIM
+        out = _like(x, (B, T, dout)) if out is None else out
+        _check(self._lib.kimodo_denoiser_forward_noalloc(self._ctx, int(net), _ptr(x), _ptr(emb), int(t),
+                                                         _ptr(lengths), B, T, _ptr(out), _stream(stream, x, out)))
         return out
 
     def ddim_step(self, x_t, text_emb, null_emb, lengths, t, t_prev, cfg_scale, out=None, stream=None):

@@ -866,3 +866,149 @@ int kimodo_layernorm(const float* y, void* out, int out_bf16, const float* gamma
 }
 
 }  // extern "C"
+
+// ====================================================================== allocation-free forward
+//
+// kimodo_denoiser_forward_noalloc runs the same kernels as kimodo_denoiser_forward,
+// but its activation workspace is the file-scope device array below instead of the
+// context's lazily cudaMalloc'ed workspace.  The array is sized for the largest
+// call it accepts (NOALLOC_MAX_ROWS tokens, NOALLOC_MAX_BATCH sequences, fp32
+// elements, which bounds the bf16 layout too).  Its device address is looked up
+// once per device with cudaGetSymbolAddress, on the first call made on that device.
+
+namespace {
+
+constexpr int NOALLOC_MAX_ROWS = 512;    // batch * (frames + 1)
+constexpr int NOALLOC_MAX_BATCH = 16;
+
+// Lays out a Workspace for (rows, nseq, nseq*frames) with element size e starting
+// at `base`; returns the bytes used.  With base == nullptr it only measures.
+constexpr size_t noalloc_layout(char* base, size_t e, size_t rows, size_t nseq, size_t nframes, Workspace* w) {
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    char* p = base ? base + off : nullptr;
+    off += (bytes + 255) & ~size_t(255);
+    return p;
+  };
+  char* h = take(rows * D * e);
+  char* qkv = take(rows * 3 * D * e);
+  char* attn = take(rows * D * e);
+  char* u = take(rows * F * e);
+  char* y = take(rows * D * 4);
+  char* ar = take(rows * ROOT_IN_LD * e);
+  char* ab = take(rows * BODY_IN_LD * e);
+  char* rh = take(nframes * ROOT_F * 4);
+  char* bh = take(nframes * BODY_F * 4);
+  char* x = take(nframes * MOTION_F * 4);
+  char* emb = take(nseq * DTXT * e);
+  char* txt0 = take(nseq * D * 4);
+  char* txt1 = take(nseq * D * 4);
+  char* tpe = take(D * e);
+  char* thid = take(D * e);
+  char* tm0 = take(D * 4);
+  char* tm1 = take(D * 4);
+  char* len = take(nseq * 4);
+  char* stt = take(nseq * DTXT * 4);
+  if (w) {
+    w->h = h; w->qkv = qkv; w->attn = attn; w->u = u; w->y = reinterpret_cast<float*>(y);
+    w->A_root = ar; w->A_body = ab;
+    w->root_hat = reinterpret_cast<float*>(rh); w->body_hat = reinterpret_cast<float*>(bh);
+    w->x = reinterpret_cast<float*>(x); w->emb = emb;
+    w->txt[0] = reinterpret_cast<float*>(txt0); w->txt[1] = reinterpret_cast<float*>(txt1);
+    w->tpe = tpe; w->thid = thid;
+    w->tmlp[0] = reinterpret_cast<float*>(tm0); w->tmlp[1] = reinterpret_cast<float*>(tm1);
+    w->lengths = reinterpret_cast<int*>(len); w->st_text = reinterpret_cast<float*>(stt); w->st_null = nullptr;
+  }
+  return off;
+}
+
+constexpr size_t NOALLOC_BYTES =
+    noalloc_layout(nullptr, 4, NOALLOC_MAX_ROWS, NOALLOC_MAX_BATCH, NOALLOC_MAX_ROWS, nullptr);
+
+}  // namespace
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[NOALLOC_BYTES];
+
+namespace {
+
+// Device address of g_noalloc_scratch on the current device (set-up on first use).
+int noalloc_scratch(char** out) {
+  static void* addr[64] = {};
+  int dev = 0;
+  KD_CUDA(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64) return set_error(KIMODO_EINVAL, "device index %d", dev);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess || !p)
+      return set_error(KIMODO_ECUDA, "cudaGetSymbolAddress of the static scratch failed: %s", cudaGetErrorString(e));
+    addr[dev] = p;
+  }
+  *out = static_cast<char*>(addr[dev]);
+  return KIMODO_OK;
+}
+
+// Restores the context's own workspace and profiling flag on every exit path.
+struct WorkspaceSwap {
+  kimodo_ctx* c;
+  Workspace saved;
+  bool prof;
+  WorkspaceSwap(kimodo_ctx* ctx, const Workspace& w) : c(ctx), saved(ctx->ws), prof(ctx->profiling) {
+    c->ws = w;
+    c->profiling = false;
+  }
+  ~WorkspaceSwap() {
+    c->ws = saved;
+    c->profiling = prof;
+  }
+};
+
+}  // namespace
+
+extern "C" int kimodo_denoiser_forward_noalloc(kimodo_ctx* c, int net, const float* x, const float* emb, int t,
+                                               const int* lengths, int batch, int frames, float* out,
+                                               void* stream) {
+  g_last_error.clear();
+  KD_TRY(check_ctx(c));
+  if (net != KIMODO_NET_ROOT && net != KIMODO_NET_BODY) return set_error(KIMODO_EINVAL, "net must be 0 or 1");
+  if (!x || !emb || !out) return set_error(KIMODO_EINVAL, "NULL tensor argument");
+  if (t < 0 || t >= N_TRAIN) return set_error(KIMODO_EINVAL, "t must be in [0, 999] (got %d)", t);
+  KD_TRY(check_shape(batch, frames));
+  if (batch > NOALLOC_MAX_BATCH || (long)batch * (frames + 1) > NOALLOC_MAX_ROWS)
+    return set_error(KIMODO_EINVAL,
+                     "kimodo_denoiser_forward_noalloc: batch %d x (frames %d + 1) exceeds its static scratch "
+                     "(at most %d sequences and %d tokens); use kimodo_denoiser_forward",
+                     batch, frames, NOALLOC_MAX_BATCH, NOALLOC_MAX_ROWS);
+  char* base = nullptr;
+  KD_TRY(noalloc_scratch(&base));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int rows = batch * (frames + 1);
+  Workspace w;
+  const size_t used = noalloc_layout(base, c->elem(), rows, batch, (size_t)batch * frames, &w);
+  if (used > NOALLOC_BYTES) return set_error(KIMODO_EINVAL, "internal: static scratch layout overflow");
+  WorkspaceSwap swap(c, w);
+  const long long l0 = c->launches;
+  NetW& n = c->net[net];
+  // the scratch keeps the previous call's contents: the zero-padded K columns of
+  // the input matrices must read as 0, so clear both matrices
+  KD_CUDA(cudaMemsetAsync(w.A_root, 0, (size_t)rows * ROOT_IN_LD * c->elem(), st));
+  KD_CUDA(cudaMemsetAsync(w.A_body, 0, (size_t)rows * BODY_IN_LD * c->elem(), st));
+  KD_TRY(stage_lengths(c, lengths, batch, frames, st));
+  KD_CUDA(cudaMemcpyAsync(w.x, x, (size_t)batch * frames * n.din * 4, cudaMemcpyDefault, st));
+  KD_CUDA(cudaMemcpyAsync(w.st_text, emb, (size_t)batch * DTXT * 4, cudaMemcpyDefault, st));
+  KD_TRY(launch(c, CLS_SETUP, 0, (double)batch * DTXT * 6, st, "pack_embeddings", [&] {
+    return pack_embeddings(w.st_text, batch, nullptr, 1, 0, w.emb, c->bf16(), st);
+  }));
+  KD_TRY(timestep_rows(c, t, 1, 1, st));
+  KD_TRY(condition_setup(c, net, batch, 1, st));
+  void* A = net == 0 ? w.A_root : w.A_body;
+  const int lda = net == 0 ? ROOT_IN_LD : BODY_IN_LD;
+  KD_TRY(launch(c, CLS_MOTION, 0, (double)batch * frames * n.din * 8, st, "pack_frames", [&] {
+    return pack_frames(w.x, batch, n.din, 0, n.din, A, c->bf16(), lda, 0, batch, frames, frames + 1, st);
+  }));
+  float* hat = net == 0 ? w.root_hat : w.body_hat;
+  KD_TRY(run_net(c, net, batch, frames, batch, A, w.tmlp[net], w.txt[net], hat, st));
+  KD_CUDA(cudaMemcpyAsync(out, hat, (size_t)batch * frames * n.dout * 4, cudaMemcpyDefault, st));
+  c->last_launches = c->launches - l0;
+  return finish_outputs(c, out, st);
+}
