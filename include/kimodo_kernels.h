@@ -33,6 +33,7 @@ enum {
  * aligned with lda, ldw multiples of 8 and >= K.  bias: fp32 [N].
  * resid: fp32 [M, ldr] (KIMODO_EPI_BIAS_RESID only, else NULL); may equal out.
  * out: bf16 (out_f32 = 0) or fp32 (out_f32 = 1), row stride ldo.
+ * out, resid, bias 16-byte aligned; ldo, ldr multiples of 4.
  * KIMODO_EPI_BIAS_RESID requires out_f32 = 1.  tile_n: 128 or 256 (output
  * columns per tile), or 0 to let the library choose.
  */

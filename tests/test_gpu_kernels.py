@@ -55,8 +55,10 @@ def test_gemm_tcgen05_vs_oracle(M, N, K, lda, epi, out_f32, tile):
     bias = torch.from_numpy(synth.random_vectors((N,), seed + 2, 0.1))
     resid = torch.from_numpy(synth.random_vectors((M, N), seed + 3)) if epi == kb.EPI_BIAS_RESID else None
     dev = "cuda"
+    ldo = (N + 7) // 8 * 8     # output rows padded to a 16-byte multiple
+    buf = torch.empty((M, ldo), dtype=torch.float32 if out_f32 else torch.bfloat16, device=dev)
     out = kb.gemm_bf16(A.to(dev), W.to(dev), bias.to(dev), epi, out_f32,
-                       None if resid is None else resid.to(dev), K=K, tile_n=tile)
+                       None if resid is None else resid.to(dev), out=buf[:, :N], K=K, tile_n=tile)
     torch.cuda.synchronize()
     ref = _epi_ref(epi, ko.linear(_f64(A)[:, :K], _f64(W)[:, :K], bias.double().numpy()),
                    None if resid is None else resid.double().numpy())

@@ -91,6 +91,15 @@ def _ptr(a):
     return a.data_ptr()
 
 
+def _ptr_rows(a):
+    """Data pointer of a row-major 2-D tensor whose rows may be padded (stride(1) == 1)."""
+    if a is None:
+        return None
+    if a.dim() != 2 or a.stride(1) != 1:
+        raise ValueError("need a 2-D tensor with unit column stride")
+    return a.data_ptr()
+
+
 def _is_cuda(a):
     return hasattr(a, "is_cuda") and a.is_cuda
 
@@ -138,8 +147,8 @@ def gemm_bf16(A, W, bias, epilogue=EPI_BIAS, out_f32=False, resid=None, out=None
     K = A.shape[1] if K is None else K
     if out is None:
         out = torch.empty((M, N), dtype=torch.float32 if out_f32 else torch.bfloat16, device=A.device)
-    _check(lib.kimodo_gemm_bf16(_ptr(A), A.stride(0), _ptr(W), W.stride(0), _ptr(bias), _ptr(resid),
-                                0 if resid is None else resid.stride(0), _ptr(out), out.stride(0), M, N, K,
+    _check(lib.kimodo_gemm_bf16(_ptr_rows(A), A.stride(0), _ptr_rows(W), W.stride(0), _ptr(bias), _ptr_rows(resid),
+                                0 if resid is None else resid.stride(0), _ptr_rows(out), out.stride(0), M, N, K,
                                 int(epilogue), int(bool(out_f32)), int(tile_n), _cur_stream()))
     return out
 

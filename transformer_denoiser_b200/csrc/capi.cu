@@ -807,6 +807,9 @@ int kimodo_gemm_bf16(const void* A, int lda, const void* W, int ldw, const float
   KD_TRY(check_gemm_args(A, lda, W, ldw, bias, resid, out, ldo, M, N, K, epilogue));
   if (lda % 8 || ldw % 8 || (reinterpret_cast<uintptr_t>(A) & 15) || (reinterpret_cast<uintptr_t>(W) & 15))
     return set_error(KIMODO_EINVAL, "bf16 operands need 16-byte aligned rows (lda, ldw multiples of 8)");
+  if (ldo % 4 || (reinterpret_cast<uintptr_t>(out) & 15) || (epilogue == 3 && (ldr % 4 ||
+      (reinterpret_cast<uintptr_t>(resid) & 15))) || (reinterpret_cast<uintptr_t>(bias) & 15))
+    return set_error(KIMODO_EINVAL, "out, resid and bias need 16-byte alignment and ldo, ldr multiples of 4");
   if (epilogue == 3 && !out_f32) return set_error(KIMODO_EINVAL, "residual epilogue writes fp32");
   if ((epilogue == 1 || epilogue == 2) && out_f32) return set_error(KIMODO_EINVAL, "GELU/SiLU epilogues write bf16");
   if (tile_n != 0 && tile_n != 128 && tile_n != 256) return set_error(KIMODO_EINVAL, "tile_n must be 0, 128 or 256");

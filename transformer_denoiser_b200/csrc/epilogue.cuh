@@ -123,3 +123,135 @@ __device__ __forceinline__ void epilogue_row(const EpiParams& e, int row, int co
 }
 
 }  // namespace kd
+
+namespace kd {
+
+// ---------------------------------------------------------------------------
+// Coalesced epilogue of the tensor-core GEMM.  A warp owns 32 accumulator rows;
+// after tcgen05.ld each thread holds one row's CW consecutive columns.  The warp
+// writes them to its shared-memory tile st[32][CW + 4] and then walks the rows
+// with lanes along the columns (4 columns per lane), so every global load and
+// store of bias, residual, sinusoid table and output is a contiguous row segment.
+
+template <typename OutT>
+__device__ __forceinline__ void store4(OutT* p, float a, float b, float c, float d);
+template <>
+__device__ __forceinline__ void store4<float>(float* p, float a, float b, float c, float d) {
+  *reinterpret_cast<float4*>(p) = make_float4(a, b, c, d);
+}
+template <>
+__device__ __forceinline__ void store4<bf16>(bf16* p, float a, float b, float c, float d) {
+  __nv_bfloat162 lo = __floats2bfloat162_rn(a, b), hi = __floats2bfloat162_rn(c, d);
+  uint2 u;
+  u.x = *reinterpret_cast<uint32_t*>(&lo);
+  u.y = *reinterpret_cast<uint32_t*>(&hi);
+  *reinterpret_cast<uint2*>(p) = u;
+}
+
+__device__ __forceinline__ float4 ld4(const float* p) { return *reinterpret_cast<const float4*>(p); }
+
+template <int CW>
+struct EpiLanes {
+  static constexpr int LDE = CW + 4;
+  static constexpr int LPR = CW / 4;        // lanes per row
+  static constexpr int RPP = 32 / LPR;      // rows per pass
+  static constexpr int PASSES = 32 / RPP;
+};
+
+// Global operands of one chunk that do not depend on the accumulator (residual
+// rows, sinusoid rows), loaded before the accumulator is read so their latency
+// overlaps the TMEM load.  Rows past M are clamped for the load only.
+template <int KIND, int CW>
+__device__ __forceinline__ void epilogue_prefetch(const EpiParams& e, int row0, int col0, int lane,
+                                                  float4 (&pre)[EpiLanes<CW>::PASSES]) {
+  using Ln = EpiLanes<CW>;
+  const int rsub = lane / Ln::LPR;
+  const int col = col0 + (lane % Ln::LPR) * 4;
+  if constexpr (KIND == EPI_BIAS_RESID || KIND == EPI_INPROJ) {
+    if (col + 4 > e.N) return;
+#pragma unroll
+    for (int p = 0; p < Ln::PASSES; ++p) {
+      const int row = min(row0 + p * Ln::RPP + rsub, e.M - 1);
+      if constexpr (KIND == EPI_BIAS_RESID) {
+        pre[p] = ld4(reinterpret_cast<const float*>(e.resid) + (long)row * e.ldr + col);
+      } else {
+        const int pos = row % e.S;
+        pre[p] = ld4(e.pe + (long)pos * e.N + col);
+      }
+    }
+  }
+}
+
+template <int KIND, typename OutT, int CW>
+__device__ __forceinline__ void epilogue_warp_tile(const EpiParams& e, const float* st, int row0, int col0,
+                                                   int lane, const float4 (&pre)[EpiLanes<CW>::PASSES]) {
+  using Ln = EpiLanes<CW>;
+  const int rsub = lane / Ln::LPR;
+  const int cq = (lane % Ln::LPR) * 4;
+  const int col = col0 + cq;
+  if (col >= e.N) return;
+  const bool full = col + 4 <= e.N;  // all 4 columns valid (N % 4 != 0 only at the output projection)
+  float b4[4] = {0.f, 0.f, 0.f, 0.f};
+  if (full) {
+    const float4 t = ld4(e.bias + col);
+    b4[0] = t.x; b4[1] = t.y; b4[2] = t.z; b4[3] = t.w;
+  } else {
+    for (int j = 0; j < 4; ++j) b4[j] = col + j < e.N ? e.bias[col + j] : 0.f;
+  }
+#pragma unroll
+  for (int p = 0; p < Ln::PASSES; ++p) {
+    const int r = p * Ln::RPP + rsub;
+    const int row = row0 + r;
+    const bool in_rows = row < e.M;
+    const float4 a = *reinterpret_cast<const float4*>(st + r * Ln::LDE + cq);
+    float v[4] = {a.x, a.y, a.z, a.w};
+    if constexpr (KIND == EPI_OUTPROJ) {
+      const int seq = row / e.S, pos = row - seq * e.S;
+      if (in_rows && pos != 0) {
+        const int frame = pos - 1;
+        const bool valid = frame < e.lengths[seq % e.len_mod];
+        OutT* o = reinterpret_cast<OutT*>(e.out) + ((long)seq * e.T + frame) * e.ldo + col;
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          if (col + j < e.N) o[j] = from_f<OutT>(valid ? v[j] + b4[j] : 0.f);
+      }
+    } else {
+      if constexpr (KIND == EPI_INPROJ) {
+        const int seq = row / e.S, pos = row - seq * e.S;
+        if (pos == 0) {
+          const float4 cv = ld4(e.cond + (long)seq * e.N + col);
+          const float4 tv = ld4(e.tvec + col);
+          const float4 pv = ld4(e.pe + col);
+          v[0] = cv.x + tv.x + pv.x; v[1] = cv.y + tv.y + pv.y;
+          v[2] = cv.z + tv.z + pv.z; v[3] = cv.w + tv.w + pv.w;
+        } else {
+          const float4 pv = pre[p];
+          v[0] += b4[0] + pv.x; v[1] += b4[1] + pv.y; v[2] += b4[2] + pv.z; v[3] += b4[3] + pv.w;
+        }
+        if (in_rows && e.out32 != nullptr) store4<float>(e.out32 + (long)row * e.ldo + col, v[0], v[1], v[2], v[3]);
+      } else {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          float x = v[j] + b4[j];
+          if constexpr (KIND == EPI_BIAS_GELU) x = gelu_erf(x);
+          if constexpr (KIND == EPI_BIAS_SILU) x = silu_f(x);
+          v[j] = x;
+        }
+        if constexpr (KIND == EPI_BIAS_RESID) {
+          v[0] += pre[p].x; v[1] += pre[p].y; v[2] += pre[p].z; v[3] += pre[p].w;
+        }
+      }
+      if (in_rows) {
+        OutT* o = reinterpret_cast<OutT*>(e.out) + (long)row * e.ldo + col;
+        if (full) {
+          store4<OutT>(o, v[0], v[1], v[2], v[3]);
+        } else {
+          for (int j = 0; j < 4; ++j)
+            if (col + j < e.N) o[j] = from_f<OutT>(v[j]);
+        }
+      }
+    }
+  }
+}
+
+}  // namespace kd

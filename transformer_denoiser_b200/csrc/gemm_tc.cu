@@ -47,7 +47,9 @@ struct TcCfg {
   static constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr uint32_t TMEM_COLS = tmem_cols_for(2 * BN);
   static constexpr uint32_t NUM_BARS = 2 * STAGES + 5;
-  static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE_BYTES + NUM_BARS * 8 + 16;
+  static constexpr int CW = BN < 32 ? BN : 32;                 // epilogue chunk: columns per tcgen05.ld
+  static constexpr uint32_t EPI_BYTES = 4 * 32 * (CW + 4) * 4;  // one staging tile per epilogue warp
+  static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE_BYTES + EPI_BYTES + NUM_BARS * 8 + 16;
   static constexpr uint32_t IDESC = ptx::idesc_bf16_f32(BM, BN);
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "UMMA N for M=128");
   static_assert(SMEM <= 232448, "shared memory");
@@ -70,7 +72,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sA = ptx::smem_u32(smem);
   const uint32_t sB = sA + STAGES * C::A_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * C::STAGE_BYTES);
+  float* epi_smem = reinterpret_cast<float*>(smem + STAGES * C::STAGE_BYTES);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * C::STAGE_BYTES + C::EPI_BYTES);
   const uint32_t bar0 = ptx::smem_u32(bars);
   auto full_bar = [&](int s) { return bar0 + 8u * s; };
   auto empty_bar = [&](int s) { return bar0 + 8u * (STAGES + s); };
@@ -203,20 +206,32 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       }
       ptx::tc_fence_after();
       const int m_blk = tile % num_m_tiles, n_blk = tile / num_m_tiles;
-      const int row = m_blk * BM + quarter * 32 + lane;
+      const int row0 = m_blk * BM + quarter * 32;
       const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * BN;
+      constexpr int CW = C::CW;
+      float* st = epi_smem + quarter * 32 * (CW + 4);
+      // chunks that hold at least one valid output column
+      const int valid_cols = min(BN, ep.N - n_blk * BN);
+      const int nchunks = (valid_cols + CW - 1) / CW;
 #pragma unroll 1
-      for (int c = 0; c < BN / 16; ++c) {
-        float v[16];
-        ptx::tmem_ld16(taddr + c * 16, v);
+      for (int c = 0; c < nchunks; ++c) {
+        float4 pre[EpiLanes<CW>::PASSES];
+        epilogue_prefetch<KIND, CW>(ep, row0, n_blk * BN + c * CW, lane, pre);
+        float v[CW];
+        ptx::tmem_ld(taddr + c * CW, v);
         ptx::tmem_ld_wait();
-        if (c == BN / 16 - 1) {
+        if (c == nchunks - 1) {
+          // accumulator fully read: hand it back to the MMA warp
           ptx::tc_fence_before();
           __syncwarp();
           if (lane == 0) ptx::mbar_arrive(tempty_bar(acc));
         }
-        const int col0 = n_blk * BN + c * 16;
-        if (col0 < ep.N) epilogue_row<KIND, OutT, ResT, 16>(ep, row, col0, v);
+#pragma unroll
+        for (int j = 0; j < CW; j += 4)
+          *reinterpret_cast<float4*>(st + lane * (CW + 4) + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+        __syncwarp();
+        epilogue_warp_tile<KIND, OutT, CW>(ep, st, row0, n_blk * BN + c * CW, lane, pre);
+        __syncwarp();
       }
     }
   }
