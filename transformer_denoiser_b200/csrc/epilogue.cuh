@@ -163,10 +163,18 @@ struct EpiLanes {
 // overlaps the TMEM load.  Rows past M are clamped for the load only.
 template <int KIND, int CW>
 __device__ __forceinline__ void epilogue_prefetch(const EpiParams& e, int row0, int col0, int lane,
-                                                  float4 (&pre)[EpiLanes<CW>::PASSES]) {
+                                                  float4 (&pre)[EpiLanes<CW>::PASSES], float4& bias4) {
   using Ln = EpiLanes<CW>;
   const int rsub = lane / Ln::LPR;
   const int col = col0 + (lane % Ln::LPR) * 4;
+  if (col + 4 <= e.N) {
+    bias4 = ld4(e.bias + col);
+  } else {
+    bias4.x = col < e.N ? e.bias[col] : 0.f;
+    bias4.y = col + 1 < e.N ? e.bias[col + 1] : 0.f;
+    bias4.z = col + 2 < e.N ? e.bias[col + 2] : 0.f;
+    bias4.w = col + 3 < e.N ? e.bias[col + 3] : 0.f;
+  }
   if constexpr (KIND == EPI_BIAS_RESID || KIND == EPI_INPROJ) {
     if (col + 4 > e.N) return;
 #pragma unroll
@@ -184,20 +192,15 @@ __device__ __forceinline__ void epilogue_prefetch(const EpiParams& e, int row0, 
 
 template <int KIND, typename OutT, int CW>
 __device__ __forceinline__ void epilogue_warp_tile(const EpiParams& e, const float* st, int row0, int col0,
-                                                   int lane, const float4 (&pre)[EpiLanes<CW>::PASSES]) {
+                                                   int lane, const float4 (&pre)[EpiLanes<CW>::PASSES],
+                                                   const float4 bias4) {
   using Ln = EpiLanes<CW>;
   const int rsub = lane / Ln::LPR;
   const int cq = (lane % Ln::LPR) * 4;
   const int col = col0 + cq;
   if (col >= e.N) return;
   const bool full = col + 4 <= e.N;  // all 4 columns valid (N % 4 != 0 only at the output projection)
-  float b4[4] = {0.f, 0.f, 0.f, 0.f};
-  if (full) {
-    const float4 t = ld4(e.bias + col);
-    b4[0] = t.x; b4[1] = t.y; b4[2] = t.z; b4[3] = t.w;
-  } else {
-    for (int j = 0; j < 4; ++j) b4[j] = col + j < e.N ? e.bias[col + j] : 0.f;
-  }
+  const float b4[4] = {bias4.x, bias4.y, bias4.z, bias4.w};
 #pragma unroll
   for (int p = 0; p < Ln::PASSES; ++p) {
     const int r = p * Ln::RPP + rsub;

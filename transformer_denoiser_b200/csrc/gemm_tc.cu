@@ -32,7 +32,9 @@ namespace {
 
 constexpr int BM = 128;
 constexpr int BK = 64;                       // 64 bf16 = one 128-byte swizzle row
-constexpr int NUM_THREADS = 192;
+constexpr int EPI_WARPS = 8;                 // two per TMEM lane quarter, splitting the columns
+constexpr int EPI_PARTS = EPI_WARPS / 4;
+constexpr int NUM_THREADS = 64 + 32 * EPI_WARPS;
 constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;
 constexpr int KIMODO_ETIMEOUT_CODE = -5;
 
@@ -47,8 +49,9 @@ struct TcCfg {
   static constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr uint32_t TMEM_COLS = tmem_cols_for(2 * BN);
   static constexpr uint32_t NUM_BARS = 2 * STAGES + 5;
-  static constexpr int CW = BN < 32 ? BN : 32;                 // epilogue chunk: columns per tcgen05.ld
-  static constexpr uint32_t EPI_BYTES = 4 * 32 * (CW + 4) * 4;  // one staging tile per epilogue warp
+  static constexpr int CW = 16;                                        // epilogue chunk: columns per tcgen05.ld
+  static constexpr int WCOLS = BN / EPI_PARTS >= 16 ? BN / EPI_PARTS : 16;  // columns per epilogue warp
+  static constexpr uint32_t EPI_BYTES = EPI_WARPS * 32 * (CW + 4) * 4;  // one staging tile per epilogue warp
   static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE_BYTES + EPI_BYTES + NUM_BARS * 8 + 16;
   static constexpr uint32_t IDESC = ptx::idesc_bf16_f32(BM, BN);
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "UMMA N for M=128");
@@ -98,7 +101,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     }
     for (int a = 0; a < 2; ++a) {
       ptx::mbar_init(tfull_bar(a), 1);
-      ptx::mbar_init(tempty_bar(a), 4);
+      ptx::mbar_init(tempty_bar(a), EPI_WARPS);
     }
     ptx::mbar_init(drain_bar, 1);
     ptx::fence_mbar_init();
@@ -194,8 +197,13 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       if (!ptx::mbar_wait_bounded(drain_bar, 0, &never, WAIT_LIMIT_NS)) record_timeout(err, WHERE_GEMM_DRAIN, abort);
     }
   } else {
-    // ---------------- epilogue warps 2..5: TMEM lane quarter = warp % 4
+    // ---------------- epilogue warps 2..(1 + EPI_WARPS): TMEM lane quarter = warp % 4; part (warp - 2) / 4
+    // takes columns [part * WCOLS, (part + 1) * WCOLS) of the tile (parts past BN idle)
     const int quarter = warp & 3;
+    const int part = (warp - 2) >> 2;
+    constexpr int CW = C::CW;
+    constexpr int PASSES = EpiLanes<CW>::PASSES;
+    float* st = epi_smem + (warp - 2) * 32 * (CW + 4);
     int local = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++local) {
       const int acc = local & 1;
@@ -207,31 +215,57 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       ptx::tc_fence_after();
       const int m_blk = tile % num_m_tiles, n_blk = tile / num_m_tiles;
       const int row0 = m_blk * BM + quarter * 32;
-      const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * BN;
-      constexpr int CW = C::CW;
-      float* st = epi_smem + quarter * 32 * (CW + 4);
-      // chunks that hold at least one valid output column
-      const int valid_cols = min(BN, ep.N - n_blk * BN);
-      const int nchunks = (valid_cols + CW - 1) / CW;
-#pragma unroll 1
-      for (int c = 0; c < nchunks; ++c) {
-        float4 pre[EpiLanes<CW>::PASSES];
-        epilogue_prefetch<KIND, CW>(ep, row0, n_blk * BN + c * CW, lane, pre);
-        float v[CW];
-        ptx::tmem_ld(taddr + c * CW, v);
-        ptx::tmem_ld_wait();
-        if (c == nchunks - 1) {
-          // accumulator fully read: hand it back to the MMA warp
-          ptx::tc_fence_before();
-          __syncwarp();
-          if (lane == 0) ptx::mbar_arrive(tempty_bar(acc));
-        }
+      const int cbeg = min(part * C::WCOLS, BN);
+      const int cend = min(cbeg + C::WCOLS, BN);
+      const int valid_end = min(cend, ep.N - n_blk * BN);
+      const int nch = valid_end > cbeg ? (valid_end - cbeg + CW - 1) / CW : 0;
+      const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * BN + cbeg;
+      const int gcol = n_blk * BN + cbeg;
+      if (nch == 0) {
+        ptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(tempty_bar(acc));
+        continue;
+      }
+      // two register buffers: the TMEM load and global prefetch of chunk c + 1 are in
+      // flight while chunk c is transposed and stored
+      float va[CW], vb[CW];
+      float4 pa[PASSES], pb[PASSES];
+      float4 ba, bb;
+      auto process = [&](float (&v)[CW], const float4 (&pre)[PASSES], const float4 bias4, int c) {
 #pragma unroll
         for (int j = 0; j < CW; j += 4)
           *reinterpret_cast<float4*>(st + lane * (CW + 4) + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
         __syncwarp();
-        epilogue_warp_tile<KIND, OutT, CW>(ep, st, row0, n_blk * BN + c * CW, lane, pre);
+        epilogue_warp_tile<KIND, OutT, CW>(ep, st, row0, gcol + c * CW, lane, pre, bias4);
         __syncwarp();
+      };
+      auto release_if_last = [&](int c) {
+        if (c == nch - 1) {
+          ptx::tc_fence_before();
+          __syncwarp();
+          if (lane == 0) ptx::mbar_arrive(tempty_bar(acc));
+        }
+      };
+      epilogue_prefetch<KIND, CW>(ep, row0, gcol, lane, pa, ba);
+      ptx::tmem_ld(taddr, va);
+#pragma unroll 1
+      for (int c = 0; c < nch; c += 2) {
+        ptx::tmem_ld_wait();
+        release_if_last(c);
+        if (c + 1 < nch) {
+          epilogue_prefetch<KIND, CW>(ep, row0, gcol + (c + 1) * CW, lane, pb, bb);
+          ptx::tmem_ld(taddr + (c + 1) * CW, vb);
+        }
+        process(va, pa, ba, c);
+        if (c + 1 >= nch) break;
+        ptx::tmem_ld_wait();
+        release_if_last(c + 1);
+        if (c + 2 < nch) {
+          epilogue_prefetch<KIND, CW>(ep, row0, gcol + (c + 2) * CW, lane, pa, ba);
+          ptx::tmem_ld(taddr + (c + 2) * CW, va);
+        }
+        process(vb, pb, bb, c + 1);
       }
     }
   }
