@@ -41,6 +41,17 @@ KIMODO_API int kimodo_gemm_bf16(const void* A, int lda, const void* W, int ldw, 
                                 const void* resid, int ldr, void* out, int ldo, int M, int N, int K,
                                 int epilogue, int out_f32, int tile_n, void* stream);
 
+/*
+ * The same product on pairs of SMs (one 256-row output tile per CTA pair,
+ * tcgen05 cta_group::2), the kernel the denoiser uses for its large projections.
+ * Arguments as kimodo_gemm_bf16; epilogues KIMODO_EPI_BIAS and KIMODO_EPI_BIAS_GELU
+ * with bf16 output and KIMODO_EPI_BIAS_RESID with fp32 output.  tile_n: output
+ * columns per pair tile, 144, 160, 208 or 256, or 0 for the library's choice.
+ */
+KIMODO_API int kimodo_gemm_bf16_pair(const void* A, int lda, const void* W, int ldw, const float* bias,
+                                     const void* resid, int ldr, void* out, int ldo, int M, int N, int K,
+                                     int epilogue, int out_f32, int tile_n, void* stream);
+
 /* fp32 SIMT GEMM with the same epilogues; all operands fp32; K % 16 == 0,
  * lda, ldw multiples of 4. */
 KIMODO_API int kimodo_gemm_f32(const float* A, int lda, const float* W, int ldw, const float* bias,

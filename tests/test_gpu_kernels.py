@@ -70,6 +70,39 @@ def test_gemm_tcgen05_vs_oracle(M, N, K, lda, epi, out_f32, tile):
         np.testing.assert_allclose(got, ref, rtol=2 ** -8, atol=1e-5 * scale)
 
 
+PAIR_CASES = [
+    # M, N, K, epilogue, out_f32, tile_n (CTA-pair kernel: 256-row tiles)
+    (4832, 3072, 1024, kb.EPI_BIAS, False, 208),
+    (4832, 3072, 1024, kb.EPI_BIAS, False, 256),
+    (4832, 2048, 1024, kb.EPI_BIAS_GELU, False, 144),
+    (4832, 1024, 1024, kb.EPI_BIAS_RESID, True, 160),
+    (4832, 1024, 2048, kb.EPI_BIAS_RESID, True, 208),
+    (300, 1024, 1024, kb.EPI_BIAS, False, 160),           # second CTA of the last pair tile fully out of range
+    (1283, 2048, 1024, kb.EPI_BIAS_GELU, False, 256),
+]
+
+
+@pytest.mark.parametrize("M,N,K,epi,out_f32,tile", PAIR_CASES)
+def test_gemm_tcgen05_pair_vs_oracle(M, N, K, epi, out_f32, tile):
+    require_cuda()
+    seed = M * 5 + N * 7 + K + tile
+    A = _bf16(synth.random_vectors((M, K), seed))
+    W = _bf16(synth.random_vectors((N, K), seed + 1, 0.05))
+    bias = torch.from_numpy(synth.random_vectors((N,), seed + 2, 0.1))
+    resid = torch.from_numpy(synth.random_vectors((M, N), seed + 3)) if epi == kb.EPI_BIAS_RESID else None
+    out = kb.gemm_bf16(A.cuda(), W.cuda(), bias.cuda(), epi, out_f32, None if resid is None else resid.cuda(),
+                       tile_n=tile, pair=True)
+    torch.cuda.synchronize()
+    ref = _epi_ref(epi, ko.linear(_f64(A), _f64(W), bias.double().numpy()),
+                   None if resid is None else resid.double().numpy())
+    got = out.float().cpu().double().numpy()
+    scale = np.abs(ref).max()
+    if out_f32:
+        np.testing.assert_allclose(got, ref, rtol=0, atol=2e-5 * scale)
+    else:
+        np.testing.assert_allclose(got, ref, rtol=2 ** -8, atol=1e-5 * scale)
+
+
 def test_gemm_residual_in_place():
     """The residual epilogue may read and write the same fp32 buffer."""
     require_cuda()
@@ -98,6 +131,26 @@ def test_gemm_f32_vs_oracle(M, N, K, epi):
     ref = _epi_ref(epi, ko.linear(A.double().numpy(), W.double().numpy(), bias.double().numpy()),
                    None if resid is None else resid.double().numpy())
     np.testing.assert_allclose(out.cpu().double().numpy(), ref, rtol=0, atol=2e-6 * np.abs(ref).max())
+
+
+def test_gelu_epilogue_error_bound():
+    """GELU of the epilogues against the exact erf GELU on a dense grid.  The erf
+    approximation (Abramowitz & Stegun 7.1.26) is within 1.5e-7 of erf; evaluating
+    1 - p(t) exp(-z^2) in fp32 adds up to 2 ulp of 1.0 (2.4e-7), so
+    |GELU error| <= 0.5 |x| (1.5e-7 + 2.4e-7) plus the fp32 rounding of the result."""
+    require_cuda()
+    x = np.linspace(-9, 9, 4096).astype(np.float32)
+    A = np.zeros((x.size, 16), np.float32)
+    A[:, 0] = x
+    W = np.zeros((16, 16), np.float32)
+    W[0, 0] = 1.0
+    out = kb.gemm_f32(torch.from_numpy(A).cuda(), torch.from_numpy(W).cuda(), torch.zeros(16, device="cuda"),
+                      kb.EPI_BIAS_GELU)
+    got = out[:, 0].cpu().double().numpy()
+    ref = ko.gelu(x.astype(np.float64))
+    bound = 0.5 * np.abs(x) * (1.5e-7 + 2 * np.finfo(np.float32).eps) \
+        + 4 * np.finfo(np.float32).eps * np.maximum(np.abs(ref), 1e-3)
+    assert np.all(np.abs(got - ref) <= bound), float(np.max(np.abs(got - ref) - bound))
 
 
 def _attention_ref(qkv, lengths, S):

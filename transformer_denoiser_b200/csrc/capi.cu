@@ -13,6 +13,7 @@
 #include <math.h>
 #include <stdarg.h>
 #include <stdio.h>
+#include <stdlib.h>
 #include <string.h>
 
 #include <map>
@@ -104,6 +105,7 @@ struct kimodo_ctx {
   size_t ev_used = 0;
   long long launches = 0;
   long long last_launches = 0;
+  bool pair_gemm = true;   // 256-row CTA-pair GEMM tiles for the large projections (KIMODO_PAIR_GEMM=0 disables)
   bool bf16() const { return precision == KIMODO_BF16; }
   size_t elem() const { return bf16() ? 2 : 4; }
 };
@@ -160,6 +162,11 @@ int gemm(kimodo_ctx* c, const void* A, int lda, const void* W, int ldw, int M, i
                        (double)M * N * (out_f32 ? 4.0 : (double)c->elem()) +
                        (kind == EPI_BIAS_RESID ? (double)M * N * 4.0 : 0.0);
   if (c->bf16()) {
+    if (c->pair_gemm && M >= 1024 && N >= 256 && gemm_tc2_supports(kind, out_f32)) {
+      const int bn = gemm_tc2_pick_bn(M, N);
+      return launch(c, cls_override >= 0 ? cls_override : CLS_GEMM_TC, flops, bytes, st, "gemm_tc2",
+                    [&] { return gemm_tc2(g, bn, kind, out_f32, ep, c->derr, st); });
+    }
     const int bn = pick_bn(c, M, N);
     return launch(c, cls_override >= 0 ? cls_override : CLS_GEMM_TC, flops, bytes, st, "gemm_tc",
                   [&] { return gemm_tc(g, bn, kind, out_f32, ep, c->derr, st, c->num_sms); });
@@ -497,13 +504,14 @@ int kimodo_load_weights(kimodo_ctx** out_ctx, const float* host_blob, size_t n_f
   if (precision == KIMODO_BF16 && !gemm_tc_available())
     return set_error(KIMODO_EUNSUPPORTED, "cuTensorMapEncodeTiled is unavailable in this driver");
 
-  if (gemm_tc_prepare() != cudaSuccess || attention_prepare() != cudaSuccess) {
+  if (gemm_tc_prepare() != cudaSuccess || gemm_tc2_prepare() != cudaSuccess || attention_prepare() != cudaSuccess) {
     cudaGetLastError();
     return set_error(KIMODO_EUNSUPPORTED, "kernel attributes could not be set on device %d", device);
   }
   kimodo_ctx* c = new kimodo_ctx();
   c->device = device;
   c->precision = precision;
+  if (const char* ev = getenv("KIMODO_PAIR_GEMM")) c->pair_gemm = ev[0] != '0';
   c->num_sms = prop.multiProcessorCount;
   auto fail = [&](int code) {
     kimodo_free(c);
@@ -781,6 +789,7 @@ int prepared_device() {
   if (dev < 0 || dev >= 64) return set_error(KIMODO_EINVAL, "device index");
   if (!done[dev]) {
     KD_CUDA(gemm_tc_prepare());
+    KD_CUDA(gemm_tc2_prepare());
     KD_CUDA(attention_prepare());
     done[dev] = true;
   }
@@ -825,6 +834,30 @@ int kimodo_gemm_bf16(const void* A, int lda, const void* W, int ldw, const float
   ep.bias = bias; ep.out = out; ep.ldo = ldo; ep.resid = resid; ep.ldr = ldr; ep.N = N; ep.M = M;
   const int bn = tile_n ? tile_n : 128;
   KD_CUDA(gemm_tc(g, bn, epilogue, out_f32 != 0, ep, kernel_error_word(), static_cast<cudaStream_t>(stream), sms));
+  return KIMODO_OK;
+}
+
+int kimodo_gemm_bf16_pair(const void* A, int lda, const void* W, int ldw, const float* bias, const void* resid,
+                          int ldr, void* out, int ldo, int M, int N, int K, int epilogue, int out_f32, int tile_n,
+                          void* stream) {
+  g_last_error.clear();
+  KD_TRY(check_gemm_args(A, lda, W, ldw, bias, resid, out, ldo, M, N, K, epilogue));
+  if (lda % 8 || ldw % 8 || (reinterpret_cast<uintptr_t>(A) & 15) || (reinterpret_cast<uintptr_t>(W) & 15))
+    return set_error(KIMODO_EINVAL, "bf16 operands need 16-byte aligned rows (lda, ldw multiples of 8)");
+  if (ldo % 4 || (reinterpret_cast<uintptr_t>(out) & 15) || (epilogue == 3 && (ldr % 4 ||
+      (reinterpret_cast<uintptr_t>(resid) & 15))) || (reinterpret_cast<uintptr_t>(bias) & 15))
+    return set_error(KIMODO_EINVAL, "out, resid and bias need 16-byte alignment and ldo, ldr multiples of 4");
+  if (!gemm_tc2_supports(epilogue, out_f32 != 0))
+    return set_error(KIMODO_EINVAL, "pair GEMM epilogues: bias or GELU with bf16 output, residual with fp32 output");
+  if (tile_n != 0 && tile_n != 144 && tile_n != 160 && tile_n != 208 && tile_n != 256)
+    return set_error(KIMODO_EINVAL, "tile_n must be 0, 144, 160, 208 or 256");
+  KD_TRY(prepared_device());
+  GemmArgs g;
+  g.A = A; g.B = W; g.M = M; g.N = N; g.K = K; g.lda = lda; g.ldb = ldw;
+  EpiParams ep;
+  ep.bias = bias; ep.out = out; ep.ldo = ldo; ep.resid = resid; ep.ldr = ldr; ep.N = N; ep.M = M;
+  const int bn = tile_n ? tile_n : gemm_tc2_pick_bn(M, N);
+  KD_CUDA(gemm_tc2(g, bn, epilogue, out_f32 != 0, ep, kernel_error_word(), static_cast<cudaStream_t>(stream)));
   return KIMODO_OK;
 }
 

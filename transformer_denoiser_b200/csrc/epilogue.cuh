@@ -37,8 +37,25 @@ struct EpiParams {
   int M = 0;                     // valid rows
 };
 
+// erf by Abramowitz & Stegun, Handbook of Mathematical Functions, formula 7.1.26:
+// erf(z) = 1 - (a1 t + a2 t^2 + a3 t^3 + a4 t^4 + a5 t^5) exp(-z^2), t = 1 / (1 + p z),
+// z >= 0, absolute error <= 1.5e-7; erf is odd.  Cheaper than a full-precision erf
+// and far below the bf16 rounding of the GELU output (and the fp32 path's 1e-4).
+__device__ __forceinline__ float erf_as7126(float z) {
+  const float a = fabsf(z);
+  const float t = __fdividef(1.0f, fmaf(0.3275911f, a, 1.0f));
+  float p = fmaf(1.061405429f, t, -1.453152027f);
+  p = fmaf(p, t, 1.421413741f);
+  p = fmaf(p, t, -0.284496736f);
+  p = fmaf(p, t, 0.254829592f);
+  const float e = exp2f(-a * a * 1.4426950408889634f);
+  const float r = fmaf(-p * t, e, 1.0f);
+  return copysignf(r, z);
+}
+
+// GELU(x) = x Phi(x) = 0.5 x (1 + erf(x / sqrt 2)) (the exact, erf-based GELU).
 __device__ __forceinline__ float gelu_erf(float x) {
-  return 0.5f * x * (1.0f + erff(x * 0.70710678118654752f));
+  return 0.5f * x * (1.0f + erf_as7126(x * 0.70710678118654752f));
 }
 __device__ __forceinline__ float silu_f(float x) { return x / (1.0f + expf(-x)); }
 

@@ -298,8 +298,28 @@ EncodeTiledFn get_encode_fn() {
   return fn;
 }
 
+template <int BN, int STAGES, int KIND, typename OutT, typename ResT>
+cudaError_t launch_impl(const GemmArgs& g, const EpiParams& ep, DevError* err, cudaStream_t st, int num_sms,
+                        bool prepare_only) {
+  using Cf = TcCfg<BN, STAGES>;
+  auto kern = gemm_tc_kernel<BN, STAGES, KIND, OutT, ResT>;
+  if (prepare_only)
+    return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cf::SMEM);
+  CUtensorMap ta, tb;
+  if (make_tmap_bf16(&ta, g.A, g.M, g.K, g.lda, BM) || make_tmap_bf16(&tb, g.B, g.N, g.K, g.ldb, BN))
+    return cudaErrorInvalidValue;
+  const int mt = (g.M + BM - 1) / BM, nt = (g.N + BN - 1) / BN;
+  const int tiles = mt * nt;
+  const int grid = tiles < num_sms ? tiles : num_sms;
+  const int kb = (g.K + BK - 1) / BK;
+  kern<<<grid, NUM_THREADS, Cf::SMEM, st>>>(ta, tb, mt, nt, kb, ep, err);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
 // Row-major bf16 matrix [rows, ld] whose first `cols` columns are the K extent.
-int make_tmap(CUtensorMap* m, const void* base, int rows, int cols, int ld, int box_rows) {
+int make_tmap_bf16(CUtensorMap* m, const void* base, int rows, int cols, int ld, int box_rows) {
   EncodeTiledFn enc = get_encode_fn();
   if (!enc) return -1;
   if ((reinterpret_cast<uintptr_t>(base) & 15) || (ld * 2) % 16) return -2;
@@ -313,25 +333,6 @@ int make_tmap(CUtensorMap* m, const void* base, int rows, int cols, int ld, int 
   return r == CUDA_SUCCESS ? 0 : -3;
 }
 
-template <int BN, int STAGES, int KIND, typename OutT, typename ResT>
-cudaError_t launch_impl(const GemmArgs& g, const EpiParams& ep, DevError* err, cudaStream_t st, int num_sms,
-                        bool prepare_only) {
-  using Cf = TcCfg<BN, STAGES>;
-  auto kern = gemm_tc_kernel<BN, STAGES, KIND, OutT, ResT>;
-  if (prepare_only)
-    return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cf::SMEM);
-  CUtensorMap ta, tb;
-  if (make_tmap(&ta, g.A, g.M, g.K, g.lda, BM) || make_tmap(&tb, g.B, g.N, g.K, g.ldb, BN))
-    return cudaErrorInvalidValue;
-  const int mt = (g.M + BM - 1) / BM, nt = (g.N + BN - 1) / BN;
-  const int tiles = mt * nt;
-  const int grid = tiles < num_sms ? tiles : num_sms;
-  const int kb = (g.K + BK - 1) / BK;
-  kern<<<grid, NUM_THREADS, Cf::SMEM, st>>>(ta, tb, mt, nt, kb, ep, err);
-  return cudaGetLastError();
-}
-
-}  // namespace
 
 // Dispatch on (tile N, epilogue kind, output type).  The residual is fp32 (the
 // residual stream of the post-norm layers is kept in fp32; operands are bf16).

@@ -1,0 +1,403 @@
+// Tensor-core GEMM on SM pairs (tcgen05 cta_group::2) for the large per-layer
+// projections: D[M,N] = A[M,K] . B[N,K]^T + fused epilogue, bf16 in, fp32 accumulate.
+//
+// A cluster of two CTAs computes a 256 x BN output tile.  Each CTA stages its own
+// 128 rows of A and BN/2 rows of B (TMA, 128-byte swizzle, no multicast) into the
+// same shared-memory offsets; the pair's leader (cluster rank 0) issues one
+// 256 x BN x 16 MMA per K step that reads both CTAs' shared memory and writes
+// each CTA's 128 accumulator rows into its own TMEM.  Per SM this halves the B
+// traffic of a 128 x BN single-CTA tile.
+//
+// Roles (320 threads per CTA): warp 0 = TMA producer (both CTAs; completions are
+// counted on the leader's "full" barriers), warp 1 = TMEM allocation and, in the
+// leader, the MMA issuer, warps 2-9 = epilogue (two per TMEM lane quarter).  The
+// leader's MMA commits arrive on both CTAs' "empty" and "accumulator full" barriers
+// (tcgen05.commit multicast); both CTAs' epilogues release the accumulator on the
+// leader's "accumulator empty" barrier.  Two TMEM accumulators per CTA.  Every
+// wait is bounded; a timeout is recorded in the device error word.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <type_traits>
+
+#include "common.cuh"
+#include "epilogue.cuh"
+#include "kernels.h"
+#include "ptx.cuh"
+
+namespace kd {
+namespace {
+
+constexpr int BMC = 128;                     // rows per CTA (256 per pair)
+constexpr int BK = 64;
+constexpr int EPI_WARPS = 8;
+constexpr int NUM_THREADS = 64 + 32 * EPI_WARPS;
+constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;
+constexpr int KIMODO_ETIMEOUT_CODE = -5;
+
+constexpr uint32_t tmem_cols_for(uint32_t n) {
+  return n <= 32 ? 32 : n <= 64 ? 64 : n <= 128 ? 128 : n <= 256 ? 256 : 512;
+}
+
+template <int BN, int STAGES>
+struct Tc2Cfg {
+  static constexpr uint32_t A_BYTES = BMC * BK * 2;
+  static constexpr uint32_t B_BYTES = (BN / 2) * BK * 2;
+  static constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr uint32_t TMEM_COLS = tmem_cols_for(2 * BN);
+  static constexpr int CW = 16;
+  static constexpr int NCH = BN / CW;
+  static constexpr int PART_CH = (NCH + 1) / 2;
+  static constexpr uint32_t EPI_BYTES = EPI_WARPS * 32 * (CW + 4) * 4;
+  static constexpr uint32_t NUM_BARS = 2 * STAGES + 5;
+  static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE_BYTES + EPI_BYTES + NUM_BARS * 8 + 16;
+  static constexpr uint32_t IDESC = ptx::idesc_bf16_f32(2 * BMC, BN);
+  static_assert(BN % 16 == 0 && BN >= 32 && BN <= 256, "UMMA N for M=256");
+  static_assert((BN / 2) % 8 == 0, "B half-tile rows must fill 8-row swizzle atoms");
+  static_assert(SMEM <= 232448, "shared memory");
+};
+
+__device__ __forceinline__ void record_timeout(DevError* err, int where, volatile int* abort) {
+  *abort = 1;
+  if (err && atomicCAS(&err->code, 0, KIMODO_ETIMEOUT_CODE) == 0) {
+    err->where = where;
+    err->block = blockIdx.x;
+  }
+}
+
+template <int BN, int STAGES, int KIND, typename OutT>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                int num_m_tiles, int num_n_tiles, int num_kb, EpiParams ep, DevError* err) {
+  using C = Tc2Cfg<BN, STAGES>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sA = ptx::smem_u32(smem);
+  const uint32_t sB = sA + STAGES * C::A_BYTES;
+  float* epi_smem = reinterpret_cast<float*>(smem + STAGES * C::STAGE_BYTES);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * C::STAGE_BYTES + C::EPI_BYTES);
+  const uint32_t bar0 = ptx::smem_u32(bars);
+  auto full_bar = [&](int s) { return bar0 + 8u * s; };
+  auto empty_bar = [&](int s) { return bar0 + 8u * (STAGES + s); };
+  auto tfull_bar = [&](int a) { return bar0 + 8u * (2 * STAGES + a); };
+  auto tempty_bar = [&](int a) { return bar0 + 8u * (2 * STAGES + 2 + a); };
+  const uint32_t drain_bar = bar0 + 8u * (2 * STAGES + 4);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NUM_BARS);
+  volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = ptx::cluster_ctarank();
+  const int pair = blockIdx.x >> 1;
+  const int npairs = gridDim.x >> 1;
+
+  // A launch after a recorded timeout does no work; both CTAs of a pair read the
+  // same word written by an earlier kernel, so they agree.
+  if (threadIdx.x == 0) *abort = (err != nullptr && *reinterpret_cast<volatile int*>(&err->code) != 0) ? 1 : 0;
+  __syncthreads();
+  if (*abort) return;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      ptx::mbar_init(full_bar(s), 1);
+      ptx::mbar_init(empty_bar(s), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      ptx::mbar_init(tfull_bar(a), 1);
+      ptx::mbar_init(tempty_bar(a), 2 * EPI_WARPS);
+    }
+    ptx::mbar_init(drain_bar, 1);
+    ptx::fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    ptx::tma_prefetch_desc(&tmA);
+    ptx::tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc_pair(ptx::smem_u32(tmem_slot), C::TMEM_COLS);
+    ptx::tmem_relinquish_pair();
+  }
+  ptx::tc_fence_before();
+  __syncwarp();
+  ptx::cluster_sync();
+  ptx::tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int num_tiles = num_m_tiles * num_n_tiles;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------- TMA producer (both CTAs)
+      int stage = 0;
+      uint32_t phase = 0;
+      long issued = 0;
+      bool ok = true;
+      for (int tile = pair; tile < num_tiles && ok; tile += npairs) {
+        const int m_blk = tile % num_m_tiles, n_blk = tile / num_m_tiles;
+        const int arow = m_blk * 2 * BMC + (int)rank * BMC;
+        const int brow = n_blk * BN + (int)rank * (BN / 2);
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!ptx::mbar_wait_bounded(empty_bar(stage), phase ^ 1u, abort, WAIT_LIMIT_NS)) {
+            ok = false;
+            break;
+          }
+          if (rank == 0) ptx::mbar_arrive_expect_tx(full_bar(stage), 2 * C::STAGE_BYTES);
+          const uint32_t lbar = ptx::mapa_shared(full_bar(stage), 0);
+          ptx::tma_load_2d_pair(sA + stage * C::A_BYTES, &tmA, lbar, kb * BK, arow);
+          ptx::tma_load_2d_pair(sB + stage * C::B_BYTES, &tmB, lbar, kb * BK, brow);
+          ++issued;
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+      }
+      if (!ok) {
+        if (!*abort) record_timeout(err, WHERE_GEMM_PRODUCER, abort);
+        if (rank == 0) {   // the leader's full barriers count both CTAs' loads
+          const long n = issued < STAGES ? issued : STAGES;
+          int s = stage;
+          uint32_t ph = phase;
+          volatile int never = 0;
+          for (long i = 0; i < n; ++i) {
+            if (--s < 0) { s = STAGES - 1; ph ^= 1u; }
+            ptx::mbar_wait_bounded(full_bar(s), ph, &never, WAIT_LIMIT_NS);
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && rank == 0) {
+      // ---------------- MMA issuer (leader CTA)
+      int stage = 0;
+      uint32_t phase = 0;
+      int local = 0;
+      bool ok = true;
+      for (int tile = pair; tile < num_tiles && ok; tile += npairs, ++local) {
+        const int acc = local & 1;
+        const uint32_t acc_phase = (local >> 1) & 1;
+        if (!ptx::mbar_wait_bounded(tempty_bar(acc), acc_phase ^ 1u, abort, WAIT_LIMIT_NS)) {
+          ok = false;
+          break;
+        }
+        ptx::tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * BN;
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!ptx::mbar_wait_bounded(full_bar(stage), phase, abort, WAIT_LIMIT_NS)) {
+            ok = false;
+            break;
+          }
+          ptx::tc_fence_after();
+          const uint32_t a0 = sA + stage * C::A_BYTES;
+          const uint32_t b0 = sB + stage * C::B_BYTES;
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k)
+            ptx::tc_mma_bf16_pair(d_tmem, ptx::smem_desc_sw128(a0 + k * 32), ptx::smem_desc_sw128(b0 + k * 32),
+                                  C::IDESC, (kb | k) != 0);
+          ptx::tc_commit_pair(empty_bar(stage), 0x3);
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        ptx::tc_commit_pair(tfull_bar(acc), 0x3);
+      }
+      if (!ok && !*abort) record_timeout(err, WHERE_GEMM_MMA, abort);
+      ptx::tc_commit_pair(drain_bar, 0x1);
+      volatile int never = 0;
+      if (!ptx::mbar_wait_bounded(drain_bar, 0, &never, WAIT_LIMIT_NS)) record_timeout(err, WHERE_GEMM_DRAIN, abort);
+    }
+  } else {
+    // ---------------- epilogue warps 2..9: TMEM lane quarter = warp % 4; part (warp - 2) / 4
+    // takes chunks [part * PART_CH, ...) of the tile's BN / 16 column chunks
+    const int quarter = warp & 3;
+    const int part = (warp - 2) >> 2;
+    constexpr int CW = C::CW;
+    constexpr int PASSES = EpiLanes<CW>::PASSES;
+    float* st = epi_smem + (warp - 2) * 32 * (CW + 4);
+    const uint32_t leader_tempty0 = ptx::mapa_shared(tempty_bar(0), 0);
+    const uint32_t leader_tempty1 = ptx::mapa_shared(tempty_bar(1), 0);
+    int local = 0;
+    for (int tile = pair; tile < num_tiles; tile += npairs, ++local) {
+      const int acc = local & 1;
+      const uint32_t acc_phase = (local >> 1) & 1;
+      if (!ptx::mbar_wait_bounded(tfull_bar(acc), acc_phase, abort, WAIT_LIMIT_NS)) {
+        if (!*abort) record_timeout(err, WHERE_GEMM_EPILOGUE, abort);
+        break;
+      }
+      ptx::tc_fence_after();
+      const int m_blk = tile % num_m_tiles, n_blk = tile / num_m_tiles;
+      const int row0 = m_blk * 2 * BMC + (int)rank * BMC + quarter * 32;
+      const int cbeg = min(part * C::PART_CH * CW, BN);
+      const int cend = min(cbeg + C::PART_CH * CW, BN);
+      const int valid_end = min(cend, ep.N - n_blk * BN);
+      const int nch = valid_end > cbeg ? (valid_end - cbeg + CW - 1) / CW : 0;
+      const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * BN + cbeg;
+      const int gcol = n_blk * BN + cbeg;
+      auto release = [&]() {
+        ptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive_remote(acc ? leader_tempty1 : leader_tempty0);
+      };
+      if (nch == 0) {
+        release();
+        continue;
+      }
+      float va[CW], vb[CW];
+      float4 pa[PASSES], pb[PASSES];
+      float4 ba, bb;
+      auto process = [&](float (&v)[CW], const float4 (&pre)[PASSES], const float4 bias4, int c) {
+#pragma unroll
+        for (int j = 0; j < CW; j += 4)
+          *reinterpret_cast<float4*>(st + lane * (CW + 4) + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+        __syncwarp();
+        epilogue_warp_tile<KIND, OutT, CW>(ep, st, row0, gcol + c * CW, lane, pre, bias4);
+        __syncwarp();
+      };
+      epilogue_prefetch<KIND, CW>(ep, row0, gcol, lane, pa, ba);
+      ptx::tmem_ld(taddr, va);
+#pragma unroll 1
+      for (int c = 0; c < nch; c += 2) {
+        ptx::tmem_ld_wait();
+        if (c == nch - 1) release();
+        if (c + 1 < nch) {
+          epilogue_prefetch<KIND, CW>(ep, row0, gcol + (c + 1) * CW, lane, pb, bb);
+          ptx::tmem_ld(taddr + (c + 1) * CW, vb);
+        }
+        process(va, pa, ba, c);
+        if (c + 1 >= nch) break;
+        ptx::tmem_ld_wait();
+        if (c + 1 == nch - 1) release();
+        if (c + 2 < nch) {
+          epilogue_prefetch<KIND, CW>(ep, row0, gcol + (c + 2) * CW, lane, pa, ba);
+          ptx::tmem_ld(taddr + (c + 2) * CW, va);
+        }
+        process(vb, pb, bb, c + 1);
+      }
+    }
+  }
+
+  // both CTAs finish every access to the pair's shared memory and TMEM before either leaves
+  ptx::tc_fence_before();
+  __syncwarp();
+  ptx::cluster_sync();
+  if (warp == 1) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc_pair(tmem_base, C::TMEM_COLS);
+  }
+}
+
+// ------------------------------------------------------------------ host side
+
+template <int BN, int STAGES, int KIND, typename OutT>
+struct Tc2Launcher {
+  static int max_clusters;
+  static cudaError_t prepare() {
+    using Cf = Tc2Cfg<BN, STAGES>;
+    auto kern = gemm_tc2_kernel<BN, STAGES, KIND, OutT>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cf::SMEM);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 0);
+    cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3(2 * 74);
+    cfg.blockDim = dim3(NUM_THREADS);
+    cfg.dynamicSmemBytes = Cf::SMEM;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    e = cudaOccupancyMaxActiveClusters(&n, kern, &cfg);
+    if (e != cudaSuccess || n < 1) {
+      cudaGetLastError();
+      n = 0;
+    }
+    max_clusters = n;
+    return cudaSuccess;
+  }
+  static cudaError_t launch(const GemmArgs& g, const EpiParams& ep, DevError* err, cudaStream_t st) {
+    using Cf = Tc2Cfg<BN, STAGES>;
+    if (max_clusters < 1) return cudaErrorInvalidConfiguration;
+    CUtensorMap ta, tb;
+    if (make_tmap_bf16(&ta, g.A, g.M, g.K, g.lda, BMC) || make_tmap_bf16(&tb, g.B, g.N, g.K, g.ldb, BN / 2))
+      return cudaErrorInvalidValue;
+    const int mt = (g.M + 2 * BMC - 1) / (2 * BMC), nt = (g.N + BN - 1) / BN;
+    const int tiles = mt * nt;
+    const int pairs = tiles < max_clusters ? tiles : max_clusters;
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3(2 * pairs);
+    cfg.blockDim = dim3(NUM_THREADS);
+    cfg.dynamicSmemBytes = Cf::SMEM;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, gemm_tc2_kernel<BN, STAGES, KIND, OutT>, ta, tb, mt, nt, (g.K + BK - 1) / BK,
+                              ep, err);
+  }
+};
+template <int BN, int STAGES, int KIND, typename OutT>
+int Tc2Launcher<BN, STAGES, KIND, OutT>::max_clusters = 0;
+
+// (tile N, pipeline stages) per instantiation: stages fill the shared memory left
+// by the epilogue staging tiles
+#define KD_TC2_LIST(X)                                  \
+  X(256, 6, EPI_BIAS, bf16) X(208, 6, EPI_BIAS, bf16)   \
+  X(160, 7, EPI_BIAS, bf16) X(144, 7, EPI_BIAS, bf16)   \
+  X(256, 6, EPI_BIAS_GELU, bf16) X(208, 6, EPI_BIAS_GELU, bf16) \
+  X(160, 7, EPI_BIAS_GELU, bf16) X(144, 7, EPI_BIAS_GELU, bf16) \
+  X(256, 6, EPI_BIAS_RESID, float) X(208, 6, EPI_BIAS_RESID, float) \
+  X(160, 7, EPI_BIAS_RESID, float) X(144, 7, EPI_BIAS_RESID, float)
+
+}  // namespace
+
+cudaError_t gemm_tc2_prepare() {
+#define KD_PREP(BN_, ST_, KIND_, OUT_)                                  \
+  {                                                                    \
+    cudaError_t e_ = Tc2Launcher<BN_, ST_, KIND_, OUT_>::prepare();    \
+    if (e_ != cudaSuccess) return e_;                                  \
+  }
+  KD_TC2_LIST(KD_PREP)
+#undef KD_PREP
+  return cudaSuccess;
+}
+
+bool gemm_tc2_supports(int kind, bool out_f32) {
+  return (kind == EPI_BIAS && !out_f32) || (kind == EPI_BIAS_GELU && !out_f32) ||
+         (kind == EPI_BIAS_RESID && out_f32);
+}
+
+// Tile N minimizing (rounds of pair tiles) x N over the available CTA pairs.
+int gemm_tc2_pick_bn(int M, int N) {
+  const int cands[4] = {256, 208, 160, 144};
+  const int pairs = Tc2Launcher<256, 6, EPI_BIAS, bf16>::max_clusters > 0
+                        ? Tc2Launcher<256, 6, EPI_BIAS, bf16>::max_clusters : 74;
+  const long mt = (M + 2 * BMC - 1) / (2 * BMC);
+  int best = 256;
+  long best_cost = -1;
+  for (int bn : cands) {
+    const long tiles = mt * ((N + bn - 1) / bn);
+    const long rounds = (tiles + pairs - 1) / pairs;
+    const long cost = rounds * bn;
+    if (best_cost < 0 || cost < best_cost) {
+      best_cost = cost;
+      best = bn;
+    }
+  }
+  return best;
+}
+
+cudaError_t gemm_tc2(const GemmArgs& g, int bn, int kind, bool out_f32, const EpiParams& ep, DevError* err,
+                     cudaStream_t st) {
+  if (g.M <= 0 || g.N <= 0) return cudaSuccess;
+  if (g.K <= 0) return cudaErrorInvalidValue;
+#define KD_RUN(BN_, ST_, KIND_, OUT_)                                                   \
+  if (bn == BN_ && kind == KIND_ && out_f32 == std::is_same<OUT_, float>::value)        \
+    return Tc2Launcher<BN_, ST_, KIND_, OUT_>::launch(g, ep, err, st);
+  KD_TC2_LIST(KD_RUN)
+#undef KD_RUN
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace kd

@@ -1,6 +1,7 @@
 // Internal launchers of the denoiser kernels (not part of the public C ABI).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include "common.cuh"
 #include "epilogue.cuh"
@@ -20,6 +21,18 @@ struct GemmArgs {
 cudaError_t gemm_tc(const GemmArgs& g, int bn, int kind, bool out_f32, const EpiParams& ep, DevError* err,
                     cudaStream_t st, int num_sms);
 bool gemm_tc_available();
+
+// TMA descriptor of a row-major bf16 matrix [rows, ld] whose first `cols` columns are
+// the K extent; boxes of 64 columns x box_rows rows, 128-byte swizzle, zero fill.
+int make_tmap_bf16(CUtensorMap* m, const void* base, int rows, int cols, int ld, int box_rows);
+
+// tcgen05 GEMM on CTA pairs (256-row tiles).  bn in {144, 160, 208, 256}; kinds
+// EPI_BIAS / EPI_BIAS_GELU with bf16 output and EPI_BIAS_RESID with fp32 output.
+cudaError_t gemm_tc2(const GemmArgs& g, int bn, int kind, bool out_f32, const EpiParams& ep, DevError* err,
+                     cudaStream_t st);
+cudaError_t gemm_tc2_prepare();
+bool gemm_tc2_supports(int kind, bool out_f32);
+int gemm_tc2_pick_bn(int M, int N);
 // Set the dynamic shared-memory limits of every kernel instantiation (call once
 // per device before any launch or graph capture).
 cudaError_t gemm_tc_prepare();
