@@ -20,6 +20,7 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "launch.cuh"
 #include "ptx.cuh"
 
 namespace kd {
@@ -56,6 +57,8 @@ __global__ void __launch_bounds__(ATT_MAX_WARPS * 32, 1)
 attn_bf16_kernel(const bf16* __restrict__ qkv, bf16* __restrict__ out, const int* __restrict__ lengths,
                  int len_mod, int S) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
+  ptx::pdl_wait();
+  ptx::pdl_trigger();
   const int h = blockIdx.x, seq = blockIdx.y;
   int n_valid = 1 + lengths[seq % len_mod];
   n_valid = n_valid < 1 ? 1 : (n_valid > S ? S : n_valid);
@@ -193,6 +196,8 @@ attn_bf16_kernel(const bf16* __restrict__ qkv, bf16* __restrict__ out, const int
 
 __global__ void __launch_bounds__(128) attn_f32_kernel(const float* __restrict__ qkv, float* __restrict__ out,
                                                        const int* __restrict__ lengths, int len_mod, int S) {
+  ptx::pdl_wait();
+  ptx::pdl_trigger();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int q = blockIdx.x * 4 + warp, h = blockIdx.y, seq = blockIdx.z;
   if (q >= S) return;
@@ -239,8 +244,7 @@ cudaError_t attention_bf16(const bf16* qkv, bf16* out, const int* lengths, int l
   int warps = (S + 15) / 16;
   warps = warps > ATT_MAX_WARPS ? ATT_MAX_WARPS : warps;
   dim3 grid(H, nseq);
-  attn_bf16_kernel<<<grid, 32 * warps, smem, st>>>(qkv, out, lengths, len_mod, S);
-  return cudaGetLastError();
+  return launch_kernel(attn_bf16_kernel, grid, dim3(32 * warps), smem, st, qkv, out, lengths, len_mod, S);
 }
 
 cudaError_t attention_prepare() {
@@ -252,8 +256,7 @@ cudaError_t attention_f32(const float* qkv, float* out, const int* lengths, int 
                           cudaStream_t st) {
   if (nseq <= 0 || S <= 0) return cudaSuccess;
   dim3 grid((S + 3) / 4, H, nseq);
-  attn_f32_kernel<<<grid, 128, 0, st>>>(qkv, out, lengths, len_mod, S);
-  return cudaGetLastError();
+  return launch_kernel(attn_f32_kernel, grid, dim3(128), 0, st, qkv, out, lengths, len_mod, S);
 }
 
 }  // namespace kd

@@ -7,6 +7,8 @@
 #include "common.cuh"
 #include "epilogue.cuh"
 #include "kernels.h"
+#include "launch.cuh"
+#include "ptx.cuh"
 
 namespace kd {
 namespace {
@@ -18,6 +20,8 @@ __global__ void __launch_bounds__(256) gemm_f32_kernel(const float* __restrict__
                                                        int M, int N, int K, int lda, int ldb, EpiParams ep) {
   __shared__ __align__(16) float As[TK][TM + 4];
   __shared__ __align__(16) float Bs[TK][TN + 4];
+  ptx::pdl_wait();
+  ptx::pdl_trigger();
   const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
   const int m0 = blockIdx.y * TM, n0 = blockIdx.x * TN;
   float acc[4][4] = {};
@@ -59,12 +63,12 @@ cudaError_t gemm_f32(const GemmArgs& g, int kind, const EpiParams& ep, cudaStrea
   const float* A = static_cast<const float*>(g.A);
   const float* B = static_cast<const float*>(g.B);
   switch (kind) {
-    case EPI_BIAS: gemm_f32_kernel<EPI_BIAS><<<grid, 256, 0, st>>>(A, B, g.M, g.N, g.K, g.lda, g.ldb, ep); break;
-    case EPI_BIAS_GELU: gemm_f32_kernel<EPI_BIAS_GELU><<<grid, 256, 0, st>>>(A, B, g.M, g.N, g.K, g.lda, g.ldb, ep); break;
-    case EPI_BIAS_SILU: gemm_f32_kernel<EPI_BIAS_SILU><<<grid, 256, 0, st>>>(A, B, g.M, g.N, g.K, g.lda, g.ldb, ep); break;
-    case EPI_BIAS_RESID: gemm_f32_kernel<EPI_BIAS_RESID><<<grid, 256, 0, st>>>(A, B, g.M, g.N, g.K, g.lda, g.ldb, ep); break;
-    case EPI_INPROJ: gemm_f32_kernel<EPI_INPROJ><<<grid, 256, 0, st>>>(A, B, g.M, g.N, g.K, g.lda, g.ldb, ep); break;
-    case EPI_OUTPROJ: gemm_f32_kernel<EPI_OUTPROJ><<<grid, 256, 0, st>>>(A, B, g.M, g.N, g.K, g.lda, g.ldb, ep); break;
+    case EPI_BIAS: return launch_kernel(gemm_f32_kernel<EPI_BIAS>, grid, dim3(256), 0, st, A, B, g.M, g.N, g.K, g.lda, g.ldb, ep);
+    case EPI_BIAS_GELU: return launch_kernel(gemm_f32_kernel<EPI_BIAS_GELU>, grid, dim3(256), 0, st, A, B, g.M, g.N, g.K, g.lda, g.ldb, ep);
+    case EPI_BIAS_SILU: return launch_kernel(gemm_f32_kernel<EPI_BIAS_SILU>, grid, dim3(256), 0, st, A, B, g.M, g.N, g.K, g.lda, g.ldb, ep);
+    case EPI_BIAS_RESID: return launch_kernel(gemm_f32_kernel<EPI_BIAS_RESID>, grid, dim3(256), 0, st, A, B, g.M, g.N, g.K, g.lda, g.ldb, ep);
+    case EPI_INPROJ: return launch_kernel(gemm_f32_kernel<EPI_INPROJ>, grid, dim3(256), 0, st, A, B, g.M, g.N, g.K, g.lda, g.ldb, ep);
+    case EPI_OUTPROJ: return launch_kernel(gemm_f32_kernel<EPI_OUTPROJ>, grid, dim3(256), 0, st, A, B, g.M, g.N, g.K, g.lda, g.ldb, ep);
     default: return cudaErrorInvalidValue;
   }
   return cudaGetLastError();

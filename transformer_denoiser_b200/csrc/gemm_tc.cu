@@ -24,6 +24,7 @@
 #include "common.cuh"
 #include "epilogue.cuh"
 #include "kernels.h"
+#include "launch.cuh"
 #include "ptx.cuh"
 
 namespace kd {
@@ -89,11 +90,6 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // A launch after a recorded timeout does no work (its inputs are already invalid).
-  if (threadIdx.x == 0) *abort = (err != nullptr && *reinterpret_cast<volatile int*>(&err->code) != 0) ? 1 : 0;
-  __syncthreads();
-  if (*abort) return;
-
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       ptx::mbar_init(full_bar(s), 1);
@@ -114,12 +110,17 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     ptx::tmem_alloc(ptx::smem_u32(tmem_slot), C::TMEM_COLS);
     ptx::tmem_relinquish();
   }
+  // prologue done: let the next kernel launch, then wait for the previous one
+  ptx::pdl_trigger();
+  ptx::pdl_wait();
+  // A launch after a recorded timeout does no work (its inputs are already invalid).
+  if (threadIdx.x == 0) *abort = (err != nullptr && *reinterpret_cast<volatile int*>(&err->code) != 0) ? 1 : 0;
   ptx::tc_fence_before();
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  const int num_tiles = num_m_tiles * num_n_tiles;
+  const int num_tiles = *abort ? 0 : num_m_tiles * num_n_tiles;
 
   if (warp == 0) {
     if (lane == 0) {
@@ -312,8 +313,7 @@ cudaError_t launch_impl(const GemmArgs& g, const EpiParams& ep, DevError* err, c
   const int tiles = mt * nt;
   const int grid = tiles < num_sms ? tiles : num_sms;
   const int kb = (g.K + BK - 1) / BK;
-  kern<<<grid, NUM_THREADS, Cf::SMEM, st>>>(ta, tb, mt, nt, kb, ep, err);
-  return cudaGetLastError();
+  return launch_kernel(kern, dim3(grid), dim3(NUM_THREADS), Cf::SMEM, st, ta, tb, mt, nt, kb, ep, err);
 }
 
 }  // namespace

@@ -22,6 +22,7 @@
 #include "common.cuh"
 #include "epilogue.cuh"
 #include "kernels.h"
+#include "launch.cuh"
 #include "ptx.cuh"
 
 namespace kd {
@@ -90,12 +91,6 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
   const int pair = blockIdx.x >> 1;
   const int npairs = gridDim.x >> 1;
 
-  // A launch after a recorded timeout does no work; both CTAs of a pair read the
-  // same word written by an earlier kernel, so they agree.
-  if (threadIdx.x == 0) *abort = (err != nullptr && *reinterpret_cast<volatile int*>(&err->code) != 0) ? 1 : 0;
-  __syncthreads();
-  if (*abort) return;
-
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       ptx::mbar_init(full_bar(s), 1);
@@ -116,12 +111,18 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
     ptx::tmem_alloc_pair(ptx::smem_u32(tmem_slot), C::TMEM_COLS);
     ptx::tmem_relinquish_pair();
   }
+  // prologue done: let the next kernel launch, then wait for the previous one
+  ptx::pdl_trigger();
+  ptx::pdl_wait();
+  // A launch after a recorded timeout does no work; both CTAs of a pair read the
+  // same word (written by an earlier kernel, visible after the wait), so they agree.
+  if (threadIdx.x == 0) *abort = (err != nullptr && *reinterpret_cast<volatile int*>(&err->code) != 0) ? 1 : 0;
   ptx::tc_fence_before();
   __syncwarp();
   ptx::cluster_sync();
   ptx::tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  const int num_tiles = num_m_tiles * num_n_tiles;
+  const int num_tiles = *abort ? 0 : num_m_tiles * num_n_tiles;
 
   if (warp == 0) {
     if (lane == 0) {
@@ -322,17 +323,19 @@ struct Tc2Launcher {
     const int tiles = mt * nt;
     const int pairs = tiles < max_clusters ? tiles : max_clusters;
     cudaLaunchConfig_t cfg = {};
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 2;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.gridDim = dim3(2 * pairs);
     cfg.blockDim = dim3(NUM_THREADS);
     cfg.dynamicSmemBytes = Cf::SMEM;
     cfg.stream = st;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = pdl_enabled() ? 2 : 1;
     return cudaLaunchKernelEx(&cfg, gemm_tc2_kernel<BN, STAGES, KIND, OutT>, ta, tb, mt, nt, (g.K + BK - 1) / BK,
                               ep, err);
   }

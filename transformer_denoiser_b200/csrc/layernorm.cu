@@ -9,6 +9,8 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "launch.cuh"
+#include "ptx.cuh"
 
 namespace kd {
 namespace {
@@ -23,6 +25,8 @@ template <typename OutT>
 __global__ void __launch_bounds__(256) layernorm_kernel(const float* y, OutT* __restrict__ out,
                                                         const float* __restrict__ gamma,
                                                         const float* __restrict__ beta, int M, float* out32) {
+  ptx::pdl_wait();
+  ptx::pdl_trigger();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int row = blockIdx.x * 8 + warp;
   if (row >= M) return;
@@ -74,10 +78,10 @@ cudaError_t layernorm(const float* y, void* out, bool out_bf16, const float* gam
   if (M <= 0) return cudaSuccess;
   const int grid = (M + 7) / 8;
   if (out_bf16)
-    layernorm_kernel<bf16><<<grid, 256, 0, st>>>(y, static_cast<bf16*>(out), gamma, beta, M, out32);
-  else
-    layernorm_kernel<float><<<grid, 256, 0, st>>>(y, static_cast<float*>(out), gamma, beta, M, out32);
-  return cudaGetLastError();
+    return launch_kernel(layernorm_kernel<bf16>, dim3(grid), dim3(256), 0, st, y, static_cast<bf16*>(out), gamma, beta,
+                         M, out32);
+  return launch_kernel(layernorm_kernel<float>, dim3(grid), dim3(256), 0, st, y, static_cast<float*>(out), gamma, beta,
+                       M, out32);
 }
 
 }  // namespace kd

@@ -9,6 +9,8 @@
 #include "common.cuh"
 #include "epilogue.cuh"
 #include "kernels.h"
+#include "launch.cuh"
+#include "ptx.cuh"
 
 namespace kd {
 namespace {
@@ -16,6 +18,8 @@ namespace {
 template <typename T>
 __global__ void pack_frames_kernel(const float* __restrict__ src, int nsrc, int ld_src, int f0, int nf,
                                    T* __restrict__ A, int lda, int col0, int nseq, int T_, int S) {
+  ptx::pdl_wait();
+  ptx::pdl_trigger();
   const long total = (long)nseq * T_ * nf;
   for (long idx = blockIdx.x * (long)blockDim.x + threadIdx.x; idx < total; idx += (long)gridDim.x * blockDim.x) {
     const int f = idx % nf;
@@ -53,6 +57,8 @@ template <typename T>
 __global__ void g2l_body_input_kernel(const float* __restrict__ root_hat, const float* __restrict__ x,
                                       const int* __restrict__ lengths, int B, int nseq, int T_, int S,
                                       T* __restrict__ A, int lda) {
+  ptx::pdl_wait();
+  ptx::pdl_trigger();
   const int warp_global = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (warp_global >= nseq * T_) return;
@@ -75,6 +81,8 @@ template <typename T>
 __global__ void cfg_ddim_kernel(const float* __restrict__ root_hat, const float* __restrict__ body_hat,
                                 float* __restrict__ x, const int* __restrict__ lengths, int B, int T_, float w,
                                 float c0, float c1, T* __restrict__ A_next, int lda, int S) {
+  ptx::pdl_wait();
+  ptx::pdl_trigger();
   const long total = (long)B * T_ * MOTION_F;
   for (long idx = blockIdx.x * (long)blockDim.x + threadIdx.x; idx < total; idx += (long)gridDim.x * blockDim.x) {
     const int f = idx % MOTION_F;
@@ -105,6 +113,8 @@ __global__ void cfg_ddim_kernel(const float* __restrict__ root_hat, const float*
 template <typename T>
 __global__ void pack_embeddings_kernel(const float* __restrict__ text, int B, const float* __restrict__ null_emb,
                                        int null_batch, int null_rows, T* __restrict__ out) {
+  ptx::pdl_wait();
+  ptx::pdl_trigger();
   const long total = (long)(B + null_rows) * DTXT;
   for (long idx = blockIdx.x * (long)blockDim.x + threadIdx.x; idx < total; idx += (long)gridDim.x * blockDim.x) {
     const int r = idx / DTXT, c = idx % DTXT;
@@ -115,12 +125,16 @@ __global__ void pack_embeddings_kernel(const float* __restrict__ text, int B, co
 
 template <typename T>
 __global__ void gather_rows_kernel(const float* __restrict__ pe, int t0, int stride, int n, T* __restrict__ out) {
+  ptx::pdl_wait();
+  ptx::pdl_trigger();
   const long total = (long)n * D;
   for (long idx = blockIdx.x * (long)blockDim.x + threadIdx.x; idx < total; idx += (long)gridDim.x * blockDim.x) {
     const int k = idx / D, c = idx % D;
     out[idx] = from_f<T>(pe[(long)(t0 - k * stride) * D + c]);
   }
 }
+
+#define LAUNCHK(K, G, B, ST, ...) return launch_kernel(K, dim3(G), dim3(B), 0, ST, __VA_ARGS__)
 
 inline int blocks_for(long n, int threads = 256) {
   long b = (n + threads - 1) / threads;
@@ -134,10 +148,10 @@ cudaError_t pack_frames(const float* src, int nsrc, int ld_src, int f0, int nf, 
   const long n = (long)nseq * T * nf;
   if (n <= 0) return cudaSuccess;
   if (a_bf16)
-    pack_frames_kernel<bf16><<<blocks_for(n), 256, 0, st>>>(src, nsrc, ld_src, f0, nf, static_cast<bf16*>(A), lda,
+    LAUNCHK(pack_frames_kernel<bf16>, blocks_for(n), 256, st, src, nsrc, ld_src, f0, nf, static_cast<bf16*>(A), lda,
                                                             col0, nseq, T, S);
   else
-    pack_frames_kernel<float><<<blocks_for(n), 256, 0, st>>>(src, nsrc, ld_src, f0, nf, static_cast<float*>(A), lda,
+    LAUNCHK(pack_frames_kernel<float>, blocks_for(n), 256, st, src, nsrc, ld_src, f0, nf, static_cast<float*>(A), lda,
                                                              col0, nseq, T, S);
   return cudaGetLastError();
 }
@@ -148,9 +162,9 @@ cudaError_t g2l_body_input(const float* root_hat, const float* x, const int* len
   if (warps <= 0) return cudaSuccess;
   const int grid = (int)((warps * 32 + 255) / 256);
   if (a_bf16)
-    g2l_body_input_kernel<bf16><<<grid, 256, 0, st>>>(root_hat, x, lengths, B, nseq, T, S, static_cast<bf16*>(A), lda);
+    LAUNCHK(g2l_body_input_kernel<bf16>, grid, 256, st, root_hat, x, lengths, B, nseq, T, S, static_cast<bf16*>(A), lda);
   else
-    g2l_body_input_kernel<float><<<grid, 256, 0, st>>>(root_hat, x, lengths, B, nseq, T, S, static_cast<float*>(A),
+    LAUNCHK(g2l_body_input_kernel<float>, grid, 256, st, root_hat, x, lengths, B, nseq, T, S, static_cast<float*>(A),
                                                        lda);
   return cudaGetLastError();
 }
@@ -160,10 +174,10 @@ cudaError_t cfg_ddim(const float* root_hat, const float* body_hat, float* x, con
   const long n = (long)B * T * MOTION_F;
   if (n <= 0) return cudaSuccess;
   if (a_bf16)
-    cfg_ddim_kernel<bf16><<<blocks_for(n), 256, 0, st>>>(root_hat, body_hat, x, lengths, B, T, w, c0, c1,
+    LAUNCHK(cfg_ddim_kernel<bf16>, blocks_for(n), 256, st, root_hat, body_hat, x, lengths, B, T, w, c0, c1,
                                                          static_cast<bf16*>(A_next), lda, S);
   else
-    cfg_ddim_kernel<float><<<blocks_for(n), 256, 0, st>>>(root_hat, body_hat, x, lengths, B, T, w, c0, c1,
+    LAUNCHK(cfg_ddim_kernel<float>, blocks_for(n), 256, st, root_hat, body_hat, x, lengths, B, T, w, c0, c1,
                                                           static_cast<float*>(A_next), lda, S);
   return cudaGetLastError();
 }
@@ -173,10 +187,10 @@ cudaError_t pack_embeddings(const float* text_emb, int B, const float* null_emb,
   const long n = (long)(B + null_rows) * DTXT;
   if (n <= 0) return cudaSuccess;
   if (out_bf16)
-    pack_embeddings_kernel<bf16><<<blocks_for(n), 256, 0, st>>>(text_emb, B, null_emb, null_batch, null_rows,
+    LAUNCHK(pack_embeddings_kernel<bf16>, blocks_for(n), 256, st, text_emb, B, null_emb, null_batch, null_rows,
                                                                 static_cast<bf16*>(out));
   else
-    pack_embeddings_kernel<float><<<blocks_for(n), 256, 0, st>>>(text_emb, B, null_emb, null_batch, null_rows,
+    LAUNCHK(pack_embeddings_kernel<float>, blocks_for(n), 256, st, text_emb, B, null_emb, null_batch, null_rows,
                                                                  static_cast<float*>(out));
   return cudaGetLastError();
 }
@@ -186,9 +200,9 @@ cudaError_t gather_timestep_rows(const float* pe, int t0, int stride, int n, voi
   const long total = (long)n * D;
   if (total <= 0) return cudaSuccess;
   if (out_bf16)
-    gather_rows_kernel<bf16><<<blocks_for(total), 256, 0, st>>>(pe, t0, stride, n, static_cast<bf16*>(out));
+    LAUNCHK(gather_rows_kernel<bf16>, blocks_for(total), 256, st, pe, t0, stride, n, static_cast<bf16*>(out));
   else
-    gather_rows_kernel<float><<<blocks_for(total), 256, 0, st>>>(pe, t0, stride, n, static_cast<float*>(out));
+    LAUNCHK(gather_rows_kernel<float>, blocks_for(total), 256, st, pe, t0, stride, n, static_cast<float*>(out));
   return cudaGetLastError();
 }
 
