@@ -45,8 +45,10 @@ KIMODO_API int kimodo_gemm_bf16(const void* A, int lda, const void* W, int ldw, 
  * The same product on pairs of SMs (one 256-row output tile per CTA pair,
  * tcgen05 cta_group::2), the kernel the denoiser uses for its large projections.
  * Arguments as kimodo_gemm_bf16; epilogues KIMODO_EPI_BIAS and KIMODO_EPI_BIAS_GELU
- * with bf16 output and KIMODO_EPI_BIAS_RESID with fp32 output.  tile_n: output
- * columns per pair tile, 144, 160, 208 or 256, or 0 for the library's choice.
+ * with bf16 output and KIMODO_EPI_BIAS_RESID with fp32 output; N % 16 == 0 and output
+ * rows a multiple of 16 bytes.  tile_n: output
+ * columns per pair tile, 144, 160, 208 or 256 (144 or 160 with the residual
+ * epilogue), or 0 for the library's choice.
  */
 KIMODO_API int kimodo_gemm_bf16_pair(const void* A, int lda, const void* W, int ldw, const float* bias,
                                      const void* resid, int ldr, void* out, int ldo, int M, int N, int K,

@@ -76,7 +76,8 @@ PAIR_CASES = [
     (4832, 3072, 1024, kb.EPI_BIAS, False, 256),
     (4832, 2048, 1024, kb.EPI_BIAS_GELU, False, 144),
     (4832, 1024, 1024, kb.EPI_BIAS_RESID, True, 160),
-    (4832, 1024, 2048, kb.EPI_BIAS_RESID, True, 208),
+    (4832, 1024, 2048, kb.EPI_BIAS_RESID, True, 144),
+    (611, 1024, 1024, kb.EPI_BIAS_RESID, True, 160),
     (300, 1024, 1024, kb.EPI_BIAS, False, 160),           # second CTA of the last pair tile fully out of range
     (1283, 2048, 1024, kb.EPI_BIAS_GELU, False, 256),
 ]

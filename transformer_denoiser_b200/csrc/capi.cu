@@ -163,7 +163,7 @@ int gemm(kimodo_ctx* c, const void* A, int lda, const void* W, int ldw, int M, i
                        (kind == EPI_BIAS_RESID ? (double)M * N * 4.0 : 0.0);
   if (c->bf16()) {
     if (c->pair_gemm && M >= 1024 && N >= 256 && gemm_tc2_supports(kind, out_f32)) {
-      const int bn = gemm_tc2_pick_bn(M, N);
+      const int bn = gemm_tc2_pick_bn(M, N, kind);
       return launch(c, cls_override >= 0 ? cls_override : CLS_GEMM_TC, flops, bytes, st, "gemm_tc2",
                     [&] { return gemm_tc2(g, bn, kind, out_f32, ep, c->derr, st); });
     }
@@ -849,14 +849,18 @@ int kimodo_gemm_bf16_pair(const void* A, int lda, const void* W, int ldw, const 
     return set_error(KIMODO_EINVAL, "out, resid and bias need 16-byte alignment and ldo, ldr multiples of 4");
   if (!gemm_tc2_supports(epilogue, out_f32 != 0))
     return set_error(KIMODO_EINVAL, "pair GEMM epilogues: bias or GELU with bf16 output, residual with fp32 output");
+  if (N % 16 || ((long)ldo * (out_f32 ? 4 : 2)) % 16)
+    return set_error(KIMODO_EINVAL, "pair GEMM needs N % 16 == 0 and 16-byte output rows");
   if (tile_n != 0 && tile_n != 144 && tile_n != 160 && tile_n != 208 && tile_n != 256)
     return set_error(KIMODO_EINVAL, "tile_n must be 0, 144, 160, 208 or 256");
+  if (epilogue == KIMODO_EPI_BIAS_RESID && tile_n > 160)
+    return set_error(KIMODO_EINVAL, "the residual epilogue is built for tile_n 144 and 160");
   KD_TRY(prepared_device());
   GemmArgs g;
   g.A = A; g.B = W; g.M = M; g.N = N; g.K = K; g.lda = lda; g.ldb = ldw;
   EpiParams ep;
   ep.bias = bias; ep.out = out; ep.ldo = ldo; ep.resid = resid; ep.ldr = ldr; ep.N = N; ep.M = M;
-  const int bn = tile_n ? tile_n : gemm_tc2_pick_bn(M, N);
+  const int bn = tile_n ? tile_n : gemm_tc2_pick_bn(M, N, epilogue);
   KD_CUDA(gemm_tc2(g, bn, epilogue, out_f32 != 0, ep, kernel_error_word(), static_cast<cudaStream_t>(stream)));
   return KIMODO_OK;
 }

@@ -334,6 +334,23 @@ int make_tmap_bf16(CUtensorMap* m, const void* base, int rows, int cols, int ld,
 }
 
 
+// Row-major matrix [rows, ld] of fp32 (elem 4) or bf16 (elem 2), K extent `cols`,
+// boxes of box_cols x box_rows, no swizzle (epilogue staging tiles).
+int make_tmap_plain(CUtensorMap* m, const void* base, int elem, int rows, int cols, long ld, int box_cols,
+                    int box_rows) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return -1;
+  if ((reinterpret_cast<uintptr_t>(base) & 15) || (ld * elem) % 16 || (box_cols * elem) % 16) return -2;
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)ld * elem};
+  cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(m, elem == 4 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                   const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? 0 : -3;
+}
+
 // Dispatch on (tile N, epilogue kind, output type).  The residual is fp32 (the
 // residual stream of the post-norm layers is kept in fp32; operands are bf16).
 static cudaError_t dispatch(const GemmArgs& g, int bn, int kind, bool out_f32, const EpiParams& ep, DevError* err,

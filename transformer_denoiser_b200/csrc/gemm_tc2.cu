@@ -39,17 +39,21 @@ constexpr uint32_t tmem_cols_for(uint32_t n) {
   return n <= 32 ? 32 : n <= 64 ? 64 : n <= 128 ? 128 : n <= 256 ? 256 : 512;
 }
 
-template <int BN, int STAGES>
+template <int BN, int STAGES, int KIND>
 struct Tc2Cfg {
   static constexpr uint32_t A_BYTES = BMC * BK * 2;
   static constexpr uint32_t B_BYTES = (BN / 2) * BK * 2;
   static constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr uint32_t TMEM_COLS = tmem_cols_for(2 * BN);
-  static constexpr int CW = 16;
+  static constexpr int CW = 16;                         // columns per epilogue chunk
   static constexpr int NCH = BN / CW;
   static constexpr int PART_CH = (NCH + 1) / 2;
-  static constexpr uint32_t EPI_BYTES = EPI_WARPS * 32 * (CW + 4) * 4;
-  static constexpr uint32_t NUM_BARS = 2 * STAGES + 5;
+  static constexpr uint32_t STG_BYTES = 32 * CW * 4;     // one 32-row staging tile (fp32 size)
+  // staging tiles per epilogue warp: two alternating ones, or, with a residual, one per
+  // chunk of the warp's tile share so the whole residual share is loaded ahead of the MMA
+  static constexpr int NBUF = KIND == EPI_BIAS_RESID ? PART_CH : 2;
+  static constexpr uint32_t EPI_BYTES = EPI_WARPS * NBUF * STG_BYTES;
+  static constexpr uint32_t NUM_BARS = 2 * STAGES + 5 + NBUF * EPI_WARPS;
   static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE_BYTES + EPI_BYTES + NUM_BARS * 8 + 16;
   static constexpr uint32_t IDESC = ptx::idesc_bf16_f32(2 * BMC, BN);
   static_assert(BN % 16 == 0 && BN >= 32 && BN <= 256, "UMMA N for M=256");
@@ -68,8 +72,9 @@ __device__ __forceinline__ void record_timeout(DevError* err, int where, volatil
 template <int BN, int STAGES, int KIND, typename OutT>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                const __grid_constant__ CUtensorMap tmO, const __grid_constant__ CUtensorMap tmR,
                 int num_m_tiles, int num_n_tiles, int num_kb, EpiParams ep, DevError* err) {
-  using C = Tc2Cfg<BN, STAGES>;
+  using C = Tc2Cfg<BN, STAGES, KIND>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sA = ptx::smem_u32(smem);
@@ -82,6 +87,7 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
   auto tfull_bar = [&](int a) { return bar0 + 8u * (2 * STAGES + a); };
   auto tempty_bar = [&](int a) { return bar0 + 8u * (2 * STAGES + 2 + a); };
   const uint32_t drain_bar = bar0 + 8u * (2 * STAGES + 4);
+  auto res_bar = [&](int ew, int b) { return bar0 + 8u * (2 * STAGES + 5 + C::NBUF * ew + b); };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NUM_BARS);
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -101,11 +107,14 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
       ptx::mbar_init(tempty_bar(a), 2 * EPI_WARPS);
     }
     ptx::mbar_init(drain_bar, 1);
+    for (int i = 0; i < C::NBUF * EPI_WARPS; ++i) ptx::mbar_init(res_bar(i / C::NBUF, i % C::NBUF), 1);
     ptx::fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
     ptx::tma_prefetch_desc(&tmA);
     ptx::tma_prefetch_desc(&tmB);
+    ptx::tma_prefetch_desc(&tmO);
+    if (KIND == EPI_BIAS_RESID) ptx::tma_prefetch_desc(&tmR);
   }
   if (warp == 1) {
     ptx::tmem_alloc_pair(ptx::smem_u32(tmem_slot), C::TMEM_COLS);
@@ -203,31 +212,59 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
     }
   } else {
     // ---------------- epilogue warps 2..9: TMEM lane quarter = warp % 4; part (warp - 2) / 4
-    // takes chunks [part * PART_CH, ...) of the tile's BN / 16 column chunks
+    // takes chunks [part * PART_CH, ...) of the tile's BN / 16 column chunks.  Per chunk each
+    // thread finishes its accumulator row (bias, activation, residual) in registers and
+    // writes it into a dense 32 x 16 staging tile; one lane stores the tile with TMA.  Two
+    // staging tiles per warp alternate; the residual chunk arrives in the staging tile by TMA.
     const int quarter = warp & 3;
-    const int part = (warp - 2) >> 2;
+    const int ew = warp - 2;
+    const int part = ew >> 2;
     constexpr int CW = C::CW;
-    constexpr int PASSES = EpiLanes<CW>::PASSES;
-    float* st = epi_smem + (warp - 2) * 32 * (CW + 4);
+    uint8_t* stg_base = smem + STAGES * C::STAGE_BYTES + ew * C::NBUF * C::STG_BYTES;
     const uint32_t leader_tempty0 = ptx::mapa_shared(tempty_bar(0), 0);
     const uint32_t leader_tempty1 = ptx::mapa_shared(tempty_bar(1), 0);
+    int cc = 0;   // chunks processed by this warp so far: staging tile cc & 1
     int local = 0;
-    for (int tile = pair; tile < num_tiles; tile += npairs, ++local) {
+    bool failed = false;
+    for (int tile = pair; tile < num_tiles && !failed; tile += npairs, ++local) {
       const int acc = local & 1;
       const uint32_t acc_phase = (local >> 1) & 1;
-      if (!ptx::mbar_wait_bounded(tfull_bar(acc), acc_phase, abort, WAIT_LIMIT_NS)) {
-        if (!*abort) record_timeout(err, WHERE_GEMM_EPILOGUE, abort);
-        break;
-      }
-      ptx::tc_fence_after();
       const int m_blk = tile % num_m_tiles, n_blk = tile / num_m_tiles;
       const int row0 = m_blk * 2 * BMC + (int)rank * BMC + quarter * 32;
       const int cbeg = min(part * C::PART_CH * CW, BN);
       const int cend = min(cbeg + C::PART_CH * CW, BN);
       const int valid_end = min(cend, ep.N - n_blk * BN);
-      const int nch = valid_end > cbeg ? (valid_end - cbeg + CW - 1) / CW : 0;
-      const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * BN + cbeg;
+      // a warp whose 32 rows all lie past M issues no loads or stores for this tile
+      const int nch = (valid_end > cbeg && row0 < ep.M) ? (valid_end - cbeg + CW - 1) / CW : 0;
       const int gcol = n_blk * BN + cbeg;
+      // chunk k of this tile is the warp's chunk number cc0 + k and uses staging tile (cc0 + k) % NBUF
+      const int cc0 = cc;
+      auto stage_tile = [&](int a) { return stg_base + (a % C::NBUF) * C::STG_BYTES; };
+      auto load_bias = [&](int k, float4 (&b4)[CW / 4]) {
+#pragma unroll
+        for (int j = 0; j < CW / 4; ++j) b4[j] = ld4(ep.bias + gcol + k * CW + 4 * j);
+      };
+      float4 ba[CW / 4], bb[CW / 4];
+      if (nch > 0) {
+        if (KIND == EPI_BIAS_RESID && lane == 0) {
+          // the whole residual share of this tile, one staging tile per chunk, loaded while
+          // the MMAs run; the previous tile's stores have read their staging tiles first
+          ptx::bulk_wait_read<0>();
+          for (int k = 0; k < nch; ++k) {
+            const int b = (cc0 + k) % C::NBUF;
+            ptx::mbar_arrive_expect_tx(res_bar(ew, b), 32 * CW * 4);
+            ptx::tma_load_2d(ptx::smem_u32(stage_tile(cc0 + k)), &tmR, res_bar(ew, b), gcol + k * CW, row0);
+          }
+        }
+        load_bias(0, ba);
+      }
+      if (!ptx::mbar_wait_bounded(tfull_bar(acc), acc_phase, abort, WAIT_LIMIT_NS)) {
+        if (!*abort) record_timeout(err, WHERE_GEMM_EPILOGUE, abort);
+        failed = true;
+        break;
+      }
+      ptx::tc_fence_after();
+      const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * BN + cbeg;
       auto release = [&]() {
         ptx::tc_fence_before();
         __syncwarp();
@@ -237,38 +274,74 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
         release();
         continue;
       }
-      float va[CW], vb[CW];
-      float4 pa[PASSES], pb[PASSES];
-      float4 ba, bb;
-      auto process = [&](float (&v)[CW], const float4 (&pre)[PASSES], const float4 bias4, int c) {
+      // finish chunk k (the warp's chunk number cc == cc0 + k) from accumulator values v, bias b4
+      auto process = [&](float (&v)[CW], const float4 (&b4)[CW / 4], int k) -> bool {
+        uint8_t* st = stage_tile(cc);
+        float x[CW];
 #pragma unroll
-        for (int j = 0; j < CW; j += 4)
-          *reinterpret_cast<float4*>(st + lane * (CW + 4) + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+        for (int j = 0; j < CW / 4; ++j) {
+          x[4 * j] = v[4 * j] + b4[j].x;
+          x[4 * j + 1] = v[4 * j + 1] + b4[j].y;
+          x[4 * j + 2] = v[4 * j + 2] + b4[j].z;
+          x[4 * j + 3] = v[4 * j + 3] + b4[j].w;
+        }
+        if constexpr (KIND == EPI_BIAS_GELU) {
+#pragma unroll
+          for (int j = 0; j < CW; ++j) x[j] = gelu_erf(x[j]);
+        }
+        if constexpr (KIND == EPI_BIAS_SILU) {
+#pragma unroll
+          for (int j = 0; j < CW; ++j) x[j] = silu_f(x[j]);
+        }
+        if constexpr (KIND == EPI_BIAS_RESID) {
+          if (!ptx::mbar_wait_bounded(res_bar(ew, cc % C::NBUF), (cc / C::NBUF) & 1, abort, WAIT_LIMIT_NS))
+            return false;
+          const float* rrow = reinterpret_cast<const float*>(st) + lane * CW;
+#pragma unroll
+          for (int j = 0; j < CW / 4; ++j) {
+            const float4 r = *reinterpret_cast<const float4*>(rrow + 4 * j);
+            x[4 * j] += r.x; x[4 * j + 1] += r.y; x[4 * j + 2] += r.z; x[4 * j + 3] += r.w;
+          }
+        } else {
+          if (lane == 0) ptx::bulk_wait_read<1>();   // store of chunk cc - 2 has read this tile
+          __syncwarp();
+        }
+        OutT* orow = reinterpret_cast<OutT*>(st) + lane * CW;
+#pragma unroll
+        for (int j = 0; j < CW; j += 4) store4<OutT>(orow + j, x[j], x[j + 1], x[j + 2], x[j + 3]);
+        ptx::fence_proxy_async_smem();
         __syncwarp();
-        epilogue_warp_tile<KIND, OutT, CW>(ep, st, row0, gcol + c * CW, lane, pre, bias4);
-        __syncwarp();
+        if (lane == 0) {
+          ptx::tma_store_2d(&tmO, ptx::smem_u32(st), gcol + k * CW, row0);
+          ptx::bulk_commit();
+        }
+        ++cc;
+        return true;
       };
-      epilogue_prefetch<KIND, CW>(ep, row0, gcol, lane, pa, ba);
+      float va[CW], vb[CW];
       ptx::tmem_ld(taddr, va);
 #pragma unroll 1
       for (int c = 0; c < nch; c += 2) {
         ptx::tmem_ld_wait();
         if (c == nch - 1) release();
         if (c + 1 < nch) {
-          epilogue_prefetch<KIND, CW>(ep, row0, gcol + (c + 1) * CW, lane, pb, bb);
           ptx::tmem_ld(taddr + (c + 1) * CW, vb);
+          load_bias(c + 1, bb);
         }
-        process(va, pa, ba, c);
+        if (!process(va, ba, c)) { failed = true; break; }
         if (c + 1 >= nch) break;
         ptx::tmem_ld_wait();
         if (c + 1 == nch - 1) release();
         if (c + 2 < nch) {
-          epilogue_prefetch<KIND, CW>(ep, row0, gcol + (c + 2) * CW, lane, pa, ba);
           ptx::tmem_ld(taddr + (c + 2) * CW, va);
+          load_bias(c + 2, ba);
         }
-        process(vb, pb, bb, c + 1);
+        if (!process(vb, bb, c + 1)) { failed = true; break; }
       }
+      if (failed && !*abort) record_timeout(err, WHERE_GEMM_EPILOGUE, abort);
     }
+    if (lane == 0) ptx::bulk_wait_all();
+    __syncwarp();
   }
 
   // both CTAs finish every access to the pair's shared memory and TMEM before either leaves
@@ -287,7 +360,7 @@ template <int BN, int STAGES, int KIND, typename OutT>
 struct Tc2Launcher {
   static int max_clusters;
   static cudaError_t prepare() {
-    using Cf = Tc2Cfg<BN, STAGES>;
+    using Cf = Tc2Cfg<BN, STAGES, KIND>;
     auto kern = gemm_tc2_kernel<BN, STAGES, KIND, OutT>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cf::SMEM);
     if (e != cudaSuccess) return e;
@@ -314,11 +387,17 @@ struct Tc2Launcher {
     return cudaSuccess;
   }
   static cudaError_t launch(const GemmArgs& g, const EpiParams& ep, DevError* err, cudaStream_t st) {
-    using Cf = Tc2Cfg<BN, STAGES>;
+    using Cf = Tc2Cfg<BN, STAGES, KIND>;
     if (max_clusters < 1) return cudaErrorInvalidConfiguration;
-    CUtensorMap ta, tb;
+    CUtensorMap ta, tb, to, tr;
     if (make_tmap_bf16(&ta, g.A, g.M, g.K, g.lda, BMC) || make_tmap_bf16(&tb, g.B, g.N, g.K, g.ldb, BN / 2))
       return cudaErrorInvalidValue;
+    if (make_tmap_plain(&to, ep.out, (int)sizeof(OutT), g.M, g.N, ep.ldo, Cf::CW, 32)) return cudaErrorInvalidValue;
+    if (KIND == EPI_BIAS_RESID) {
+      if (make_tmap_plain(&tr, ep.resid, 4, g.M, g.N, ep.ldr, Cf::CW, 32)) return cudaErrorInvalidValue;
+    } else {
+      tr = to;
+    }
     const int mt = (g.M + 2 * BMC - 1) / (2 * BMC), nt = (g.N + BN - 1) / BN;
     const int tiles = mt * nt;
     const int pairs = tiles < max_clusters ? tiles : max_clusters;
@@ -336,8 +415,8 @@ struct Tc2Launcher {
     cfg.stream = st;
     cfg.attrs = attr;
     cfg.numAttrs = pdl_enabled() ? 2 : 1;
-    return cudaLaunchKernelEx(&cfg, gemm_tc2_kernel<BN, STAGES, KIND, OutT>, ta, tb, mt, nt, (g.K + BK - 1) / BK,
-                              ep, err);
+    return cudaLaunchKernelEx(&cfg, gemm_tc2_kernel<BN, STAGES, KIND, OutT>, ta, tb, to, tr, mt, nt,
+                              (g.K + BK - 1) / BK, ep, err);
   }
 };
 template <int BN, int STAGES, int KIND, typename OutT>
@@ -350,8 +429,7 @@ int Tc2Launcher<BN, STAGES, KIND, OutT>::max_clusters = 0;
   X(160, 7, EPI_BIAS, bf16) X(144, 7, EPI_BIAS, bf16)   \
   X(256, 6, EPI_BIAS_GELU, bf16) X(208, 6, EPI_BIAS_GELU, bf16) \
   X(160, 7, EPI_BIAS_GELU, bf16) X(144, 7, EPI_BIAS_GELU, bf16) \
-  X(256, 6, EPI_BIAS_RESID, float) X(208, 6, EPI_BIAS_RESID, float) \
-  X(160, 7, EPI_BIAS_RESID, float) X(144, 7, EPI_BIAS_RESID, float)
+  X(160, 5, EPI_BIAS_RESID, float) X(144, 5, EPI_BIAS_RESID, float)
 
 }  // namespace
 
@@ -371,18 +449,24 @@ bool gemm_tc2_supports(int kind, bool out_f32) {
          (kind == EPI_BIAS_RESID && out_f32);
 }
 
-// Tile N minimizing (rounds of pair tiles) x N over the available CTA pairs.
-int gemm_tc2_pick_bn(int M, int N) {
-  const int cands[4] = {256, 208, 160, 144};
+// Tile N minimizing (rounds of pair tiles) x (N + per-tile overhead) over the available
+// CTA pairs; the overhead (prologue, pipeline fill, last epilogue) was measured to be worth
+// about 160 columns of MMA time per tile at K = 1024.
+int gemm_tc2_pick_bn(int M, int N, int kind) {
+  const int all[4] = {256, 208, 160, 144};
+  const int resid[2] = {160, 144};
+  const int* cands = kind == EPI_BIAS_RESID ? resid : all;
+  const int ncand = kind == EPI_BIAS_RESID ? 2 : 4;
   const int pairs = Tc2Launcher<256, 6, EPI_BIAS, bf16>::max_clusters > 0
                         ? Tc2Launcher<256, 6, EPI_BIAS, bf16>::max_clusters : 74;
   const long mt = (M + 2 * BMC - 1) / (2 * BMC);
-  int best = 256;
+  int best = cands[0];
   long best_cost = -1;
-  for (int bn : cands) {
+  for (int i = 0; i < ncand; ++i) {
+    const int bn = cands[i];
     const long tiles = mt * ((N + bn - 1) / bn);
     const long rounds = (tiles + pairs - 1) / pairs;
-    const long cost = rounds * bn;
+    const long cost = rounds * (bn + 160);
     if (best_cost < 0 || cost < best_cost) {
       best_cost = cost;
       best = bn;
@@ -394,7 +478,7 @@ int gemm_tc2_pick_bn(int M, int N) {
 cudaError_t gemm_tc2(const GemmArgs& g, int bn, int kind, bool out_f32, const EpiParams& ep, DevError* err,
                      cudaStream_t st) {
   if (g.M <= 0 || g.N <= 0) return cudaSuccess;
-  if (g.K <= 0) return cudaErrorInvalidValue;
+  if (g.K <= 0 || g.N % 16) return cudaErrorInvalidValue;
 #define KD_RUN(BN_, ST_, KIND_, OUT_)                                                   \
   if (bn == BN_ && kind == KIND_ && out_f32 == std::is_same<OUT_, float>::value)        \
     return Tc2Launcher<BN_, ST_, KIND_, OUT_>::launch(g, ep, err, st);

@@ -25,14 +25,17 @@ bool gemm_tc_available();
 // TMA descriptor of a row-major bf16 matrix [rows, ld] whose first `cols` columns are
 // the K extent; boxes of 64 columns x box_rows rows, 128-byte swizzle, zero fill.
 int make_tmap_bf16(CUtensorMap* m, const void* base, int rows, int cols, int ld, int box_rows);
+// Row-major fp32 (elem 4) or bf16 (elem 2) matrix, boxes box_cols x box_rows, no swizzle.
+int make_tmap_plain(CUtensorMap* m, const void* base, int elem, int rows, int cols, long ld, int box_cols,
+                    int box_rows);
 
-// tcgen05 GEMM on CTA pairs (256-row tiles).  bn in {144, 160, 208, 256}; kinds
-// EPI_BIAS / EPI_BIAS_GELU with bf16 output and EPI_BIAS_RESID with fp32 output.
+// tcgen05 GEMM on CTA pairs (256-row tiles).  bn in {144, 160, 208, 256} for EPI_BIAS /
+// EPI_BIAS_GELU with bf16 output, {144, 160} for EPI_BIAS_RESID with fp32 output.
 cudaError_t gemm_tc2(const GemmArgs& g, int bn, int kind, bool out_f32, const EpiParams& ep, DevError* err,
                      cudaStream_t st);
 cudaError_t gemm_tc2_prepare();
 bool gemm_tc2_supports(int kind, bool out_f32);
-int gemm_tc2_pick_bn(int M, int N);
+int gemm_tc2_pick_bn(int M, int N, int kind);
 // Set the dynamic shared-memory limits of every kernel instantiation (call once
 // per device before any launch or graph capture).
 cudaError_t gemm_tc_prepare();
