@@ -161,8 +161,11 @@ KIMODO_API int kimodo_ddim_sample(kimodo_ctx* ctx, const float* text_emb, const 
 KIMODO_API int kimodo_sync_status(kimodo_ctx* ctx, void* stream);
 
 /* Per-kernel-class timing of the next calls (instrumentation, off by default).
- * With enable != 0, kimodo_ddim_sample runs eagerly (no graph) and brackets every
- * launch with CUDA events; kimodo_profile_read() returns, for each of
+ * With enable != 0, every launch is bracketed by CUDA events; kimodo_ddim_sample
+ * then captures a fresh, uncached graph whose kernel nodes sit between timing
+ * event nodes (so the times carry no host gaps, but consecutive kernels no longer
+ * overlap through programmatic dependent launch), runs it and waits for it.
+ * kimodo_profile_read() returns, for each of
  * n_classes <= 8 classes (0 tensor-core GEMM, 1 attention, 2 LayerNorm,
  * 3 elementwise/motion, 4 fp32 GEMM, 5 setup), the summed milliseconds, the
  * number of launches and the algorithmic FLOPs and bytes since the last reset. */

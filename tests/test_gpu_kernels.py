@@ -154,6 +154,30 @@ def test_gelu_epilogue_error_bound():
     assert np.all(np.abs(got - ref) <= bound), float(np.max(np.abs(got - ref) - bound))
 
 
+@pytest.mark.parametrize("pair,tile", [(False, 128), (True, 160)])
+def test_gelu_bf16_epilogue_error_bound(pair, tile):
+    """GELU of the bf16-output tensor-core epilogues against the exact erf GELU on a
+    dense grid.  erf there is Abramowitz & Stegun 7.1.28 (|error| <= 3e-7) with an
+    approximate reciprocal raised to the 16th power (relative error <= 16 * 2^-22),
+    so with fp32 evaluation |GELU error| <= 0.5 |x| * 8e-6 before the result is rounded to bf16 (half an
+    ulp of 8 significant bits)."""
+    require_cuda()
+    x = torch.linspace(-9, 9, 4096).to(torch.bfloat16)
+    A = torch.zeros((x.numel(), 64), dtype=torch.bfloat16)
+    A[:, 0] = x
+    W = torch.zeros((16, 64), dtype=torch.bfloat16)
+    W[:, 0] = 1.0
+    out = kb.gemm_bf16(A.cuda(), W.cuda(), torch.zeros(16, device="cuda"), kb.EPI_BIAS_GELU, False,
+                       tile_n=tile, pair=pair)
+    torch.cuda.synchronize()
+    got = out.float().cpu().double().numpy()
+    xd = x.double().numpy()
+    ref = ko.gelu(xd)[:, None]
+    err = 0.5 * np.abs(xd)[:, None] * 8e-6
+    bound = 2.0 ** -8 * np.abs(ref) + 1.01 * err + 1e-30
+    assert np.all(np.abs(got - ref) <= bound), float(np.max(np.abs(got - ref) - bound))
+
+
 def _attention_ref(qkv, lengths, S):
     nseq = len(lengths)
     out = np.zeros((nseq * S, 1024))

@@ -100,6 +100,7 @@ struct kimodo_ctx {
   cudaStream_t cap_stream = nullptr;
   std::map<std::tuple<int, int, int, int, uint32_t>, std::pair<cudaGraphExec_t, long long>> graphs;
   bool profiling = false;
+  unsigned prof_flags = cudaEventRecordDefault;   // cudaEventRecordExternal while a profiled graph is captured
   std::vector<ProfRec> prof;
   std::vector<cudaEvent_t> ev_pool;
   size_t ev_used = 0;
@@ -130,12 +131,12 @@ int launch(kimodo_ctx* c, int cls, double flops, double bytes, cudaStream_t st, 
   if (c->profiling) {
     a = next_event(c);
     b = next_event(c);
-    if (a && b) cudaEventRecord(a, st);
+    if (a && b) cudaEventRecordWithFlags(a, st, c->prof_flags);
   }
   cudaError_t e = fn();
   if (e != cudaSuccess) return set_error(KIMODO_ECUDA, "launch of %s failed: %s", what, cudaGetErrorString(e));
   if (c->profiling && a && b) {
-    cudaEventRecord(b, st);
+    cudaEventRecordWithFlags(b, st, c->prof_flags);
     c->prof.push_back({a, b, cls, flops, bytes});
   }
   return KIMODO_OK;
@@ -687,7 +688,28 @@ int kimodo_ddim_sample(kimodo_ctx* c, const float* text_emb, const float* null_e
   KD_CUDA(cudaMemcpyAsync(w.st_null, null_emb, (size_t)null_batch * DTXT * 4, cudaMemcpyDefault, st));
   const long long l0 = c->launches;
   if (c->profiling) {
-    KD_TRY(enqueue_sample(c, batch, frames, steps, cfg_scale, null_batch, st));
+    // The profiled generation runs as a graph too, with a timing event node on
+    // each side of every kernel node, so per-kernel times carry no host gaps.
+    // The graph is not cached: its event nodes belong to this profile.
+    KD_CUDA(cudaStreamBeginCapture(c->cap_stream, cudaStreamCaptureModeThreadLocal));
+    c->prof_flags = cudaEventRecordExternal;
+    int s = enqueue_sample(c, batch, frames, steps, cfg_scale, null_batch, c->cap_stream);
+    c->prof_flags = cudaEventRecordDefault;
+    cudaGraph_t g = nullptr;
+    cudaError_t e = cudaStreamEndCapture(c->cap_stream, &g);
+    if (s != KIMODO_OK) {
+      if (g) cudaGraphDestroy(g);
+      return s;
+    }
+    if (e != cudaSuccess) return set_error(KIMODO_ECUDA, "graph capture failed: %s", cudaGetErrorString(e));
+    cudaGraphExec_t ge;
+    e = cudaGraphInstantiate(&ge, g, 0);
+    cudaGraphDestroy(g);
+    if (e != cudaSuccess) return set_error(KIMODO_ECUDA, "graph instantiate failed: %s", cudaGetErrorString(e));
+    e = cudaGraphLaunch(ge, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    cudaGraphExecDestroy(ge);
+    if (e != cudaSuccess) return set_error(KIMODO_ECUDA, "profiled graph failed: %s", cudaGetErrorString(e));
     c->last_launches = c->launches - l0;
   } else {
     uint32_t cfg_bits;

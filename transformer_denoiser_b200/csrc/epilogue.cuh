@@ -6,6 +6,8 @@
 // of a sequence is the condition token, token j >= 1 is frame j - 1.
 #pragma once
 
+#include <type_traits>
+
 #include "common.cuh"
 
 namespace kd {
@@ -58,6 +60,66 @@ __device__ __forceinline__ float gelu_erf(float x) {
   return 0.5f * x * (1.0f + erf_as7126(x * 0.70710678118654752f));
 }
 __device__ __forceinline__ float silu_f(float x) { return x / (1.0f + expf(-x)); }
+
+// ---- packed fp32 pairs (sm_100 f32x2 arithmetic: two lanes of work per instruction)
+__device__ __forceinline__ uint64_t pk2(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ void upk2(uint64_t r, float& a, float& b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(r));
+}
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ float rcp_approx(float x) {
+  float r;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r;
+}
+
+// GELU of two values for the bf16-output tensor-core epilogues, with erf by
+// Abramowitz & Stegun formula 7.1.28: for z >= 0,
+//   erf(z) = 1 - (1 + a1 z + a2 z^2 + ... + a6 z^6)^-16,  |error| <= 3e-7,
+// so GELU(x) = x - h for x >= 0 and h for x < 0, h = 0.5 x (1 + a1|z| + ...)^-16,
+// z = x / sqrt 2.  One approximate reciprocal (relative error ~2^-22, x16 by the
+// power) and f32x2 arithmetic; the total, a few 1e-6 of |x|, is far below the
+// bf16 rounding of the stored result.
+__device__ __forceinline__ void gelu2_as7128(float& x0, float& x1) {
+  const uint64_t x = pk2(x0, x1);
+  const uint64_t a = mul2(x, pk2(0.70710678118654752f, 0.70710678118654752f)) & 0x7FFFFFFF7FFFFFFFull;
+  uint64_t p = fma2(a, pk2(0.0000430638f, 0.0000430638f), pk2(0.0002765672f, 0.0002765672f));
+  p = fma2(p, a, pk2(0.0001520143f, 0.0001520143f));
+  p = fma2(p, a, pk2(0.0092705272f, 0.0092705272f));
+  p = fma2(p, a, pk2(0.0422820123f, 0.0422820123f));
+  p = fma2(p, a, pk2(0.0705230784f, 0.0705230784f));
+  p = fma2(p, a, pk2(1.0f, 1.0f));
+  float p0, p1;
+  upk2(p, p0, p1);
+  uint64_t r = pk2(rcp_approx(p0), rcp_approx(p1));
+  r = mul2(r, r);
+  r = mul2(r, r);
+  r = mul2(r, r);
+  r = mul2(r, r);
+  const uint64_t h = mul2(mul2(x, pk2(0.5f, 0.5f)), r);
+  float h0, h1;
+  upk2(h, h0, h1);
+  x0 = x0 >= 0.f ? x0 - h0 : h0;
+  x1 = x1 >= 0.f ? x1 - h1 : h1;
+}
 
 template <typename T> __device__ __forceinline__ float to_f(T v);
 template <> __device__ __forceinline__ float to_f<float>(float v) { return v; }
@@ -167,6 +229,12 @@ __device__ __forceinline__ void store4<bf16>(bf16* p, float a, float b, float c,
 
 __device__ __forceinline__ float4 ld4(const float* p) { return *reinterpret_cast<const float4*>(p); }
 
+// Eight values as one 16-byte unit: fp32 stores two units of four, bf16 one unit of eight.
+__device__ __forceinline__ uint32_t bf16x2_bits(float a, float b) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
 template <int CW>
 struct EpiLanes {
   static constexpr int LDE = CW + 4;
@@ -253,9 +321,18 @@ __device__ __forceinline__ void epilogue_warp_tile(const EpiParams& e, const flo
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           float x = v[j] + b4[j];
-          if constexpr (KIND == EPI_BIAS_GELU) x = gelu_erf(x);
           if constexpr (KIND == EPI_BIAS_SILU) x = silu_f(x);
           v[j] = x;
+        }
+        if constexpr (KIND == EPI_BIAS_GELU) {
+          // bf16 outputs take the packed GELU of the pair GEMM, fp32 outputs the A&S 7.1.26 one
+          if constexpr (std::is_same<OutT, bf16>::value) {
+            gelu2_as7128(v[0], v[1]);
+            gelu2_as7128(v[2], v[3]);
+          } else {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) v[j] = gelu_erf(v[j]);
+          }
         }
         if constexpr (KIND == EPI_BIAS_RESID) {
           v[0] += pre[p].x; v[1] += pre[p].y; v[2] += pre[p].z; v[3] += pre[p].w;

@@ -335,19 +335,26 @@ int make_tmap_bf16(CUtensorMap* m, const void* base, int rows, int cols, int ld,
 
 
 // Row-major matrix [rows, ld] of fp32 (elem 4) or bf16 (elem 2), K extent `cols`,
-// boxes of box_cols x box_rows, no swizzle (epilogue staging tiles).
+// boxes of box_cols x box_rows (epilogue staging tiles), shared-memory swizzle of
+// 0 (none), 32, 64 or 128 bytes; a swizzled box row must span exactly that many bytes.
 int make_tmap_plain(CUtensorMap* m, const void* base, int elem, int rows, int cols, long ld, int box_cols,
-                    int box_rows) {
+                    int box_rows, int swizzle) {
   EncodeTiledFn enc = get_encode_fn();
   if (!enc) return -1;
   if ((reinterpret_cast<uintptr_t>(base) & 15) || (ld * elem) % 16 || (box_cols * elem) % 16) return -2;
+  CUtensorMapSwizzle sw = CU_TENSOR_MAP_SWIZZLE_NONE;
+  if (swizzle == 32) sw = CU_TENSOR_MAP_SWIZZLE_32B;
+  else if (swizzle == 64) sw = CU_TENSOR_MAP_SWIZZLE_64B;
+  else if (swizzle == 128) sw = CU_TENSOR_MAP_SWIZZLE_128B;
+  else if (swizzle != 0) return -2;
+  if (swizzle != 0 && box_cols * elem != swizzle) return -2;
   cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
   cuuint64_t strides[1] = {(cuuint64_t)ld * elem};
   cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = enc(m, elem == 4 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
                    const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                   CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                   sw, CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? 0 : -3;
 }
 

@@ -49,6 +49,8 @@ struct Tc2Cfg {
   static constexpr int NCH = BN / CW;
   static constexpr int PART_CH = (NCH + 1) / 2;
   static constexpr uint32_t STG_BYTES = 32 * CW * 4;     // one 32-row staging tile (fp32 size)
+  // bytes of one staging row of the stored type (fp32 64, bf16 32): also the TMA swizzle span
+  static constexpr int ROW_BYTES = CW * (KIND == EPI_BIAS_RESID ? 4 : 2);
   // staging tiles per epilogue warp: two alternating ones, or, with a residual, one per
   // chunk of the warp's tile share so the whole residual share is loaded ahead of the MMA
   static constexpr int NBUF = KIND == EPI_BIAS_RESID ? PART_CH : 2;
@@ -214,7 +216,7 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
     // ---------------- epilogue warps 2..9: TMEM lane quarter = warp % 4; part (warp - 2) / 4
     // takes chunks [part * PART_CH, ...) of the tile's BN / 16 column chunks.  Per chunk each
     // thread finishes its accumulator row (bias, activation, residual) in registers and
-    // writes it into a dense 32 x 16 staging tile; one lane stores the tile with TMA.  Two
+    // writes it into a swizzled 32 x 16 staging tile; one lane stores the tile with TMA.  Two
     // staging tiles per warp alternate; the residual chunk arrives in the staging tile by TMA.
     const int quarter = warp & 3;
     const int ew = warp - 2;
@@ -277,6 +279,10 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
       // finish chunk k (the warp's chunk number cc == cc0 + k) from accumulator values v, bias b4
       auto process = [&](float (&v)[CW], const float4 (&b4)[CW / 4], int k) -> bool {
         uint8_t* st = stage_tile(cc);
+        // this lane's row of the staging tile; its 16-byte unit u sits at unit u ^ swz
+        // (the tile's TMA swizzle, so that the warp's row-per-lane accesses hit distinct banks)
+        uint8_t* srow = st + lane * C::ROW_BYTES;
+        const int swz = C::ROW_BYTES == 64 ? (lane >> 1) & 3 : (lane >> 2) & 1;
         float x[CW];
 #pragma unroll
         for (int j = 0; j < CW / 4; ++j) {
@@ -287,7 +293,7 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
         }
         if constexpr (KIND == EPI_BIAS_GELU) {
 #pragma unroll
-          for (int j = 0; j < CW; ++j) x[j] = gelu_erf(x[j]);
+          for (int j = 0; j < CW; j += 2) gelu2_as7128(x[j], x[j + 1]);
         }
         if constexpr (KIND == EPI_BIAS_SILU) {
 #pragma unroll
@@ -296,19 +302,27 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
         if constexpr (KIND == EPI_BIAS_RESID) {
           if (!ptx::mbar_wait_bounded(res_bar(ew, cc % C::NBUF), (cc / C::NBUF) & 1, abort, WAIT_LIMIT_NS))
             return false;
-          const float* rrow = reinterpret_cast<const float*>(st) + lane * CW;
 #pragma unroll
-          for (int j = 0; j < CW / 4; ++j) {
-            const float4 r = *reinterpret_cast<const float4*>(rrow + 4 * j);
-            x[4 * j] += r.x; x[4 * j + 1] += r.y; x[4 * j + 2] += r.z; x[4 * j + 3] += r.w;
+          for (int u = 0; u < CW / 4; ++u) {
+            const float4 r = *reinterpret_cast<const float4*>(srow + ((u ^ swz) << 4));
+            x[4 * u] += r.x; x[4 * u + 1] += r.y; x[4 * u + 2] += r.z; x[4 * u + 3] += r.w;
           }
         } else {
           if (lane == 0) ptx::bulk_wait_read<1>();   // store of chunk cc - 2 has read this tile
           __syncwarp();
         }
-        OutT* orow = reinterpret_cast<OutT*>(st) + lane * CW;
+        if constexpr (std::is_same<OutT, float>::value) {
 #pragma unroll
-        for (int j = 0; j < CW; j += 4) store4<OutT>(orow + j, x[j], x[j + 1], x[j + 2], x[j + 3]);
+          for (int u = 0; u < CW / 4; ++u)
+            *reinterpret_cast<float4*>(srow + ((u ^ swz) << 4)) =
+                make_float4(x[4 * u], x[4 * u + 1], x[4 * u + 2], x[4 * u + 3]);
+        } else {
+#pragma unroll
+          for (int u = 0; u < CW / 8; ++u)
+            *reinterpret_cast<uint4*>(srow + ((u ^ swz) << 4)) =
+                make_uint4(bf16x2_bits(x[8 * u], x[8 * u + 1]), bf16x2_bits(x[8 * u + 2], x[8 * u + 3]),
+                           bf16x2_bits(x[8 * u + 4], x[8 * u + 5]), bf16x2_bits(x[8 * u + 6], x[8 * u + 7]));
+        }
         ptx::fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
@@ -392,9 +406,11 @@ struct Tc2Launcher {
     CUtensorMap ta, tb, to, tr;
     if (make_tmap_bf16(&ta, g.A, g.M, g.K, g.lda, BMC) || make_tmap_bf16(&tb, g.B, g.N, g.K, g.ldb, BN / 2))
       return cudaErrorInvalidValue;
-    if (make_tmap_plain(&to, ep.out, (int)sizeof(OutT), g.M, g.N, ep.ldo, Cf::CW, 32)) return cudaErrorInvalidValue;
+    static_assert(Cf::ROW_BYTES == Cf::CW * (int)sizeof(OutT), "staging row bytes");
+    if (make_tmap_plain(&to, ep.out, (int)sizeof(OutT), g.M, g.N, ep.ldo, Cf::CW, 32, Cf::ROW_BYTES))
+      return cudaErrorInvalidValue;
     if (KIND == EPI_BIAS_RESID) {
-      if (make_tmap_plain(&tr, ep.resid, 4, g.M, g.N, ep.ldr, Cf::CW, 32)) return cudaErrorInvalidValue;
+      if (make_tmap_plain(&tr, ep.resid, 4, g.M, g.N, ep.ldr, Cf::CW, 32, Cf::ROW_BYTES)) return cudaErrorInvalidValue;
     } else {
       tr = to;
     }

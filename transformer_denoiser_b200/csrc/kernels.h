@@ -25,9 +25,10 @@ bool gemm_tc_available();
 // TMA descriptor of a row-major bf16 matrix [rows, ld] whose first `cols` columns are
 // the K extent; boxes of 64 columns x box_rows rows, 128-byte swizzle, zero fill.
 int make_tmap_bf16(CUtensorMap* m, const void* base, int rows, int cols, int ld, int box_rows);
-// Row-major fp32 (elem 4) or bf16 (elem 2) matrix, boxes box_cols x box_rows, no swizzle.
+// Row-major fp32 (elem 4) or bf16 (elem 2) matrix, boxes box_cols x box_rows,
+// shared-memory swizzle 0, 32, 64 or 128 bytes (= the box row's bytes when nonzero).
 int make_tmap_plain(CUtensorMap* m, const void* base, int elem, int rows, int cols, long ld, int box_cols,
-                    int box_rows);
+                    int box_rows, int swizzle);
 
 // tcgen05 GEMM on CTA pairs (256-row tiles).  bn in {144, 160, 208, 256} for EPI_BIAS /
 // EPI_BIAS_GELU with bf16 output, {144, 160} for EPI_BIAS_RESID with fp32 output.
