@@ -30,8 +30,11 @@ design notes of the repository):
 
 * x0-prediction: both networks predict the clean sample.
 * Linear beta schedule 1e-4..0.02 over 1000 steps (the "Model details" table
-  says "cosine"; the workloads fix linear).  Trailing timesteps
-  t_k = 999 - k*(1000/steps); alphabar(-1) = 1.  eta = 0.
+  says "cosine"; the workloads fix linear); the cosine schedule is the option
+  of Nichol & Dhariwal (2021).  Trailing timesteps
+  t_k = 999 - k*(1000/steps) when steps divides 1000, in general
+  t_k = floor(1000 (steps - k) / steps + 1/2) - 1; alphabar(-1) = 1.  eta = 0
+  by default; eta > 0 takes the caller's per-step standard-normal draws.
 * Condition token at sequence position 0 = Linear(4096->1024)(embedding)
   + MLP(sinusoid(t)) with MLP = Linear -> SiLU -> Linear; frame j is token
   j+1.  A fixed interleaved sinusoid (sin at even, cos at odd features) is
@@ -312,6 +315,27 @@ def ddim_timesteps(steps: int, n: int = N_TRAIN_STEPS):
     return [(n - 1 - k * stride, n - 1 - (k + 1) * stride) for k in range(steps)]
 
 
+def alphabar_cosine(n: int = N_TRAIN_STEPS, s: float = 0.008, max_beta: float = 0.999):
+    """Cosine schedule (Nichol & Dhariwal, "Improved Denoising Diffusion Probabilistic
+    Models", 2021, eq. 17): alphabar(u) = f(u) / f(0), f(u) = cos^2((u + s) / (1 + s) * pi/2)
+    for u in [0, 1].  Discretised as in that paper: beta_i = min(1 - alphabar((i+1)/n) /
+    alphabar(i/n), max_beta), and the table is prod_{j<=i} (1 - beta_j) (float64)."""
+    def f(u):
+        return math.cos((u + s) / (1.0 + s) * math.pi / 2.0) ** 2
+    betas = np.array([min(1.0 - f((i + 1) / n) / f(i / n), max_beta) for i in range(n)], dtype=np.float64)
+    return np.cumprod(1.0 - betas)
+
+
+def ddim_timesteps_trailing(steps: int, n: int = N_TRAIN_STEPS):
+    """Trailing DDIM timesteps for any step count 1 <= steps <= n:
+    t_k = floor(n (steps - k) / steps + 1/2) - 1, t_prev_k = t_{k+1}, and -1 after the last.
+    Equal to ddim_timesteps when steps divides n."""
+    if steps < 1 or steps > n:
+        raise ValueError("steps must lie in [1, n]")
+    ts = [(2 * n * (steps - k) + steps) // (2 * steps) - 1 for k in range(steps)]
+    return [(ts[k], ts[k + 1] if k + 1 < steps else -1) for k in range(steps)]
+
+
 def alphabar_at(ab, t: int) -> float:
     return 1.0 if t < 0 else float(ab[t])
 
@@ -327,6 +351,25 @@ def ddim_update(x_t, x0, ab_t: float, ab_prev: float):
     x_prev = sqrt(ab_prev) x0 + sqrt(1 - ab_prev) eps."""
     eps = (x_t - math.sqrt(ab_t) * x0) / math.sqrt(1.0 - ab_t)
     return math.sqrt(ab_prev) * x0 + math.sqrt(1.0 - ab_prev) * eps
+
+
+def ddim_sigma(ab_t: float, ab_prev: float, eta: float) -> float:
+    """Per-step noise scale of DDIM (Song, Meng & Ermon, "Denoising Diffusion Implicit
+    Models", 2021, eq. 16): sigma = eta sqrt((1 - ab_prev) / (1 - ab_t)) sqrt(1 - ab_t / ab_prev)."""
+    return eta * math.sqrt((1.0 - ab_prev) / (1.0 - ab_t)) * math.sqrt(1.0 - ab_t / ab_prev)
+
+
+def ddim_update_eta(x_t, x0, ab_t: float, ab_prev: float, eta: float, z):
+    """Generalised DDIM step from an x0 prediction (same paper, eq. 12):
+    eps = (x_t - sqrt(ab_t) x0) / sqrt(1 - ab_t);
+    x_prev = sqrt(ab_prev) x0 + sqrt(1 - ab_prev - sigma^2) eps + sigma z,
+    with sigma from ddim_sigma and z the caller's standard-normal draw for this step."""
+    sigma = ddim_sigma(ab_t, ab_prev, eta)
+    eps = (x_t - math.sqrt(ab_t) * x0) / math.sqrt(1.0 - ab_t)
+    out = math.sqrt(ab_prev) * x0 + math.sqrt(1.0 - ab_prev - sigma * sigma) * eps
+    if sigma != 0.0:
+        out = out + sigma * np.asarray(z, dtype=np.float64)
+    return out
 
 
 # ---------------------------------------------------------------------------
@@ -350,11 +393,12 @@ def two_stage_predict(params, x_t, emb, t: int, length: int):
 
 
 def ddim_step(params, x_t, text_emb, null_emb, length: int, t: int, t_prev: int,
-              cfg_scale: float, ab=None, predictor=None):
+              cfg_scale: float, ab=None, predictor=None, eta: float = 0.0, z=None):
     """One two-stage DDIM step on one sequence.  Returns (x_prev, stages).
 
     predictor, if given, replaces the networks: predictor(x_t, t) -> (x0_cond,
-    x0_uncond).  It serves the closed-form checks of the sampler.
+    x0_uncond).  It serves the closed-form checks of the sampler.  eta > 0 adds
+    sigma z with the caller's draw z [T, 279] (ddim_update_eta).
     """
     ab = alphabar_linear() if ab is None else ab
     x_t = np.asarray(x_t, dtype=np.float64)
@@ -366,32 +410,42 @@ def ddim_step(params, x_t, text_emb, null_emb, length: int, t: int, t_prev: int,
         cond = unc = None
         xc, xu = (np.asarray(a, dtype=np.float64) for a in predictor(x_t, t))
     x0 = cfg_combine(xc, xu, cfg_scale)
-    x_prev = ddim_update(x_t, x0, alphabar_at(ab, t), alphabar_at(ab, t_prev))
+    if eta == 0.0:
+        x_prev = ddim_update(x_t, x0, alphabar_at(ab, t), alphabar_at(ab, t_prev))
+    else:
+        x_prev = ddim_update_eta(x_t, x0, alphabar_at(ab, t), alphabar_at(ab, t_prev), eta, z)
     x_prev[int(length):] = 0.0
     return x_prev, {"cond": cond, "uncond": unc, "x0": x0}
 
 
 def ddim_sample(params, text_emb, null_emb, noise, length: int, steps: int,
-                cfg_scale: float, predictor=None, trace=None):
-    """Full DDIM loop on one sequence from noise [T, 279]; returns the final x."""
-    ab = alphabar_linear()
+                cfg_scale: float, predictor=None, trace=None, schedule: str = "linear",
+                eta: float = 0.0, step_noise=None):
+    """Full DDIM loop on one sequence from noise [T, 279]; returns the final x.
+    schedule "linear" or "cosine"; any step count in [1, 1000] (trailing spacing);
+    eta > 0 draws step k's z from step_noise[k] [T, 279]."""
+    ab = alphabar_linear() if schedule == "linear" else alphabar_cosine()
     x = np.asarray(noise, dtype=np.float64)
-    for t, t_prev in ddim_timesteps(steps):
-        x, _ = ddim_step(params, x, text_emb, null_emb, length, t, t_prev, cfg_scale, ab, predictor)
+    for k, (t, t_prev) in enumerate(ddim_timesteps_trailing(steps)):
+        z = None if eta == 0.0 else step_noise[k]
+        x, _ = ddim_step(params, x, text_emb, null_emb, length, t, t_prev, cfg_scale, ab, predictor, eta, z)
         if trace is not None:
             trace.append(x.copy())
     return x
 
 
 def ddim_sample_batch(params, text_emb, null_emb, noise, lengths, steps: int, cfg_scale: float,
-                      indices=None):
+                      indices=None, schedule: str = "linear", eta: float = 0.0, step_noise=None):
     """Batch of independent sequences (null_emb [4096] or [B, 4096]).  Returns
-    {b: x_b} for the requested sequence indices (default: all)."""
+    {b: x_b} for the requested sequence indices (default: all).  step_noise, when
+    eta > 0, is [steps, B, T, 279]."""
     text_emb = np.asarray(text_emb)
     null_emb = np.asarray(null_emb)
     idx = range(text_emb.shape[0]) if indices is None else indices
     res = {}
     for b in idx:
         ne = null_emb if null_emb.ndim == 1 else null_emb[b]
-        res[b] = ddim_sample(params, text_emb[b], ne, noise[b], int(lengths[b]), steps, cfg_scale)
+        sn = None if step_noise is None else np.asarray(step_noise)[:, b]
+        res[b] = ddim_sample(params, text_emb[b], ne, noise[b], int(lengths[b]), steps, cfg_scale,
+                             schedule=schedule, eta=eta, step_noise=sn)
     return res

@@ -120,3 +120,32 @@ def test_layernorm_unbiased_variance_is_caught(monkeypatch):
         return (x - mu) / np.sqrt(var + eps) * g + b
     monkeypatch.setattr(ko, "layer_norm", wrong)
     _expect_fail(pins.test_layer_norm_vs_torch)
+
+
+def test_ddim_sigma_missing_root_is_caught(monkeypatch):
+    monkeypatch.setattr(ko, "ddim_sigma", lambda at, ap, eta: eta * math.sqrt((1 - ap) / (1 - at)) * (1 - at / ap))
+    _expect_fail(pins.test_ddim_eta_one_is_the_ddpm_posterior)
+
+
+def test_ddim_step_noise_sign_is_caught(monkeypatch):
+    real = ko.ddim_update_eta
+    monkeypatch.setattr(ko, "ddim_update_eta", lambda x_t, x0, at, ap, eta, z: real(x_t, x0, at, ap, eta, -np.asarray(z)))
+    _expect_fail(pins.test_ddim_eta_one_is_the_ddpm_posterior)
+
+
+def test_cosine_schedule_index_shift_is_caught(monkeypatch):
+    def shifted(n=1000, s=0.008, max_beta=0.999):
+        def f(u):
+            return math.cos((u + s) / (1.0 + s) * math.pi / 2.0) ** 2
+        betas = np.array([min(1.0 - f(i / n) / f(max(i - 1, 0) / n), max_beta) for i in range(n)])
+        return np.cumprod(1.0 - betas)
+    monkeypatch.setattr(ko, "alphabar_cosine", shifted)
+    _expect_fail(pins.test_cosine_schedule_telescopes)
+
+
+def test_timestep_rounding_down_is_caught(monkeypatch):
+    def floor_only(steps, n=1000):
+        ts = [n * (steps - k) // steps - 1 for k in range(steps)]
+        return [(ts[k], ts[k + 1] if k + 1 < steps else -1) for k in range(steps)]
+    monkeypatch.setattr(ko, "ddim_timesteps_trailing", floor_only)
+    _expect_fail(pins.test_trailing_timesteps_any_count)

@@ -381,6 +381,81 @@ def test_ddim_timesteps():
             ko.ddim_timesteps(bad)
 
 
+def test_cosine_schedule_telescopes():
+    """prod_{j<=i} (1 - beta_j) with beta_j = 1 - f((j+1)/n) / f(j/n) telescopes to
+    f((i+1)/n) / f(0) wherever no beta is clipped; only the last one is (f(1) = 0)."""
+    ab = ko.alphabar_cosine()
+    s = 0.008
+
+    def f(u):
+        return math.cos((u + s) / (1 + s) * math.pi / 2) ** 2
+    direct = np.array([f((i + 1) / 1000) / f(0.0) for i in range(1000)])
+    np.testing.assert_allclose(ab[:999], direct[:999], rtol=1e-11)
+    assert ab[999] == pytest.approx(ab[998] * (1 - 0.999), rel=1e-12)
+    assert np.all(np.diff(ab) < 0)
+    assert ab[499] == pytest.approx(0.49384, abs=1e-4)   # f(1/2) / f(0), worked by hand
+
+
+def test_trailing_timesteps_any_count():
+    # floor(1000 (15 - k) / 15 + 1/2) - 1, worked by hand
+    want = [999, 932, 866, 799, 732, 666, 599, 532, 466, 399, 332, 266, 199, 132, 66]
+    ts = ko.ddim_timesteps_trailing(15)
+    assert [t for t, _ in ts] == want and [tp for _, tp in ts] == want[1:] + [-1]
+    assert ko.ddim_timesteps_trailing(16)[3][0] == 812        # 812.5 + 1/2 rounds up to 813, minus 1
+    for steps in (1, 2, 4, 5, 8, 10, 20, 25, 40, 50, 100, 125, 200, 250, 500, 1000):
+        assert ko.ddim_timesteps_trailing(steps) == ko.ddim_timesteps(steps)
+    for steps in (3, 7, 16, 35, 999):
+        ts = ko.ddim_timesteps_trailing(steps)
+        t = [a for a, _ in ts]
+        assert len(ts) == steps and t[0] == 999 and t[-1] >= 0
+        assert all(a > b for a, b in zip(t, t[1:]))
+        assert all(tp == nxt for (_, tp), nxt in zip(ts, t[1:] + [-1]))
+    for bad in (0, 1001):
+        with pytest.raises(ValueError):
+            ko.ddim_timesteps_trailing(bad)
+
+
+def test_ddim_eta_zero_is_deterministic_ddim():
+    ab = ko.alphabar_linear()
+    rng = np.random.default_rng(31)
+    x_t, x0, z = rng.normal(size=(3, 7, 279))
+    for t, tp in [(999, 932), (400, 333), (66, -1)]:
+        ap = 1.0 if tp < 0 else ab[tp]
+        np.testing.assert_array_equal(ko.ddim_update_eta(x_t, x0, ab[t], ap, 0.0, z),
+                                      ko.ddim_update(x_t, x0, ab[t], ap))
+
+
+def test_ddim_eta_one_is_the_ddpm_posterior():
+    """With eta = 1 the DDIM update is the DDPM posterior q(x_prev | x_t, x0) (Ho, Jain &
+    Abbeel 2020, eqs. 6-7) sampled with z, for the effective alpha = ab_t / ab_prev."""
+    rng = np.random.default_rng(32)
+    x_t, x0, z = rng.normal(size=(3, 5, 279))
+    for ab in (ko.alphabar_linear(), ko.alphabar_cosine()):
+        for t, tp in [(999, 979), (500, 433), (66, 0), (66, -1)]:
+            at, ap = ab[t], (1.0 if tp < 0 else ab[tp])
+            alpha = at / ap
+            beta = 1 - alpha
+            mean = math.sqrt(ap) * beta / (1 - at) * x0 + math.sqrt(alpha) * (1 - ap) / (1 - at) * x_t
+            var = (1 - ap) / (1 - at) * beta
+            got = ko.ddim_update_eta(x_t, x0, at, ap, 1.0, z)
+            np.testing.assert_allclose(got, mean + math.sqrt(var) * z, rtol=0, atol=1e-11)
+
+
+def test_ddim_eta_keeps_the_forward_marginal():
+    """Exact x0, x_t ~ q(x_t | x0) and z ~ N(0, 1): x_prev ~ N(sqrt(ab_prev) x0, 1 - ab_prev)."""
+    ab = ko.alphabar_cosine()
+    rng = np.random.default_rng(33)
+    n = 200_000
+    x0 = 0.7
+    eps, z = rng.normal(size=(2, n))
+    at, ap = ab[600], ab[450]
+    x_t = math.sqrt(at) * x0 + math.sqrt(1 - at) * eps
+    x_prev = ko.ddim_update_eta(x_t, np.full(n, x0), at, ap, 0.6, z)
+    r = x_prev - math.sqrt(ap) * x0
+    assert abs(r.mean()) < 5 / math.sqrt(n)
+    assert r.var() == pytest.approx(1 - ap, rel=0.02)
+
+
 def test_cfg_special_cases():
     rng = np.random.default_rng(13)
     c, u = rng.normal(size=(5, 279)), rng.normal(size=(5, 279))
