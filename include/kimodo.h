@@ -145,16 +145,57 @@ KIMODO_API int kimodo_ddim_step(kimodo_ctx* ctx, const float* x_t, const float* 
 
 /*
  * Full DDIM sampling loop: `steps` two-stage steps (as kimodo_ddim_step) on the
- * trailing timesteps t_k = 999 - k (1000/steps), t_prev = t_k - 1000/steps,
- * starting from `noise`.  steps must divide 1000.  The loop runs as one CUDA
- * graph captured per (batch, frames, steps, cfg_scale) and cached in the context;
- * no host synchronisation happens between steps.
+ * trailing timesteps t_k = floor(1000 (steps - k) / steps + 1/2) - 1, k = 0..steps-1,
+ * t_prev = t_{k+1}, and -1 after the last step (for steps dividing 1000 this is
+ * t_k = 999 - k (1000/steps)), starting from `noise`; 1 <= steps <= 1000.  The loop
+ * runs as one CUDA graph captured per (batch, frames, steps, cfg_scale, sampler
+ * options) and cached in the context; no host synchronisation happens between steps.
  *
  * noise: [batch, frames, 279].  out: [batch, frames, 279] final sample; may alias noise.
  */
 KIMODO_API int kimodo_ddim_sample(kimodo_ctx* ctx, const float* text_emb, const float* null_emb,
                        int null_batch, const float* noise, const int* lengths, int batch,
                        int frames, int steps, float cfg_scale, float* out, void* stream);
+
+/*
+ * Sampler options of the _ex entry points (the "Model details" table of the
+ * "Kimodo WebGPU" page names a cosine beta schedule; the DDIM paper, Song, Meng &
+ * Ermon 2021, eqs. 12 and 16, defines the eta > 0 family).
+ *
+ * schedule: KIMODO_SCHEDULE_LINEAR (beta = linspace(1e-4, 0.02, 1000), the default)
+ *   or KIMODO_SCHEDULE_COSINE (Nichol & Dhariwal 2021: alphabar(u) = f(u) / f(0),
+ *   f(u) = cos^2((u + 0.008) / 1.008 * pi / 2), beta_i = min(1 - alphabar((i+1)/1000) /
+ *   alphabar(i/1000), 0.999), table = cumulative product of 1 - beta).
+ * eta: in [0, 1].  With sigma = eta sqrt((1 - ab_prev) / (1 - ab_t)) sqrt(1 - ab_t / ab_prev):
+ *   x_prev = sqrt(ab_prev) x0 + sqrt(1 - ab_prev - sigma^2) eps + sigma z,
+ *   eps = (x_t - sqrt(ab_t) x0) / sqrt(1 - ab_t); eta = 0 is deterministic DDIM.
+ * step_noise: the standard-normal draws z (fp32, host or device memory, read during
+ *   the call's work; the caller keeps it alive until then): [steps, batch, frames, 279]
+ *   for kimodo_ddim_sample_ex (step k uses slice k), [batch, frames, 279] for
+ *   kimodo_ddim_step_ex.  Required when eta > 0, ignored when eta = 0.  Values at
+ *   padded frames are never read into valid outputs.  A graph captured for a device
+ *   step_noise pointer reads that pointer on every replay.
+ * A NULL options pointer means { KIMODO_SCHEDULE_LINEAR, 0, NULL }.
+ */
+enum { KIMODO_SCHEDULE_LINEAR = 0, KIMODO_SCHEDULE_COSINE = 1 };
+typedef struct kimodo_sampler {
+  int schedule;
+  float eta;
+  const float* step_noise;
+} kimodo_sampler;
+
+/* kimodo_ddim_sample with sampler options (KIMODO_EINVAL on an unknown schedule,
+ * eta outside [0, 1] or not finite, or eta > 0 without step_noise). */
+KIMODO_API int kimodo_ddim_sample_ex(kimodo_ctx* ctx, const float* text_emb, const float* null_emb,
+                       int null_batch, const float* noise, const int* lengths, int batch,
+                       int frames, int steps, float cfg_scale, const kimodo_sampler* options,
+                       float* out, void* stream);
+
+/* kimodo_ddim_step with sampler options (same checks as kimodo_ddim_sample_ex). */
+KIMODO_API int kimodo_ddim_step_ex(kimodo_ctx* ctx, const float* x_t, const float* text_emb,
+                     const float* null_emb, int null_batch, const int* lengths, int batch,
+                     int frames, int t, int t_prev, float cfg_scale, const kimodo_sampler* options,
+                     float* x_prev, void* stream);
 
 /* Synchronise `stream` and report any device-side failure recorded since the
  * last check (KIMODO_ETIMEOUT with the kernel named in kimodo_last_error()). */

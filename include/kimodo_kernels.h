@@ -54,6 +54,18 @@ KIMODO_API int kimodo_gemm_bf16_pair(const void* A, int lda, const void* W, int 
                                      const void* resid, int ldr, void* out, int ldo, int M, int N, int K,
                                      int epilogue, int out_f32, int tile_n, void* stream);
 
+/*
+ * The same product with stream-K work sharing (the denoiser's kernel for its large
+ * projections): 256 x 256 pair tiles, every SM pair takes an equal contiguous share
+ * of the (tile, 64-deep k-block) units; a tile split between pairs is summed in fp32
+ * by the pair that holds its last k-block.  Arguments and epilogues as
+ * kimodo_gemm_bf16_pair (no tile choice).  The call allocates and frees its
+ * partial-sum workspace in stream order (cudaMallocAsync on `stream`).
+ */
+KIMODO_API int kimodo_gemm_bf16_streamk(const void* A, int lda, const void* W, int ldw, const float* bias,
+                                        const void* resid, int ldr, void* out, int ldo, int M, int N, int K,
+                                        int epilogue, int out_f32, void* stream);
+
 /* fp32 SIMT GEMM with the same epilogues; all operands fp32; K % 16 == 0,
  * lda, ldw multiples of 4. */
 KIMODO_API int kimodo_gemm_f32(const float* A, int lda, const float* W, int ldw, const float* bias,

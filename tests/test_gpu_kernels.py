@@ -104,6 +104,56 @@ def test_gemm_tcgen05_pair_vs_oracle(M, N, K, epi, out_f32, tile):
         np.testing.assert_allclose(got, ref, rtol=2 ** -8, atol=1e-5 * scale)
 
 
+STREAMK_CASES = [
+    # M, N, K, epilogue, out_f32 (stream-K pair kernel: 256 x 256 tiles, equal k-block shares)
+    (4832, 3072, 1024, kb.EPI_BIAS, False),        # QKV: shares of 3.08 tiles, tail and head pieces
+    (4832, 2048, 1024, kb.EPI_BIAS_GELU, False),
+    (4832, 1024, 1024, kb.EPI_BIAS_RESID, True),   # 76 tiles on the pairs: about one tile each
+    (4832, 1024, 2048, kb.EPI_BIAS_RESID, True),
+    (1283, 2048, 1024, kb.EPI_BIAS_GELU, False),   # shares shorter than a tile: several contributors
+    (300, 1024, 1024, kb.EPI_BIAS, False),         # 8 tiles over all pairs; second CTA of a pair out of range
+    (611, 1024, 2048, kb.EPI_BIAS_RESID, True),
+]
+
+
+@pytest.mark.parametrize("M,N,K,epi,out_f32", STREAMK_CASES)
+def test_gemm_tcgen05_streamk_vs_oracle(M, N, K, epi, out_f32):
+    require_cuda()
+    seed = M * 3 + N * 11 + K
+    A = _bf16(synth.random_vectors((M, K), seed))
+    W = _bf16(synth.random_vectors((N, K), seed + 1, 0.05))
+    bias = torch.from_numpy(synth.random_vectors((N,), seed + 2, 0.1))
+    resid = torch.from_numpy(synth.random_vectors((M, N), seed + 3)) if epi == kb.EPI_BIAS_RESID else None
+    out = kb.gemm_bf16(A.cuda(), W.cuda(), bias.cuda(), epi, out_f32, None if resid is None else resid.cuda(),
+                       stream_k=True)
+    torch.cuda.synchronize()
+    ref = _epi_ref(epi, ko.linear(_f64(A), _f64(W), bias.double().numpy()),
+                   None if resid is None else resid.double().numpy())
+    got = out.float().cpu().double().numpy()
+    scale = np.abs(ref).max()
+    if out_f32:
+        np.testing.assert_allclose(got, ref, rtol=0, atol=2e-5 * scale)
+    else:
+        np.testing.assert_allclose(got, ref, rtol=2 ** -8, atol=1e-5 * scale)
+
+
+def test_gemm_streamk_residual_in_place_and_repeatable():
+    """The stream-K residual epilogue may read and write the same fp32 buffer, and the
+    split-tile sums do not depend on the run."""
+    require_cuda()
+    M, N, K = 4832, 1024, 1024
+    A = _bf16(synth.random_vectors((M, K), 95)).cuda()
+    W = _bf16(synth.random_vectors((N, K), 96, 0.05)).cuda()
+    bias = torch.from_numpy(synth.random_vectors((N,), 97, 0.1)).cuda()
+    y = torch.from_numpy(synth.random_vectors((M, N), 98)).cuda()
+    want = kb.gemm_bf16(A, W, bias, kb.EPI_BIAS_RESID, True, y.clone(), stream_k=True)
+    again = kb.gemm_bf16(A, W, bias, kb.EPI_BIAS_RESID, True, y.clone(), stream_k=True)
+    kb.gemm_bf16(A, W, bias, kb.EPI_BIAS_RESID, True, y, out=y, stream_k=True)
+    torch.cuda.synchronize()
+    assert torch.equal(want, again)
+    assert torch.equal(want, y)
+
+
 def test_gemm_residual_in_place():
     """The residual epilogue may read and write the same fp32 buffer."""
     require_cuda()

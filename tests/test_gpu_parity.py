@@ -148,6 +148,33 @@ def test_host_and_device_pointers_agree(gpu_bf16):
     gpu_bf16.sync_status()
 
 
+@pytest.mark.parametrize("precision", ["bf16", "fp32"])
+def test_packed_layout_equals_padded_layout(gpu_bf16, gpu_fp32, precision):
+    """Ragged lengths given in host memory run on the packed token layout (valid tokens
+    only); the same lengths in device memory run on the padded layout.  Below the pair
+    GEMM's row threshold every output element is computed in the same order either way,
+    so the two agree bit for bit, and padded frames are 0 in both."""
+    model = gpu_bf16 if precision == "bf16" else gpu_fp32
+    B, T, L = 3, 60, np.array([60, 33, 1], np.int32)
+    x = synth.fill_padding(synth.noise(B, T, seed=71), L)
+    emb = synth.text_embeddings(B, seed=72)
+    null = np.zeros(4096, np.float32)
+    packed = model.ddim_step(x, emb, null, L, 999, 966, 2.0)
+    padded_ = model.ddim_step(x, emb, null, torch.from_numpy(L).cuda(), 999, 966, 2.0)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(packed, padded_)
+    assert np.all(padded(packed, L) == 0)
+    fp = model.denoiser_forward(kb.NET_BODY, x, emb, 500, L)
+    fd = model.denoiser_forward(kb.NET_BODY, x, emb, 500, torch.from_numpy(L).cuda())
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(fp, fd)
+    assert np.all(padded(fp, L) == 0)
+    s1 = model.ddim_sample(emb, null, x, L, 3, 2.0)
+    s2 = model.ddim_sample(emb, null, x, torch.from_numpy(L).cuda(), 3, 2.0)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(s1, s2)
+
+
 def test_c4_full_size_sampled(gpu_bf16, params):
     """100-step generation at B=16, T=150 (the throughput workload, as bench.py
     runs it): sequence 0 against the oracle over all 100 steps, sequence 15
@@ -184,6 +211,10 @@ def test_c5_ragged_garbage_sampled(gpu_bf16, params):
     np.testing.assert_array_equal(gpu_bf16.ddim_sample(emb, null, zeros, L, 50, 2.5), got)
     nans = synth.fill_padding(noise, L, nan=True)
     np.testing.assert_array_equal(gpu_bf16.ddim_sample(emb, null, nans, L, 50, 2.5), got)
+    # lengths in device memory: the padded token layout, the same result up to summation order
+    dense = gpu_bf16.ddim_sample(emb, null, garbage, torch.from_numpy(L).cuda(), 50, 2.5)
+    torch.cuda.synchronize()
+    report("bf16 sample c5 padded vs packed layout rel-L2", rel_l2(valid(dense, L), valid(got, L)), 1e-2)
     b = int(np.argmin(L))
     ref = ko.ddim_sample(params, emb[b], null, garbage[b], int(L[b]), 50, 2.5)
     report(f"bf16 sample c5 seq {b} len {L[b]} (50 steps, cfg 2.5) trajectory rel-L2",

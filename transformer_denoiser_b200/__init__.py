@@ -31,6 +31,8 @@ SIGNATURES = [
     ("kimodo_denoiser_forward_noalloc", _I, [_P, _I, _P, _P, _I, _P, _I, _I, _P, _P]),
     ("kimodo_ddim_step", _I, [_P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _F, _P, _P]),
     ("kimodo_ddim_sample", _I, [_P, _P, _P, _I, _P, _P, _I, _I, _I, _F, _P, _P]),
+    ("kimodo_ddim_step_ex", _I, [_P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _F, _P, _P, _P]),
+    ("kimodo_ddim_sample_ex", _I, [_P, _P, _P, _I, _P, _P, _I, _I, _I, _F, _P, _P, _P]),
     ("kimodo_sync_status", _I, [_P, _P]),
     ("kimodo_profile_enable", _I, [_P, _I]),
     ("kimodo_profile_read", _I, [_P, _I, _P, _P, _P, _P]),
@@ -40,12 +42,21 @@ SIGNATURES = [
     # include/kimodo_kernels.h
     ("kimodo_gemm_bf16", _I, [_P, _I, _P, _I, _P, _P, _I, _P, _I, _I, _I, _I, _I, _I, _I, _P]),
     ("kimodo_gemm_bf16_pair", _I, [_P, _I, _P, _I, _P, _P, _I, _P, _I, _I, _I, _I, _I, _I, _I, _P]),
+    ("kimodo_gemm_bf16_streamk", _I, [_P, _I, _P, _I, _P, _P, _I, _P, _I, _I, _I, _I, _I, _I, _P]),
     ("kimodo_gemm_f32", _I, [_P, _I, _P, _I, _P, _P, _I, _P, _I, _I, _I, _I, _I, _P]),
     ("kimodo_attention_bf16", _I, [_P, _P, _P, _I, _I, _P]),
     ("kimodo_attention_f32", _I, [_P, _P, _P, _I, _I, _P]),
     ("kimodo_layernorm", _I, [_P, _P, _I, _P, _P, _I, _P]),
 ]
 EPI_BIAS, EPI_BIAS_GELU, EPI_BIAS_SILU, EPI_BIAS_RESID = 0, 1, 2, 3
+
+
+SCHEDULES = {"linear": 0, "cosine": 1}
+
+
+class SamplerOptions(ctypes.Structure):
+    """struct kimodo_sampler of include/kimodo.h."""
+    _fields_ = [("schedule", ctypes.c_int), ("eta", ctypes.c_float), ("step_noise", ctypes.c_void_p)]
 
 
 class KimodoError(RuntimeError):
@@ -140,19 +151,24 @@ def _cur_stream():
 
 # ------------------------------------------------------------ kernel-level calls (torch CUDA tensors)
 
-def gemm_bf16(A, W, bias, epilogue=EPI_BIAS, out_f32=False, resid=None, out=None, K=None, tile_n=0, pair=False):
+def gemm_bf16(A, W, bias, epilogue=EPI_BIAS, out_f32=False, resid=None, out=None, K=None, tile_n=0, pair=False,
+              stream_k=False):
     """out = epilogue(A[:, :K] W[:, :K]^T + bias) on the tcgen05 GEMM (A, W bf16 CUDA tensors);
-    pair=True runs the CTA-pair kernel (256-row tiles)."""
+    pair=True runs the CTA-pair kernel (256-row tiles), stream_k=True its stream-K variant."""
     import torch
     lib = load_library()
-    fn = lib.kimodo_gemm_bf16_pair if pair else lib.kimodo_gemm_bf16
     M, N = A.shape[0], W.shape[0]
     K = A.shape[1] if K is None else K
     if out is None:
         out = torch.empty((M, N), dtype=torch.float32 if out_f32 else torch.bfloat16, device=A.device)
-    _check(fn(_ptr_rows(A), A.stride(0), _ptr_rows(W), W.stride(0), _ptr(bias), _ptr_rows(resid),
-                                0 if resid is None else resid.stride(0), _ptr_rows(out), out.stride(0), M, N, K,
-                                int(epilogue), int(bool(out_f32)), int(tile_n), _cur_stream()))
+    args = [_ptr_rows(A), A.stride(0), _ptr_rows(W), W.stride(0), _ptr(bias), _ptr_rows(resid),
+            0 if resid is None else resid.stride(0), _ptr_rows(out), out.stride(0), M, N, K,
+            int(epilogue), int(bool(out_f32))]
+    if stream_k:
+        _check(lib.kimodo_gemm_bf16_streamk(*args, _cur_stream()))
+    else:
+        fn = lib.kimodo_gemm_bf16_pair if pair else lib.kimodo_gemm_bf16
+        _check(fn(*args, int(tile_n), _cur_stream()))
     return out
 
 
@@ -231,24 +247,48 @@ class Kimodo:
                                                          _ptr(lengths), B, T, _ptr(out), _stream(stream, x, out)))
         return out
 
-    def ddim_step(self, x_t, text_emb, null_emb, lengths, t, t_prev, cfg_scale, out=None, stream=None):
+    @staticmethod
+    def _options(schedule, eta, step_noise):
+        """kimodo_sampler for the _ex calls, or None for the defaults (linear, eta 0)."""
+        if schedule == "linear" and float(eta) == 0.0:
+            return None, None
+        z = None if step_noise is None else _f32(step_noise)
+        return SamplerOptions(SCHEDULES[schedule], float(eta), _ptr(z)), z
+
+    def ddim_step(self, x_t, text_emb, null_emb, lengths, t, t_prev, cfg_scale, out=None, stream=None,
+                  schedule="linear", eta=0.0, step_noise=None):
         x_t, text_emb, null_emb, lengths = _f32(x_t), _f32(text_emb), _f32(null_emb), _i32(lengths)
         B, T = x_t.shape[0], x_t.shape[1]
         nb = 1 if null_emb.ndim == 1 else null_emb.shape[0]
         out = _like(x_t, (B, T, MOTION_DIM)) if out is None else out
-        _check(self._lib.kimodo_ddim_step(self._ctx, _ptr(x_t), _ptr(text_emb), _ptr(null_emb), nb, _ptr(lengths),
-                                          B, T, int(t), int(t_prev), float(cfg_scale), _ptr(out),
-                                          _stream(stream, x_t, out)))
+        opts, z = self._options(schedule, eta, step_noise)
+        if opts is None:
+            _check(self._lib.kimodo_ddim_step(self._ctx, _ptr(x_t), _ptr(text_emb), _ptr(null_emb), nb,
+                                              _ptr(lengths), B, T, int(t), int(t_prev), float(cfg_scale), _ptr(out),
+                                              _stream(stream, x_t, out)))
+        else:
+            _check(self._lib.kimodo_ddim_step_ex(self._ctx, _ptr(x_t), _ptr(text_emb), _ptr(null_emb), nb,
+                                                 _ptr(lengths), B, T, int(t), int(t_prev), float(cfg_scale),
+                                                 ctypes.byref(opts), _ptr(out), _stream(stream, x_t, out)))
         return out
 
-    def ddim_sample(self, text_emb, null_emb, noise, lengths, steps, cfg_scale, out=None, stream=None):
+    def ddim_sample(self, text_emb, null_emb, noise, lengths, steps, cfg_scale, out=None, stream=None,
+                    schedule="linear", eta=0.0, step_noise=None):
+        """Full sampler; schedule "linear" or "cosine", eta in [0, 1] with step_noise
+        [steps, B, T, 279] standard-normal draws when eta > 0."""
         text_emb, null_emb, noise, lengths = _f32(text_emb), _f32(null_emb), _f32(noise), _i32(lengths)
         B, T = noise.shape[0], noise.shape[1]
         nb = 1 if null_emb.ndim == 1 else null_emb.shape[0]
         out = _like(noise, (B, T, MOTION_DIM)) if out is None else out
-        _check(self._lib.kimodo_ddim_sample(self._ctx, _ptr(text_emb), _ptr(null_emb), nb, _ptr(noise),
-                                            _ptr(lengths), B, T, int(steps), float(cfg_scale), _ptr(out),
-                                            _stream(stream, noise, out)))
+        opts, z = self._options(schedule, eta, step_noise)
+        if opts is None:
+            _check(self._lib.kimodo_ddim_sample(self._ctx, _ptr(text_emb), _ptr(null_emb), nb, _ptr(noise),
+                                                _ptr(lengths), B, T, int(steps), float(cfg_scale), _ptr(out),
+                                                _stream(stream, noise, out)))
+        else:
+            _check(self._lib.kimodo_ddim_sample_ex(self._ctx, _ptr(text_emb), _ptr(null_emb), nb, _ptr(noise),
+                                                   _ptr(lengths), B, T, int(steps), float(cfg_scale),
+                                                   ctypes.byref(opts), _ptr(out), _stream(stream, noise, out)))
         return out
 
     def sync_status(self, stream=None):

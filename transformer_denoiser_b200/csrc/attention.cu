@@ -55,11 +55,14 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 // V of the valid keys (rounded up to 32) sit in shared memory for all warps.
 __global__ void __launch_bounds__(ATT_MAX_WARPS * 32, 1)
 attn_bf16_kernel(const bf16* __restrict__ qkv, bf16* __restrict__ out, const int* __restrict__ lengths,
-                 int len_mod, int S) {
+                 int len_mod, int S_pad, const int* __restrict__ tok0) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
   ptx::pdl_wait();
   ptx::pdl_trigger();
   const int h = blockIdx.x, seq = blockIdx.y;
+  // rows of this sequence: padded layout seq * S_pad + [0, S_pad), packed layout [tok0[seq], tok0[seq + 1])
+  const long row0 = tok0 ? tok0[seq] : (long)seq * S_pad;
+  const int S = tok0 ? tok0[seq + 1] - tok0[seq] : S_pad;
   int n_valid = 1 + lengths[seq % len_mod];
   n_valid = n_valid < 1 ? 1 : (n_valid > S ? S : n_valid);
   const int nkb = (n_valid + KBLK - 1) / KBLK;
@@ -67,7 +70,7 @@ attn_bf16_kernel(const bf16* __restrict__ qkv, bf16* __restrict__ out, const int
   bf16* sV = sK + nkb * KBLK * LDS;
 
   const long rs = 3L * D;
-  const bf16* base = qkv + (long)seq * S * rs + h * DH;
+  const bf16* base = qkv + row0 * rs + h * DH;
   const int tid = threadIdx.x, nthr = blockDim.x;
   for (int c = tid; c < nkb * KBLK * 16; c += nthr) {
     const int r = c >> 4, ch = c & 15;
@@ -183,7 +186,7 @@ attn_bf16_kernel(const bf16* __restrict__ qkv, bf16* __restrict__ out, const int
     l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
     const float i0 = 1.f / l0, i1 = 1.f / l1;
     const int r0 = qw + g, r1 = qw + g + 8;
-    bf16* ob = out + (long)seq * S * D + h * DH + 2 * c4;
+    bf16* ob = out + row0 * D + h * DH + 2 * c4;
 #pragma unroll
     for (int n = 0; n < 16; ++n) {
       if (r0 < S)
@@ -195,16 +198,19 @@ attn_bf16_kernel(const bf16* __restrict__ qkv, bf16* __restrict__ out, const int
 }
 
 __global__ void __launch_bounds__(128) attn_f32_kernel(const float* __restrict__ qkv, float* __restrict__ out,
-                                                       const int* __restrict__ lengths, int len_mod, int S) {
+                                                       const int* __restrict__ lengths, int len_mod, int S_pad,
+                                                       const int* __restrict__ tok0) {
   ptx::pdl_wait();
   ptx::pdl_trigger();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int q = blockIdx.x * 4 + warp, h = blockIdx.y, seq = blockIdx.z;
+  const long row0 = tok0 ? tok0[seq] : (long)seq * S_pad;
+  const int S = tok0 ? tok0[seq + 1] - tok0[seq] : S_pad;
   if (q >= S) return;
   int n_valid = 1 + lengths[seq % len_mod];
   n_valid = n_valid < 1 ? 1 : (n_valid > S ? S : n_valid);
   const long rs = 3L * D;
-  const float* base = qkv + (long)seq * S * rs + h * DH + lane * 4;
+  const float* base = qkv + row0 * rs + h * DH + lane * 4;
   const float4 qv = *reinterpret_cast<const float4*>(base + (long)q * rs);
   const float scale = 0.08838834764831845f;
   float m = -INFINITY, l = 0.f;
@@ -226,7 +232,7 @@ __global__ void __launch_bounds__(128) attn_f32_kernel(const float* __restrict__
     m = mn;
   }
   const float inv = 1.f / l;
-  *reinterpret_cast<float4*>(out + ((long)seq * S + q) * D + h * DH + lane * 4) =
+  *reinterpret_cast<float4*>(out + (row0 + q) * D + h * DH + lane * 4) =
       make_float4(o.x * inv, o.y * inv, o.z * inv, o.w * inv);
 }
 
@@ -238,13 +244,13 @@ size_t attention_bf16_smem(int S) {
 }
 
 cudaError_t attention_bf16(const bf16* qkv, bf16* out, const int* lengths, int len_mod, int nseq, int S,
-                           cudaStream_t st) {
+                           cudaStream_t st, const int* tok0) {
   if (nseq <= 0 || S <= 0) return cudaSuccess;
   const size_t smem = attention_bf16_smem(S);
   int warps = (S + 15) / 16;
   warps = warps > ATT_MAX_WARPS ? ATT_MAX_WARPS : warps;
   dim3 grid(H, nseq);
-  return launch_kernel(attn_bf16_kernel, grid, dim3(32 * warps), smem, st, qkv, out, lengths, len_mod, S);
+  return launch_kernel(attn_bf16_kernel, grid, dim3(32 * warps), smem, st, qkv, out, lengths, len_mod, S, tok0);
 }
 
 cudaError_t attention_prepare() {
@@ -253,10 +259,10 @@ cudaError_t attention_prepare() {
 }
 
 cudaError_t attention_f32(const float* qkv, float* out, const int* lengths, int len_mod, int nseq, int S,
-                          cudaStream_t st) {
+                          cudaStream_t st, const int* tok0) {
   if (nseq <= 0 || S <= 0) return cudaSuccess;
   dim3 grid((S + 3) / 4, H, nseq);
-  return launch_kernel(attn_f32_kernel, grid, dim3(128), 0, st, qkv, out, lengths, len_mod, S);
+  return launch_kernel(attn_f32_kernel, grid, dim3(128), 0, st, qkv, out, lengths, len_mod, S, tok0);
 }
 
 }  // namespace kd

@@ -77,6 +77,15 @@ struct Workspace {
   float* root_hat = nullptr; float* body_hat = nullptr; float* x = nullptr;
   void* emb = nullptr; float* txt[2] = {}; void* tpe = nullptr; void* thid = nullptr; float* tmlp[2] = {};
   int* lengths = nullptr; float* st_text = nullptr; float* st_null = nullptr;
+  int* tok0 = nullptr; int* row_seq = nullptr;   // packed token layout (valid tokens only)
+};
+
+// Token rows of a call: the padded layout (every sequence frames + 1 rows) or, when the
+// lengths are known on the host and some sequence is shorter than `frames`, the packed
+// layout of the valid tokens only (sequence s owns rows tok0[s] .. tok0[s + 1] - 1).
+struct Tokens {
+  int M = 0;
+  bool packed = false;
 };
 
 struct ProfRec {
@@ -95,10 +104,16 @@ struct kimodo_ctx {
   NetW net[2];
   float* pe = nullptr;          // [N_TRAIN, D] sinusoid table (positions and timesteps)
   DevError* derr = nullptr;
-  double alphabar[N_TRAIN];
+  double alphabar[2][N_TRAIN];   // [KIMODO_SCHEDULE_LINEAR / _COSINE][t]
   Workspace ws;
   cudaStream_t cap_stream = nullptr;
-  std::map<std::tuple<int, int, int, int, uint32_t>, std::pair<cudaGraphExec_t, long long>> graphs;
+  // sampler graphs keyed by (batch, frames, steps, null broadcast, cfg bits, schedule, eta bits, step noise,
+  // token rows: the packed layout's row count, or the padded one)
+  std::map<std::tuple<int, int, int, int, uint32_t, int, uint32_t, const float*, int>,
+           std::pair<cudaGraphExec_t, long long>>
+      graphs;
+  float* zbuf = nullptr;        // staging of host step-noise draws
+  size_t zcap = 0;              // floats
   bool profiling = false;
   unsigned prof_flags = cudaEventRecordDefault;   // cudaEventRecordExternal while a profiled graph is captured
   std::vector<ProfRec> prof;
@@ -106,7 +121,11 @@ struct kimodo_ctx {
   size_t ev_used = 0;
   long long launches = 0;
   long long last_launches = 0;
+  Tokens tk;                    // token layout of the call being enqueued
   bool pair_gemm = true;   // 256-row CTA-pair GEMM tiles for the large projections (KIMODO_PAIR_GEMM=0 disables)
+  bool stream_k = true;    // stream-K shares for them (KIMODO_STREAM_K=0: one whole tile per pair and round)
+  float* sk_partial = nullptr;   // stream-K partial accumulators
+  int* sk_flags = nullptr;       // stream-K contributor counters (zero between launches)
   bool bf16() const { return precision == KIMODO_BF16; }
   size_t elem() const { return bf16() ? 2 : 4; }
 };
@@ -163,6 +182,10 @@ int gemm(kimodo_ctx* c, const void* A, int lda, const void* W, int ldw, int M, i
                        (double)M * N * (out_f32 ? 4.0 : (double)c->elem()) +
                        (kind == EPI_BIAS_RESID ? (double)M * N * 4.0 : 0.0);
   if (c->bf16()) {
+    if (c->pair_gemm && c->stream_k && M >= 1024 && N >= 256 && gemm_tc2_supports(kind, out_f32)) {
+      return launch(c, cls_override >= 0 ? cls_override : CLS_GEMM_TC, flops, bytes, st, "gemm_sk",
+                    [&] { return gemm_sk(g, kind, out_f32, ep, c->sk_partial, c->sk_flags, c->derr, st); });
+    }
     if (c->pair_gemm && M >= 1024 && N >= 256 && gemm_tc2_supports(kind, out_f32)) {
       const int bn = gemm_tc2_pick_bn(M, N, kind);
       return launch(c, cls_override >= 0 ? cls_override : CLS_GEMM_TC, flops, bytes, st, "gemm_tc2",
@@ -282,7 +305,8 @@ int ensure_workspace(kimodo_ctx* c, int nseq, int frames, int steps) {
       {&w.tpe, (size_t)ST * D * e},                        {&w.thid, (size_t)ST * D * e},
       {(void**)&w.tmlp[0], (size_t)ST * D * 4},            {(void**)&w.tmlp[1], (size_t)ST * D * 4},
       {(void**)&w.lengths, (size_t)NS * 4},                {(void**)&w.st_text, (size_t)NS * DTXT * 4},
-      {(void**)&w.st_null, (size_t)NS * DTXT * 4}};
+      {(void**)&w.st_null, (size_t)NS * DTXT * 4},        {(void**)&w.tok0, (size_t)(NS + 1) * 4},
+      {(void**)&w.row_seq, (size_t)R2 * 4}};
   for (auto& p : plan) off += align256(p.second);
   void* arena = nullptr;
   cudaError_t err = cudaMalloc(&arena, off);
@@ -305,10 +329,16 @@ int ensure_workspace(kimodo_ctx* c, int nseq, int frames, int steps) {
 // ------------------------------------------------------------------ forward pieces
 
 // Sinusoid rows of the n_t timesteps t0, t0 - stride, ... (shared by both networks).
-int timestep_rows(kimodo_ctx* c, int t0, int stride, int n_t, cudaStream_t st) {
+// Sinusoid rows of the n_t timesteps of this call: one explicit t (steps == 0) or the
+// trailing timesteps of a `steps`-step sampler.
+int timestep_rows(kimodo_ctx* c, int t_single, int steps, int n_t, cudaStream_t st) {
   return launch(c, CLS_SETUP, 0, (double)n_t * D * 8, st, "gather_timestep_rows",
-                [&] { return gather_timestep_rows(c->pe, t0, stride, n_t, c->ws.tpe, c->bf16(), st); });
+                [&] { return gather_timestep_rows(c->pe, t_single, steps, n_t, c->ws.tpe, c->bf16(), st); });
 }
+
+// k-th trailing timestep of a `steps`-step sampler: floor(1000 (steps - k) / steps + 1/2) - 1
+// (-1 for k == steps).
+int trailing_t(int k, int steps) { return (2 * N_TRAIN * (steps - k) + steps) / (2 * steps) - 1; }
 
 // Condition vectors of one network: text projection of the packed embeddings
 // (rows) and the timestep MLP of the n_t gathered timestep rows.
@@ -334,11 +364,16 @@ int run_net(kimodo_ctx* c, int net, int nseq, int T, int len_mod, const void* A_
             const float* txt, float* hat, cudaStream_t st) {
   NetW& n = c->net[net];
   Workspace& w = c->ws;
-  const int S = T + 1, M = nseq * S;
+  const int S = T + 1;
+  const bool packed = c->tk.packed;
+  const int M = packed ? c->tk.M : nseq * S;
+  const int* tok0 = packed ? w.tok0 : nullptr;
+  const int* row_seq = packed ? w.row_seq : nullptr;
   const bool act_f32 = !c->bf16();
   {
     EpiParams e;
     e.bias = n.in_b; e.out = w.h; e.ldo = D; e.pe = c->pe; e.cond = txt; e.tvec = tvec; e.S = S; e.N = D; e.M = M;
+    e.tok0 = tok0; e.row_seq = row_seq;
     if (c->bf16()) e.out32 = w.y;   // fp32 residual stream
     KD_TRY(gemm(c, A_in, n.in_ld, n.in_W, n.in_ld, M, D, n.in_ld, EPI_INPROJ, act_f32, e, st));
   }
@@ -353,17 +388,17 @@ int run_net(kimodo_ctx* c, int net, int nseq, int T, int len_mod, const void* A_
     EpiParams e;
     e.bias = n.qkv_b[l]; e.out = w.qkv; e.ldo = 3 * D; e.N = 3 * D; e.M = M;
     KD_TRY(gemm(c, w.h, D, n.qkv_W[l], D, M, 3 * D, D, EPI_BIAS, act_f32, e, st));
-    const double aflops = 4.0 * (double)nseq * S * S * DH * H;
+    const double aflops = packed ? 4.0 * (double)M * S * DH * H : 4.0 * (double)nseq * S * S * DH * H;
     const double abytes = (double)M * 3 * D * eb + (double)M * D * eb;
     if (c->bf16()) {
       KD_TRY(launch(c, CLS_ATTN, aflops, abytes, st, "attention_bf16", [&] {
         return attention_bf16(static_cast<const bf16*>(w.qkv), static_cast<bf16*>(w.attn), w.lengths, len_mod,
-                              nseq, S, st);
+                              nseq, S, st, tok0);
       }));
     } else {
       KD_TRY(launch(c, CLS_ATTN, aflops, abytes, st, "attention_f32", [&] {
         return attention_f32(static_cast<const float*>(w.qkv), static_cast<float*>(w.attn), w.lengths, len_mod,
-                             nseq, S, st);
+                             nseq, S, st, tok0);
       }));
     }
     EpiParams eo;
@@ -383,44 +418,85 @@ int run_net(kimodo_ctx* c, int net, int nseq, int T, int len_mod, const void* A_
   }
   EpiParams eo;
   eo.bias = n.out_b; eo.out = hat; eo.ldo = n.dout; eo.lengths = w.lengths; eo.len_mod = len_mod; eo.S = S;
-  eo.T = T; eo.N = n.dout; eo.M = M;
+  eo.T = T; eo.N = n.dout; eo.M = M; eo.tok0 = tok0; eo.row_seq = row_seq;
   return gemm(c, w.h, D, n.out_W, D, M, n.dout, D, EPI_OUTPROJ, true, eo, st);
 }
 
-void ddim_coeffs(const kimodo_ctx* c, int t, int t_prev, float* c0, float* c1) {
-  const double at = c->alphabar[t];
-  const double ap = t_prev < 0 ? 1.0 : c->alphabar[t_prev];
-  // x_prev = sqrt(ap) x0 + sqrt(1 - ap) (x_t - sqrt(at) x0) / sqrt(1 - at) = c0 x0 + c1 x_t
-  const double k1 = sqrt(1.0 - ap) / sqrt(1.0 - at);
+// DDIM update coefficients (double on the host):
+//   sigma = eta sqrt((1 - ap) / (1 - at)) sqrt(1 - at / ap),
+//   x_prev = sqrt(ap) x0 + sqrt(1 - ap - sigma^2) (x_t - sqrt(at) x0) / sqrt(1 - at) + sigma z
+//          = c0 x0 + c1 x_t + c2 z.
+void ddim_coeffs(const kimodo_ctx* c, int schedule, int t, int t_prev, double eta, float* c0, float* c1,
+                 float* c2) {
+  const double at = c->alphabar[schedule][t];
+  const double ap = t_prev < 0 ? 1.0 : c->alphabar[schedule][t_prev];
+  const double sigma = eta * sqrt((1.0 - ap) / (1.0 - at)) * sqrt(1.0 - at / ap);
+  const double k1 = sqrt(fmax(1.0 - ap - sigma * sigma, 0.0)) / sqrt(1.0 - at);
   *c0 = (float)(sqrt(ap) - k1 * sqrt(at));
   *c1 = (float)k1;
+  *c2 = (float)sigma;
 }
+
+// Sampler options after validation.
+struct Sampler {
+  int schedule = KIMODO_SCHEDULE_LINEAR;
+  float eta = 0.f;
+  const float* z = nullptr;   // device draws for the call (eta > 0), step-major
+};
 
 // One two-stage step for B prompts (cond rows 0..B-1, uncond rows B..2B-1).
 // Reads ws.x, writes ws.x.  tvec_root / tvec_body are the timestep-MLP rows.
 int two_stage_step(kimodo_ctx* c, int B, int T, int t, int t_prev, float w_cfg, int k_row, bool pack_next,
-                   cudaStream_t st) {
+                   const Sampler& smp, const float* z_step, cudaStream_t st) {
   Workspace& w = c->ws;
   const int nseq = 2 * B, S = T + 1;
   const double eb = (double)c->elem();
   KD_TRY(run_net(c, 0, nseq, T, B, w.A_root, w.tmlp[0] + (long)k_row * D, w.txt[0], w.root_hat, st));
   KD_TRY(launch(c, CLS_MOTION, 0, (double)nseq * T * (ROOT_F * 4 + MOTION_F * (4 + eb)), st, "g2l_body_input", [&] {
-    return g2l_body_input(w.root_hat, w.x, w.lengths, B, nseq, T, S, w.A_body, c->bf16(), BODY_IN_LD, st);
+    return g2l_body_input(w.root_hat, w.x, w.lengths, B, nseq, T, S, w.A_body, c->bf16(), BODY_IN_LD, st,
+                          c->tk.packed ? w.tok0 : nullptr);
   }));
   KD_TRY(run_net(c, 1, nseq, T, B, w.A_body, w.tmlp[1] + (long)k_row * D, w.txt[1], w.body_hat, st));
-  float c0, c1;
-  ddim_coeffs(c, t, t_prev, &c0, &c1);
-  return launch(c, CLS_MOTION, 0, (double)B * T * MOTION_F * 4 * 4, st, "cfg_ddim", [&] {
-    return cfg_ddim(w.root_hat, w.body_hat, w.x, w.lengths, B, T, w_cfg, c0, c1, pack_next ? w.A_root : nullptr,
-                    c->bf16(), ROOT_IN_LD, S, st);
+  float c0, c1, c2;
+  ddim_coeffs(c, smp.schedule, t, t_prev, smp.eta, &c0, &c1, &c2);
+  const float* z = c2 != 0.f ? z_step : nullptr;
+  return launch(c, CLS_MOTION, 0, (double)B * T * MOTION_F * 4 * (z ? 5 : 4), st, "cfg_ddim", [&] {
+    return cfg_ddim(w.root_hat, w.body_hat, w.x, w.lengths, B, T, w_cfg, c0, c1, z, c2,
+                    pack_next ? w.A_root : nullptr, c->bf16(), ROOT_IN_LD, S, st, c->tk.packed ? w.tok0 : nullptr);
   });
 }
 
 int pack_root_input(kimodo_ctx* c, int B, int nseq, int T, cudaStream_t st) {
   Workspace& w = c->ws;
   return launch(c, CLS_MOTION, 0, (double)nseq * T * ROOT_F * 8, st, "pack_frames", [&] {
-    return pack_frames(w.x, B, MOTION_F, 0, ROOT_F, w.A_root, c->bf16(), ROOT_IN_LD, 0, nseq, T, T + 1, st);
+    return pack_frames(w.x, B, MOTION_F, 0, ROOT_F, w.A_root, c->bf16(), ROOT_IN_LD, 0, nseq, T, T + 1, st,
+                       c->tk.packed ? w.tok0 : nullptr, w.lengths, B);
   });
+}
+
+bool is_device_memory(const void* p);
+
+// Chooses the token layout of a call (lengths already validated when on the host) and,
+// for the packed layout, enqueues the token map built from the staged lengths.
+Tokens plan_tokens(const int* lengths, int batch, int nseq, int frames) {
+  Tokens tk;
+  tk.M = nseq * (frames + 1);
+  if (lengths != nullptr && !is_device_memory(lengths)) {
+    long m = 0;
+    for (int s = 0; s < nseq; ++s) m += 1 + lengths[s % batch];
+    if (m < tk.M) {
+      tk.M = (int)m;
+      tk.packed = true;
+    }
+  }
+  return tk;
+}
+
+int enqueue_token_map(kimodo_ctx* c, int batch, int nseq, cudaStream_t st) {
+  if (!c->tk.packed) return KIMODO_OK;
+  Workspace& w = c->ws;
+  return launch(c, CLS_SETUP, 0, (double)c->tk.M * 4, st, "build_token_map",
+                [&] { return build_token_map(w.lengths, batch, nseq, w.tok0, w.row_seq, st); });
 }
 
 // ------------------------------------------------------------------ argument checks
@@ -505,7 +581,8 @@ int kimodo_load_weights(kimodo_ctx** out_ctx, const float* host_blob, size_t n_f
   if (precision == KIMODO_BF16 && !gemm_tc_available())
     return set_error(KIMODO_EUNSUPPORTED, "cuTensorMapEncodeTiled is unavailable in this driver");
 
-  if (gemm_tc_prepare() != cudaSuccess || gemm_tc2_prepare() != cudaSuccess || attention_prepare() != cudaSuccess) {
+  if (gemm_tc_prepare() != cudaSuccess || gemm_tc2_prepare() != cudaSuccess || gemm_sk_prepare() != cudaSuccess ||
+      attention_prepare() != cudaSuccess) {
     cudaGetLastError();
     return set_error(KIMODO_EUNSUPPORTED, "kernel attributes could not be set on device %d", device);
   }
@@ -513,6 +590,7 @@ int kimodo_load_weights(kimodo_ctx** out_ctx, const float* host_blob, size_t n_f
   c->device = device;
   c->precision = precision;
   if (const char* ev = getenv("KIMODO_PAIR_GEMM")) c->pair_gemm = ev[0] != '0';
+  if (const char* ev = getenv("KIMODO_STREAM_K")) c->stream_k = ev[0] != '0';
   c->num_sms = prop.multiProcessorCount;
   auto fail = [&](int code) {
     kimodo_free(c);
@@ -529,7 +607,18 @@ int kimodo_load_weights(kimodo_ctx** out_ctx, const float* host_blob, size_t n_f
     for (int i = 0; i < N_TRAIN; ++i) {
       const double beta = 1e-4 + (0.02 - 1e-4) * (double)i / (double)(N_TRAIN - 1);
       prod *= 1.0 - beta;
-      c->alphabar[i] = prod;
+      c->alphabar[KIMODO_SCHEDULE_LINEAR][i] = prod;
+    }
+    // cosine (Nichol & Dhariwal 2021, eq. 17), s = 0.008, beta clipped at 0.999
+    auto fcos = [](double u) {
+      const double v = cos((u + 0.008) / 1.008 * M_PI / 2.0);
+      return v * v;
+    };
+    prod = 1.0;
+    for (int i = 0; i < N_TRAIN; ++i) {
+      const double beta = fmin(1.0 - fcos((i + 1.0) / N_TRAIN) / fcos((double)i / N_TRAIN), 0.999);
+      prod *= 1.0 - beta;
+      c->alphabar[KIMODO_SCHEDULE_COSINE][i] = prod;
     }
     std::vector<float> pe((size_t)N_TRAIN * D);
     for (int p = 0; p < N_TRAIN; ++p)
@@ -543,6 +632,10 @@ int kimodo_load_weights(kimodo_ctx** out_ctx, const float* host_blob, size_t n_f
       return fail(set_error(KIMODO_ECUDA, "pe upload"));
     if (cudaMalloc(&c->derr, sizeof(DevError)) != cudaSuccess) return fail(set_error(KIMODO_ENOMEM, "error word"));
     cudaMemset(c->derr, 0, sizeof(DevError));
+    if (cudaMalloc(&c->sk_partial, gemm_sk_workspace_floats() * 4) != cudaSuccess ||
+        cudaMalloc(&c->sk_flags, 2 * GEMM_SK_MAX_PAIRS * sizeof(int)) != cudaSuccess)
+      return fail(set_error(KIMODO_ENOMEM, "stream-K workspace"));
+    cudaMemset(c->sk_flags, 0, 2 * GEMM_SK_MAX_PAIRS * sizeof(int));
   }
 
   // weights: plan the arena, stage the fp32 blob on the device, convert
@@ -576,6 +669,9 @@ void kimodo_free(kimodo_ctx* c) {
   free_graphs(c);
   for (auto e : c->ev_pool) cudaEventDestroy(e);
   if (c->ws.arena) cudaFree(c->ws.arena);
+  if (c->zbuf) cudaFree(c->zbuf);
+  if (c->sk_partial) cudaFree(c->sk_partial);
+  if (c->sk_flags) cudaFree(c->sk_flags);
   if (c->warena) cudaFree(c->warena);
   if (c->pe) cudaFree(c->pe);
   if (c->derr) cudaFree(c->derr);
@@ -597,28 +693,71 @@ int kimodo_denoiser_forward(kimodo_ctx* c, int net, const float* x, const float*
   Workspace& w = c->ws;
   NetW& n = c->net[net];
   KD_TRY(stage_lengths(c, lengths, batch, frames, st));
+  c->tk = plan_tokens(lengths, batch, batch, frames);
+  KD_TRY(enqueue_token_map(c, batch, batch, st));
   KD_CUDA(cudaMemcpyAsync(w.x, x, (size_t)batch * frames * n.din * 4, cudaMemcpyDefault, st));
   KD_CUDA(cudaMemcpyAsync(w.st_text, emb, (size_t)batch * DTXT * 4, cudaMemcpyDefault, st));
   KD_TRY(launch(c, CLS_SETUP, 0, (double)batch * DTXT * 6, st, "pack_embeddings", [&] {
     return pack_embeddings(w.st_text, batch, nullptr, 1, 0, w.emb, c->bf16(), st);
   }));
-  KD_TRY(timestep_rows(c, t, 1, 1, st));
+  KD_TRY(timestep_rows(c, t, 0, 1, st));
   KD_TRY(condition_setup(c, net, batch, 1, st));
   void* A = net == 0 ? w.A_root : w.A_body;
   const int lda = net == 0 ? ROOT_IN_LD : BODY_IN_LD;
   KD_TRY(launch(c, CLS_MOTION, 0, (double)batch * frames * n.din * 8, st, "pack_frames", [&] {
-    return pack_frames(w.x, batch, n.din, 0, n.din, A, c->bf16(), lda, 0, batch, frames, frames + 1, st);
+    return pack_frames(w.x, batch, n.din, 0, n.din, A, c->bf16(), lda, 0, batch, frames, frames + 1, st,
+                       c->tk.packed ? w.tok0 : nullptr, w.lengths, batch);
   }));
   float* hat = net == 0 ? w.root_hat : w.body_hat;
+  // the packed layout has no rows for padded frames: their outputs are the zeros set here
+  if (c->tk.packed) KD_CUDA(cudaMemsetAsync(hat, 0, (size_t)batch * frames * n.dout * 4, st));
   KD_TRY(run_net(c, net, batch, frames, batch, A, w.tmlp[net], w.txt[net], hat, st));
   KD_CUDA(cudaMemcpyAsync(out, hat, (size_t)batch * frames * n.dout * 4, cudaMemcpyDefault, st));
   c->last_launches = c->launches - l0;
   return finish_outputs(c, out, st);
 }
 
+// Validates the sampler options; n_z = floats of step noise the call reads when eta > 0.
+static int check_sampler(kimodo_ctx* c, const kimodo_sampler* o, size_t n_z, Sampler* out, cudaStream_t st) {
+  *out = Sampler();
+  if (!o) return KIMODO_OK;
+  if (o->schedule != KIMODO_SCHEDULE_LINEAR && o->schedule != KIMODO_SCHEDULE_COSINE)
+    return set_error(KIMODO_EINVAL, "unknown schedule %d", o->schedule);
+  if (!isfinite(o->eta) || o->eta < 0.f || o->eta > 1.f)
+    return set_error(KIMODO_EINVAL, "eta must be in [0, 1]");
+  out->schedule = o->schedule;
+  out->eta = o->eta;
+  if (o->eta == 0.f) return KIMODO_OK;
+  if (!o->step_noise) return set_error(KIMODO_EINVAL, "eta > 0 needs step_noise");
+  if (is_device_memory(o->step_noise)) {
+    out->z = o->step_noise;
+    return KIMODO_OK;
+  }
+  if (c->zcap < n_z) {   // host draws: staged into a context buffer that only grows
+    if (c->zbuf) {
+      KD_CUDA(cudaStreamSynchronize(st));
+      cudaFree(c->zbuf);
+      c->zbuf = nullptr;
+      c->zcap = 0;
+    }
+    if (cudaMalloc(&c->zbuf, n_z * 4) != cudaSuccess) return set_error(KIMODO_ENOMEM, "step noise staging");
+    c->zcap = n_z;
+  }
+  KD_CUDA(cudaMemcpyAsync(c->zbuf, o->step_noise, n_z * 4, cudaMemcpyHostToDevice, st));
+  out->z = c->zbuf;
+  return KIMODO_OK;
+}
+
 int kimodo_ddim_step(kimodo_ctx* c, const float* x_t, const float* text_emb, const float* null_emb, int null_batch,
                      const int* lengths, int batch, int frames, int t, int t_prev, float cfg_scale, float* x_prev,
                      void* stream) {
+  return kimodo_ddim_step_ex(c, x_t, text_emb, null_emb, null_batch, lengths, batch, frames, t, t_prev, cfg_scale,
+                             nullptr, x_prev, stream);
+}
+
+int kimodo_ddim_step_ex(kimodo_ctx* c, const float* x_t, const float* text_emb, const float* null_emb,
+                        int null_batch, const int* lengths, int batch, int frames, int t, int t_prev,
+                        float cfg_scale, const kimodo_sampler* options, float* x_prev, void* stream) {
   g_last_error.clear();
   KD_TRY(check_ctx(c));
   if (!x_t || !text_emb || !null_emb || !x_prev) return set_error(KIMODO_EINVAL, "NULL tensor argument");
@@ -629,40 +768,46 @@ int kimodo_ddim_step(kimodo_ctx* c, const float* x_t, const float* text_emb, con
   if (null_batch != 1 && null_batch != batch)
     return set_error(KIMODO_EINVAL, "null_batch must be 1 or batch (got %d)", null_batch);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  Sampler smp;
+  KD_TRY(check_sampler(c, options, (size_t)batch * frames * MOTION_F, &smp, st));
   KD_TRY(ensure_workspace(c, 2 * batch, frames, 1));
   const long long l0 = c->launches;
   Workspace& w = c->ws;
   KD_TRY(stage_lengths(c, lengths, batch, frames, st));
+  c->tk = plan_tokens(lengths, batch, 2 * batch, frames);
+  KD_TRY(enqueue_token_map(c, batch, 2 * batch, st));
   KD_CUDA(cudaMemcpyAsync(w.x, x_t, (size_t)batch * frames * MOTION_F * 4, cudaMemcpyDefault, st));
   KD_CUDA(cudaMemcpyAsync(w.st_text, text_emb, (size_t)batch * DTXT * 4, cudaMemcpyDefault, st));
   KD_CUDA(cudaMemcpyAsync(w.st_null, null_emb, (size_t)null_batch * DTXT * 4, cudaMemcpyDefault, st));
   KD_TRY(launch(c, CLS_SETUP, 0, (double)2 * batch * DTXT * 6, st, "pack_embeddings", [&] {
     return pack_embeddings(w.st_text, batch, w.st_null, null_batch, batch, w.emb, c->bf16(), st);
   }));
-  KD_TRY(timestep_rows(c, t, 1, 1, st));
+  KD_TRY(timestep_rows(c, t, 0, 1, st));
   KD_TRY(condition_setup(c, 0, 2 * batch, 1, st));
   KD_TRY(condition_setup(c, 1, 2 * batch, 1, st));
   KD_TRY(pack_root_input(c, batch, 2 * batch, frames, st));
-  KD_TRY(two_stage_step(c, batch, frames, t, t_prev, cfg_scale, 0, false, st));
+  KD_TRY(two_stage_step(c, batch, frames, t, t_prev, cfg_scale, 0, false, smp, smp.z, st));
   KD_CUDA(cudaMemcpyAsync(x_prev, w.x, (size_t)batch * frames * MOTION_F * 4, cudaMemcpyDefault, st));
   c->last_launches = c->launches - l0;
   return finish_outputs(c, x_prev, st);
 }
 
 static int enqueue_sample(kimodo_ctx* c, int batch, int frames, int steps, float cfg, int null_batch,
-                          cudaStream_t st) {
-  const int stride = N_TRAIN / steps;
+                          const Sampler& smp, cudaStream_t st) {
   Workspace& w = c->ws;
+  KD_TRY(enqueue_token_map(c, batch, 2 * batch, st));
   KD_TRY(launch(c, CLS_SETUP, 0, (double)2 * batch * DTXT * 6, st, "pack_embeddings", [&] {
     return pack_embeddings(w.st_text, batch, w.st_null, null_batch, batch, w.emb, c->bf16(), st);
   }));
-  KD_TRY(timestep_rows(c, N_TRAIN - 1, stride, steps, st));
+  KD_TRY(timestep_rows(c, -1, steps, steps, st));
   KD_TRY(condition_setup(c, 0, 2 * batch, steps, st));
   KD_TRY(condition_setup(c, 1, 2 * batch, steps, st));
   KD_TRY(pack_root_input(c, batch, 2 * batch, frames, st));
+  const size_t zstep = (size_t)batch * frames * MOTION_F;
   for (int k = 0; k < steps; ++k) {
-    const int t = N_TRAIN - 1 - k * stride;
-    KD_TRY(two_stage_step(c, batch, frames, t, t - stride, cfg, k, k + 1 < steps, st));
+    const float* z = smp.z ? smp.z + k * zstep : nullptr;
+    KD_TRY(two_stage_step(c, batch, frames, trailing_t(k, steps), trailing_t(k + 1, steps), cfg, k, k + 1 < steps,
+                          smp, z, st));
   }
   return KIMODO_OK;
 }
@@ -670,19 +815,28 @@ static int enqueue_sample(kimodo_ctx* c, int batch, int frames, int steps, float
 int kimodo_ddim_sample(kimodo_ctx* c, const float* text_emb, const float* null_emb, int null_batch,
                        const float* noise, const int* lengths, int batch, int frames, int steps, float cfg_scale,
                        float* out, void* stream) {
+  return kimodo_ddim_sample_ex(c, text_emb, null_emb, null_batch, noise, lengths, batch, frames, steps, cfg_scale,
+                               nullptr, out, stream);
+}
+
+int kimodo_ddim_sample_ex(kimodo_ctx* c, const float* text_emb, const float* null_emb, int null_batch,
+                          const float* noise, const int* lengths, int batch, int frames, int steps, float cfg_scale,
+                          const kimodo_sampler* options, float* out, void* stream) {
   g_last_error.clear();
   KD_TRY(check_ctx(c));
   if (!text_emb || !null_emb || !noise || !out) return set_error(KIMODO_EINVAL, "NULL tensor argument");
   KD_TRY(check_shape(batch, frames));
-  if (steps < 1 || steps > N_TRAIN || N_TRAIN % steps)
-    return set_error(KIMODO_EINVAL, "steps must divide %d (got %d)", N_TRAIN, steps);
+  if (steps < 1 || steps > N_TRAIN) return set_error(KIMODO_EINVAL, "steps must be in [1, %d] (got %d)", N_TRAIN, steps);
   if (!isfinite(cfg_scale)) return set_error(KIMODO_EINVAL, "cfg_scale must be finite");
   if (null_batch != 1 && null_batch != batch)
     return set_error(KIMODO_EINVAL, "null_batch must be 1 or batch (got %d)", null_batch);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  Sampler smp;
+  KD_TRY(check_sampler(c, options, (size_t)steps * batch * frames * MOTION_F, &smp, st));
   KD_TRY(ensure_workspace(c, 2 * batch, frames, steps));
   Workspace& w = c->ws;
   KD_TRY(stage_lengths(c, lengths, batch, frames, st));
+  c->tk = plan_tokens(lengths, batch, 2 * batch, frames);
   KD_CUDA(cudaMemcpyAsync(w.x, noise, (size_t)batch * frames * MOTION_F * 4, cudaMemcpyDefault, st));
   KD_CUDA(cudaMemcpyAsync(w.st_text, text_emb, (size_t)batch * DTXT * 4, cudaMemcpyDefault, st));
   KD_CUDA(cudaMemcpyAsync(w.st_null, null_emb, (size_t)null_batch * DTXT * 4, cudaMemcpyDefault, st));
@@ -693,7 +847,7 @@ int kimodo_ddim_sample(kimodo_ctx* c, const float* text_emb, const float* null_e
     // The graph is not cached: its event nodes belong to this profile.
     KD_CUDA(cudaStreamBeginCapture(c->cap_stream, cudaStreamCaptureModeThreadLocal));
     c->prof_flags = cudaEventRecordExternal;
-    int s = enqueue_sample(c, batch, frames, steps, cfg_scale, null_batch, c->cap_stream);
+    int s = enqueue_sample(c, batch, frames, steps, cfg_scale, null_batch, smp, c->cap_stream);
     c->prof_flags = cudaEventRecordDefault;
     cudaGraph_t g = nullptr;
     cudaError_t e = cudaStreamEndCapture(c->cap_stream, &g);
@@ -712,14 +866,16 @@ int kimodo_ddim_sample(kimodo_ctx* c, const float* text_emb, const float* null_e
     if (e != cudaSuccess) return set_error(KIMODO_ECUDA, "profiled graph failed: %s", cudaGetErrorString(e));
     c->last_launches = c->launches - l0;
   } else {
-    uint32_t cfg_bits;
+    uint32_t cfg_bits, eta_bits;
     memcpy(&cfg_bits, &cfg_scale, 4);
-    const auto key = std::make_tuple(batch, frames, steps, null_batch == 1 ? 1 : 0, cfg_bits);
+    memcpy(&eta_bits, &smp.eta, 4);
+    const auto key = std::make_tuple(batch, frames, steps, null_batch == 1 ? 1 : 0, cfg_bits, smp.schedule, eta_bits,
+                                     smp.z, c->tk.packed ? c->tk.M : -1);
     auto it = c->graphs.find(key);
     if (it == c->graphs.end()) {
       KD_CUDA(cudaStreamBeginCapture(c->cap_stream, cudaStreamCaptureModeThreadLocal));
       const long long lc = c->launches;
-      int s = enqueue_sample(c, batch, frames, steps, cfg_scale, null_batch, c->cap_stream);
+      int s = enqueue_sample(c, batch, frames, steps, cfg_scale, null_batch, smp, c->cap_stream);
       cudaGraph_t g = nullptr;
       cudaError_t e = cudaStreamEndCapture(c->cap_stream, &g);
       if (s != KIMODO_OK) {
@@ -748,6 +904,8 @@ int kimodo_sync_status(kimodo_ctx* c, void* stream) {
   KD_CUDA(cudaMemcpy(&h, c->derr, sizeof(h), cudaMemcpyDeviceToHost));
   if (h.code != 0) {
     KD_CUDA(cudaMemset(c->derr, 0, sizeof(DevError)));
+    // an interrupted stream-K launch may leave contributor counters raised
+    KD_CUDA(cudaMemset(c->sk_flags, 0, 2 * GEMM_SK_MAX_PAIRS * sizeof(int)));
     return set_error(h.code, "device wait timed out in kernel stage %d (block %d)", h.where, h.block);
   }
   return KIMODO_OK;
@@ -812,6 +970,7 @@ int prepared_device() {
   if (!done[dev]) {
     KD_CUDA(gemm_tc_prepare());
     KD_CUDA(gemm_tc2_prepare());
+    KD_CUDA(gemm_sk_prepare());
     KD_CUDA(attention_prepare());
     done[dev] = true;
   }
@@ -884,6 +1043,41 @@ int kimodo_gemm_bf16_pair(const void* A, int lda, const void* W, int ldw, const 
   ep.bias = bias; ep.out = out; ep.ldo = ldo; ep.resid = resid; ep.ldr = ldr; ep.N = N; ep.M = M;
   const int bn = tile_n ? tile_n : gemm_tc2_pick_bn(M, N, epilogue);
   KD_CUDA(gemm_tc2(g, bn, epilogue, out_f32 != 0, ep, kernel_error_word(), static_cast<cudaStream_t>(stream)));
+  return KIMODO_OK;
+}
+
+int kimodo_gemm_bf16_streamk(const void* A, int lda, const void* W, int ldw, const float* bias, const void* resid,
+                             int ldr, void* out, int ldo, int M, int N, int K, int epilogue, int out_f32,
+                             void* stream) {
+  g_last_error.clear();
+  KD_TRY(check_gemm_args(A, lda, W, ldw, bias, resid, out, ldo, M, N, K, epilogue));
+  if (lda % 8 || ldw % 8 || (reinterpret_cast<uintptr_t>(A) & 15) || (reinterpret_cast<uintptr_t>(W) & 15))
+    return set_error(KIMODO_EINVAL, "bf16 operands need 16-byte aligned rows (lda, ldw multiples of 8)");
+  if (ldo % 4 || (reinterpret_cast<uintptr_t>(out) & 15) || (epilogue == 3 && (ldr % 4 ||
+      (reinterpret_cast<uintptr_t>(resid) & 15))) || (reinterpret_cast<uintptr_t>(bias) & 15))
+    return set_error(KIMODO_EINVAL, "out, resid and bias need 16-byte alignment and ldo, ldr multiples of 4");
+  if (!gemm_tc2_supports(epilogue, out_f32 != 0))
+    return set_error(KIMODO_EINVAL, "pair GEMM epilogues: bias or GELU with bf16 output, residual with fp32 output");
+  if (N % 16 || ((long)ldo * (out_f32 ? 4 : 2)) % 16)
+    return set_error(KIMODO_EINVAL, "pair GEMM needs N % 16 == 0 and 16-byte output rows");
+  KD_TRY(prepared_device());
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // a workspace of its own for this call, stream-ordered
+  float* partial = nullptr;
+  int* flags = nullptr;
+  KD_CUDA(cudaMallocAsync(reinterpret_cast<void**>(&partial), gemm_sk_workspace_floats() * 4, st));
+  cudaError_t e = cudaMallocAsync(reinterpret_cast<void**>(&flags), 2 * GEMM_SK_MAX_PAIRS * sizeof(int), st);
+  if (e == cudaSuccess) e = cudaMemsetAsync(flags, 0, 2 * GEMM_SK_MAX_PAIRS * sizeof(int), st);
+  if (e == cudaSuccess) {
+    GemmArgs g;
+    g.A = A; g.B = W; g.M = M; g.N = N; g.K = K; g.lda = lda; g.ldb = ldw;
+    EpiParams ep;
+    ep.bias = bias; ep.out = out; ep.ldo = ldo; ep.resid = resid; ep.ldr = ldr; ep.N = N; ep.M = M;
+    e = gemm_sk(g, epilogue, out_f32 != 0, ep, partial, flags, kernel_error_word(), st);
+  }
+  if (flags) cudaFreeAsync(flags, st);
+  cudaFreeAsync(partial, st);
+  KD_CUDA(e);
   return KIMODO_OK;
 }
 
@@ -1056,12 +1250,13 @@ extern "C" int kimodo_denoiser_forward_noalloc(kimodo_ctx* c, int net, const flo
   KD_CUDA(cudaMemsetAsync(w.A_root, 0, (size_t)rows * ROOT_IN_LD * c->elem(), st));
   KD_CUDA(cudaMemsetAsync(w.A_body, 0, (size_t)rows * BODY_IN_LD * c->elem(), st));
   KD_TRY(stage_lengths(c, lengths, batch, frames, st));
+  c->tk = Tokens{rows, false};   // the scratch holds the padded layout only
   KD_CUDA(cudaMemcpyAsync(w.x, x, (size_t)batch * frames * n.din * 4, cudaMemcpyDefault, st));
   KD_CUDA(cudaMemcpyAsync(w.st_text, emb, (size_t)batch * DTXT * 4, cudaMemcpyDefault, st));
   KD_TRY(launch(c, CLS_SETUP, 0, (double)batch * DTXT * 6, st, "pack_embeddings", [&] {
     return pack_embeddings(w.st_text, batch, nullptr, 1, 0, w.emb, c->bf16(), st);
   }));
-  KD_TRY(timestep_rows(c, t, 1, 1, st));
+  KD_TRY(timestep_rows(c, t, 0, 1, st));
   KD_TRY(condition_setup(c, net, batch, 1, st));
   void* A = net == 0 ? w.A_root : w.A_body;
   const int lda = net == 0 ? ROOT_IN_LD : BODY_IN_LD;

@@ -33,7 +33,11 @@ struct EpiParams {
   const float* tvec = nullptr;   // timestep-MLP output [N] for this call's timestep
   const int* lengths = nullptr;  // valid frames per sequence, indexed seq % len_mod
   int len_mod = 1;
-  int S = 1;                     // tokens per sequence
+  int S = 1;                     // tokens per sequence (padded layout)
+  // packed layout (valid tokens only): sequence s owns rows [tok0[s], tok0[s + 1]) and
+  // row_seq[r] is the sequence of row r; both null for the padded layout (row = s * S + pos)
+  const int* tok0 = nullptr;
+  const int* row_seq = nullptr;
   int T = 1;                     // frames per sequence (EPI_OUTPROJ)
   int N = 0;                     // valid output columns
   int M = 0;                     // valid rows
@@ -129,13 +133,25 @@ template <typename T> __device__ __forceinline__ T from_f(float v);
 template <> __device__ __forceinline__ float from_f<float>(float v) { return v; }
 template <> __device__ __forceinline__ bf16 from_f<bf16>(float v) { return __float2bfloat16_rn(v); }
 
+// (sequence, position) of token row `row` in either layout.
+__device__ __forceinline__ void token_of_row(const EpiParams& e, int row, int& seq, int& pos) {
+  if (e.row_seq != nullptr) {
+    seq = e.row_seq[row];
+    pos = row - e.tok0[seq];
+  } else {
+    seq = row / e.S;
+    pos = row - seq * e.S;
+  }
+}
+
 // Apply the epilogue to `n` consecutive columns [col0, col0 + n) of row `row`.
 // acc[i] holds column col0 + i.  OutT is the stored type, ResT the residual type.
 template <int KIND, typename OutT, typename ResT, int NV>
 __device__ __forceinline__ void epilogue_row(const EpiParams& e, int row, int col0, const float (&acc)[NV]) {
   if (row >= e.M) return;
   if constexpr (KIND == EPI_OUTPROJ) {
-    const int seq = row / e.S, pos = row - seq * e.S;
+    int seq, pos;
+    token_of_row(e, row, seq, pos);
     if (pos == 0) return;
     const int frame = pos - 1;
     const bool valid = frame < e.lengths[seq % e.len_mod];
@@ -149,7 +165,8 @@ __device__ __forceinline__ void epilogue_row(const EpiParams& e, int row, int co
   } else {
     float v[NV];
     if constexpr (KIND == EPI_INPROJ) {
-      const int seq = row / e.S, pos = row - seq * e.S;
+      int seq, pos;
+      token_of_row(e, row, seq, pos);
       if (pos == 0) {
 #pragma unroll
         for (int i = 0; i < NV; ++i) {
@@ -268,7 +285,8 @@ __device__ __forceinline__ void epilogue_prefetch(const EpiParams& e, int row0, 
       if constexpr (KIND == EPI_BIAS_RESID) {
         pre[p] = ld4(reinterpret_cast<const float*>(e.resid) + (long)row * e.ldr + col);
       } else {
-        const int pos = row % e.S;
+        int seq, pos;
+        token_of_row(e, row, seq, pos);
         pre[p] = ld4(e.pe + (long)pos * e.N + col);
       }
     }
@@ -294,7 +312,8 @@ __device__ __forceinline__ void epilogue_warp_tile(const EpiParams& e, const flo
     const float4 a = *reinterpret_cast<const float4*>(st + r * Ln::LDE + cq);
     float v[4] = {a.x, a.y, a.z, a.w};
     if constexpr (KIND == EPI_OUTPROJ) {
-      const int seq = row / e.S, pos = row - seq * e.S;
+      int seq = 0, pos = 0;
+      if (in_rows) token_of_row(e, row, seq, pos);
       if (in_rows && pos != 0) {
         const int frame = pos - 1;
         const bool valid = frame < e.lengths[seq % e.len_mod];
@@ -305,7 +324,8 @@ __device__ __forceinline__ void epilogue_warp_tile(const EpiParams& e, const flo
       }
     } else {
       if constexpr (KIND == EPI_INPROJ) {
-        const int seq = row / e.S, pos = row - seq * e.S;
+        int seq = 0, pos = 1;
+        if (in_rows) token_of_row(e, row, seq, pos);
         if (pos == 0) {
           const float4 cv = ld4(e.cond + (long)seq * e.N + col);
           const float4 tv = ld4(e.tvec + col);

@@ -30,6 +30,17 @@ int make_tmap_bf16(CUtensorMap* m, const void* base, int rows, int cols, int ld,
 int make_tmap_plain(CUtensorMap* m, const void* base, int elem, int rows, int cols, long ld, int box_cols,
                     int box_rows, int swizzle);
 
+// Stream-K tcgen05 GEMM on CTA pairs (256 x 256 tiles, equal k-block shares per pair).
+// Kinds: EPI_BIAS / EPI_BIAS_GELU with bf16 output, EPI_BIAS_RESID with fp32 output
+// (residual read from global memory; may alias the output).  N % 16 == 0.  partial:
+// gemm_sk_workspace_floats() floats; flags: 2 * GEMM_SK_MAX_PAIRS ints, zero before the
+// first launch (each launch leaves them zero).  Launches on one workspace must not overlap.
+constexpr int GEMM_SK_MAX_PAIRS = 80;
+cudaError_t gemm_sk_prepare();
+size_t gemm_sk_workspace_floats();
+cudaError_t gemm_sk(const GemmArgs& g, int kind, bool out_f32, const EpiParams& ep, float* partial, int* flags,
+                    DevError* err, cudaStream_t st);
+
 // tcgen05 GEMM on CTA pairs (256-row tiles).  bn in {144, 160, 208, 256} for EPI_BIAS /
 // EPI_BIAS_GELU with bf16 output, {144, 160} for EPI_BIAS_RESID with fp32 output.
 cudaError_t gemm_tc2(const GemmArgs& g, int bn, int kind, bool out_f32, const EpiParams& ep, DevError* err,
@@ -46,13 +57,19 @@ size_t attention_bf16_smem(int S);
 // fp32 SIMT GEMM with the same epilogues (fp32 everywhere).  K % 16 == 0.
 cudaError_t gemm_f32(const GemmArgs& g, int kind, const EpiParams& ep, cudaStream_t st);
 
-// Masked multi-head self-attention over the fused QKV matrix [nseq*S, 3*D]
-// (columns Q | K | V, head h at h*DH).  Keys at token index >= 1 + lengths[seq %
-// len_mod] are excluded.  out [nseq*S, D].
+// Masked multi-head self-attention over the fused QKV matrix (columns Q | K | V,
+// head h at h*DH).  Padded layout (tok0 null): sequence s owns rows s*S .. s*S + S - 1
+// and keys at token index >= 1 + lengths[s % len_mod] are excluded.  Packed layout:
+// sequence s owns rows tok0[s] .. tok0[s + 1] - 1 (its valid tokens only; S is then
+// the largest sequence).  out has the rows of qkv, D columns.
 cudaError_t attention_bf16(const bf16* qkv, bf16* out, const int* lengths, int len_mod, int nseq, int S,
-                           cudaStream_t st);
+                           cudaStream_t st, const int* tok0 = nullptr);
 cudaError_t attention_f32(const float* qkv, float* out, const int* lengths, int len_mod, int nseq, int S,
-                          cudaStream_t st);
+                          cudaStream_t st, const int* tok0 = nullptr);
+
+// Token layout of a batch: tok0[s] = sum over s' < s of (1 + lengths[s' % len_mod]) for
+// s <= nseq, and row_seq[r] = s for the rows r of sequence s (one CTA).
+cudaError_t build_token_map(const int* lengths, int len_mod, int nseq, int* tok0, int* row_seq, cudaStream_t st);
 
 // Row LayerNorm over D features: y fp32 [M, D] -> out (bf16 or fp32) [M, D], and
 // optionally an fp32 copy into out32 (which may be y itself).
@@ -61,29 +78,37 @@ cudaError_t layernorm(const float* y, void* out, bool out_bf16, const float* gam
 
 // ---- motion / sampler kernels (element type of the activation matrices: bf16 or fp32)
 
-// A[(seq*S + 1 + i) * lda + col0 + f] = src[((seq % nsrc) * T + i) * ld_src + f0 + f], f < nf, i < T.
+// A[(row(seq, i)) * lda + col0 + f] = src[((seq % nsrc) * T + i) * ld_src + f0 + f], f < nf, with
+// row(seq, i) = seq*S + 1 + i for every i < T (padded layout, tok0 null) or tok0[seq] + 1 + i
+// for the valid frames i < lengths[seq % len_mod] only (packed layout).
 cudaError_t pack_frames(const float* src, int nsrc, int ld_src, int f0, int nf, void* A, bool a_bf16, int lda,
-                        int col0, int nseq, int T, int S, cudaStream_t st);
+                        int col0, int nseq, int T, int S, cudaStream_t st, const int* tok0 = nullptr,
+                        const int* lengths = nullptr, int len_mod = 1);
 
-// Body-network input of the two-stage step: for seq in [0, nseq), frame i < T:
+// Body-network input of the two-stage step: for seq in [0, nseq), frame i < T (padded
+// layout) or i < lengths[seq % B] (packed layout, rows as pack_frames):
 //   A[.., 0:274] = x[seq % B, i, 5:279];  A[.., 274:279] = G2L(root_hat[seq])[i]  (0 for padded frames)
 cudaError_t g2l_body_input(const float* root_hat, const float* x, const int* lengths, int B, int nseq, int T,
-                           int S, void* A, bool a_bf16, int lda, cudaStream_t st);
+                           int S, void* A, bool a_bf16, int lda, cudaStream_t st, const int* tok0 = nullptr);
 
 // CFG + DDIM update in place on x [B, T, 279]: x0 = u + w (c - u) from the root /
-// body predictions of sequences b (cond) and B + b (uncond); x = c0 x0 + c1 x;
-// padded frames 0.  If A_next != nullptr the new root features are also packed
-// into the root network's input matrix for sequences b and B + b.
+// body predictions of sequences b (cond) and B + b (uncond); x = c0 x0 + c1 x
+// (+ c2 z when z [B, T, 279] is given); padded frames 0.  If A_next != nullptr the
+// new root features are also packed into the root network's input matrix for
+// sequences b and B + b.
 cudaError_t cfg_ddim(const float* root_hat, const float* body_hat, float* x, const int* lengths, int B, int T,
-                     float w, float c0, float c1, void* A_next, bool a_bf16, int lda, int S, cudaStream_t st);
+                     float w, float c0, float c1, const float* z, float c2, void* A_next, bool a_bf16, int lda, int S,
+                     cudaStream_t st, const int* tok0 = nullptr);
 
 // Condition inputs: rows [0, B) = text_emb, rows [B, B + nnull_rows) = null_emb
 // (row (r - B) % null_batch).  out (bf16 or fp32) [rows, DTXT].
 cudaError_t pack_embeddings(const float* text_emb, int B, const float* null_emb, int null_batch, int null_rows,
                             void* out, bool out_bf16, cudaStream_t st);
 
-// out[k, :] = pe[t0 - k * stride, :] for k < n (sinusoid rows of the timesteps).
-cudaError_t gather_timestep_rows(const float* pe, int t0, int stride, int n, void* out, bool out_bf16,
+// out[k, :] = pe[t_k, :] for k < n (sinusoid rows of the timesteps): t_k = t_single
+// when steps == 0, else the k-th trailing timestep of a `steps`-step sampler,
+// floor(N_TRAIN (steps - k) / steps + 1/2) - 1.
+cudaError_t gather_timestep_rows(const float* pe, int t_single, int steps, int n, void* out, bool out_bf16,
                                  cudaStream_t st);
 
 }  // namespace kd
