@@ -86,6 +86,12 @@ KIMODO_API int kimodo_attention_bf16(const void* qkv, void* out, const int* leng
 KIMODO_API int kimodo_attention_f32(const float* qkv, float* out, const int* lengths, int nseq, int S,
                                     void* stream);
 
+/* The bf16 attention on the tcgen05 tensor cores: one CTA per (head, sequence,
+ * 128-query tile), S = Q K^T and O = P V in TMEM, exact softmax over all keys of a
+ * sequence.  Arguments as kimodo_attention_bf16; qkv 16-byte aligned. */
+KIMODO_API int kimodo_attention_bf16_tc(const void* qkv, void* out, const int* lengths, int nseq, int S,
+                                        void* stream);
+
 /* LayerNorm over 1024 features, eps 1e-5, biased variance: y fp32 [M, 1024] ->
  * out bf16 (out_bf16 = 1) or fp32 [M, 1024]; gamma, beta fp32 [1024]. */
 KIMODO_API int kimodo_layernorm(const float* y, void* out, int out_bf16, const float* gamma,

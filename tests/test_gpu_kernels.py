@@ -242,13 +242,14 @@ def _attention_ref(qkv, lengths, S):
 
 
 @pytest.mark.parametrize("S,lengths", [(31, [30]), (151, [150, 60, 0]), (301, [300, 123]), (64, [63, 64])])
-def test_attention_bf16_vs_oracle(S, lengths):
+@pytest.mark.parametrize("tc", [False, True])
+def test_attention_bf16_vs_oracle(S, lengths, tc):
     require_cuda()
     lengths = [min(n, S - 1) for n in lengths]
     nseq = len(lengths)
     qkv = _bf16(synth.random_vectors((nseq * S, 3072), S + 100))
     L = torch.tensor(lengths, dtype=torch.int32)
-    out = kb.attention(qkv.cuda(), L.cuda(), nseq, S)
+    out = kb.attention(qkv.cuda(), L.cuda(), nseq, S, tc=tc)
     ref = _attention_ref(_f64(qkv), lengths, S)
     got = out.float().cpu().double().numpy()
     err = np.linalg.norm(got - ref) / np.linalg.norm(ref)
@@ -256,16 +257,17 @@ def test_attention_bf16_vs_oracle(S, lengths):
     assert np.abs(got - ref).max() < 3e-2 * np.abs(ref).max()
 
 
-def test_attention_bf16_masked_keys_never_read():
+@pytest.mark.parametrize("tc", [False, True])
+def test_attention_bf16_masked_keys_never_read(tc):
     require_cuda()
     S, lengths = 151, [40, 150]
     qkv = _bf16(synth.random_vectors((2 * S, 3072), 77)).cuda()
     L = torch.tensor(lengths, dtype=torch.int32).cuda()
-    base = kb.attention(qkv, L, 2, S)
+    base = kb.attention(qkv, L, 2, S, tc=tc)
     poisoned = qkv.clone()
     for s, n in enumerate(lengths):
         poisoned[s * S + 1 + n:(s + 1) * S, 1024:] = float("nan")
-    again = kb.attention(poisoned, L, 2, S)
+    again = kb.attention(poisoned, L, 2, S, tc=tc)
     torch.cuda.synchronize()
     assert torch.equal(base, again)
 

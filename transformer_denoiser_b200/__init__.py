@@ -46,6 +46,7 @@ SIGNATURES = [
     ("kimodo_gemm_f32", _I, [_P, _I, _P, _I, _P, _P, _I, _P, _I, _I, _I, _I, _I, _P]),
     ("kimodo_attention_bf16", _I, [_P, _P, _P, _I, _I, _P]),
     ("kimodo_attention_f32", _I, [_P, _P, _P, _I, _I, _P]),
+    ("kimodo_attention_bf16_tc", _I, [_P, _P, _P, _I, _I, _P]),
     ("kimodo_layernorm", _I, [_P, _P, _I, _P, _P, _I, _P]),
 ]
 EPI_BIAS, EPI_BIAS_GELU, EPI_BIAS_SILU, EPI_BIAS_RESID = 0, 1, 2, 3
@@ -184,12 +185,16 @@ def gemm_f32(A, W, bias, epilogue=EPI_BIAS, resid=None, out=None, K=None):
     return out
 
 
-def attention(qkv, lengths, nseq, S):
-    """Masked attention over qkv [nseq*S, 3072] (bf16 or fp32 CUDA tensor)."""
+def attention(qkv, lengths, nseq, S, tc=False):
+    """Masked attention over qkv [nseq*S, 3072] (bf16 or fp32 CUDA tensor); tc=True runs
+    the tcgen05 kernel (bf16)."""
     import torch
     lib = load_library()
     out = torch.empty((nseq * S, 1024), dtype=qkv.dtype, device=qkv.device)
-    fn = lib.kimodo_attention_bf16 if qkv.dtype == torch.bfloat16 else lib.kimodo_attention_f32
+    if tc:
+        fn = lib.kimodo_attention_bf16_tc
+    else:
+        fn = lib.kimodo_attention_bf16 if qkv.dtype == torch.bfloat16 else lib.kimodo_attention_f32
     _check(fn(_ptr(qkv), _ptr(out), _ptr(lengths), nseq, S, _cur_stream()))
     return out
 

@@ -1,0 +1,300 @@
+// Masked multi-head self-attention on the tcgen05 tensor cores ("Kimodo WebGPU",
+// "WGSL compute shaders" table: multi-head self-attention with optional key masking).
+//
+// One CTA per (head, sequence, 128-query tile).  Every key of a sequence fits in
+// one pass (at most 301 tokens), so the softmax is exact, not online:
+//   1. TMA stages the query tile (128 x 128), and the keys and values of the
+//      sequence's rows rounded up to 64 (128-byte swizzle, no multicast).
+//   2. One thread issues S = Q K^T (M = 128, N = valid keys rounded up to 16,
+//      K = 128) into TMEM.
+//   3. Eight softmax warps (two per TMEM lane quarter, one query row per thread,
+//      half of the keys each) take the row maximum over the valid keys, form
+//      p = 2^((s - max) * log2(e) / sqrt(128)) (0 for keys at or beyond 1 + length,
+//      which are never read, so padded content, even NaN, cannot leak), sum it,
+//      and write P in bf16 into the key buffer (dead once S is formed) in the
+//      K-major 128-byte-swizzle layout.  They zero the value rows past the valid
+//      keys inside the MMA's K range, so 0 * garbage cannot occur either.
+//   4. The same thread issues O = P V (M = 128, N = 128, K = keys) with V read in
+//      place as an MN-major operand; the softmax warps scale O by 1 / sum and store
+//      the valid query rows in bf16.
+// Rows of the key and value tiles past the sequence belong to other tokens or lie
+// outside the matrix (zero fill) and are masked as above.  Every wait is bounded.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+#include "epilogue.cuh"
+#include "kernels.h"
+#include "launch.cuh"
+#include "ptx.cuh"
+
+namespace kd {
+namespace {
+
+constexpr int QT = 128;                    // query rows per CTA
+constexpr int KB_ROWS = 64;                // key rows per TMA box
+constexpr int SM_WARPS = 8;                // softmax / epilogue warps
+constexpr int NUM_THREADS = 64 + 32 * SM_WARPS;
+constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;
+constexpr int KIMODO_ETIMEOUT_CODE = -5;
+constexpr uint32_t O_COL = 320;            // TMEM column of the O accumulator (S uses columns 0..303)
+constexpr uint32_t TMEM_COLS = 512;
+constexpr int MAX_KA = ((MAX_FRAMES + 1 + KB_ROWS - 1) / KB_ROWS) * KB_ROWS;   // 320 key rows
+constexpr uint32_t Q_BYTES = QT * DH * 2;  // two 64-column halves of 16 KB
+
+// Shared memory: Q [2 halves][128 rows][128 B], K [2 halves][KA rows][128 B] (later P
+// [KA / 64 blocks][128 rows][128 B]), V [2 halves][KA rows][128 B], then barriers and
+// the row-statistics exchange.
+constexpr size_t smem_bytes(int ka) {
+  return 1024 + Q_BYTES + 2 * (size_t)ka * 256 + 8 * 8 + 2 * 2 * QT * 4 + 16;
+}
+
+__device__ __forceinline__ void record_timeout(DevError* err, volatile int* abort) {
+  *abort = 1;
+  if (err && atomicCAS(&err->code, 0, KIMODO_ETIMEOUT_CODE) == 0) {
+    err->where = WHERE_ATTENTION;
+    err->block = blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z);
+  }
+}
+
+// Shared-memory descriptor of an MN-major operand in the 128-byte swizzle layout:
+// 64-element atoms along MN `lbo` bytes apart, 8-row groups along K 1024 bytes apart.
+__device__ __forceinline__ uint64_t smem_desc_sw128_mn(uint32_t saddr, uint32_t lbo) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)(1024u >> 4) << 32;
+  d |= (uint64_t)1u << 46;
+  d |= (uint64_t)2u << 61;
+  return d;
+}
+
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmKV,
+               bf16* __restrict__ out, const int* __restrict__ lengths, int len_mod, int S_pad, int ka,
+               const int* __restrict__ tok0, DevError* err) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sQ = ptx::smem_u32(smem);
+  const uint32_t sK = sQ + Q_BYTES;                       // also P
+  const uint32_t sV = sK + (uint32_t)ka * 256;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Q_BYTES + (size_t)ka * 512);
+  const uint32_t bar0 = ptx::smem_u32(bars);
+  const uint32_t bar_qk = bar0, bar_v = bar0 + 8, bar_s = bar0 + 16, bar_p = bar0 + 24, bar_o = bar0 + 32;
+  float* xmax = reinterpret_cast<float*>(bars + 8);      // [2][QT] partial row maxima, then sums
+  float* xsum = xmax + 2 * QT;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(xsum + 2 * QT);
+  volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int h = blockIdx.x, seq = blockIdx.y, qt = blockIdx.z;
+  ptx::pdl_wait();
+  ptx::pdl_trigger();
+  const long row0 = tok0 ? tok0[seq] : (long)seq * S_pad;
+  const int S = tok0 ? tok0[seq + 1] - tok0[seq] : S_pad;
+  if (qt * QT >= S) return;   // uniform over the CTA: nothing allocated yet
+  int n_valid = 1 + lengths[seq % len_mod];
+  n_valid = n_valid < 1 ? 1 : (n_valid > S ? S : n_valid);
+  const int n_cols = (n_valid + 15) & ~15;                 // MMA N for S = Q K^T, K range of O = P V
+  const int n_boxes = (n_valid + KB_ROWS - 1) / KB_ROWS;   // 64-row key / value boxes
+
+  if (threadIdx.x == 0) {
+    ptx::mbar_init(bar_qk, 1);
+    ptx::mbar_init(bar_v, 1);
+    ptx::mbar_init(bar_s, 1);
+    ptx::mbar_init(bar_p, SM_WARPS);
+    ptx::mbar_init(bar_o, 1);
+    ptx::fence_mbar_init();
+    *abort = (err != nullptr && *reinterpret_cast<volatile int*>(&err->code) != 0) ? 1 : 0;
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc(ptx::smem_u32(tmem_slot), TMEM_COLS);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const bool skip = *abort != 0;
+
+  if (warp == 0) {
+    if (lane == 0 && !skip) {
+      // ---------------- TMA: Q tile and keys first (for S), then values
+      ptx::tma_prefetch_desc(&tmQ);
+      ptx::tma_prefetch_desc(&tmKV);
+      const int qrow = (int)row0 + qt * QT;
+      ptx::mbar_arrive_expect_tx(bar_qk, Q_BYTES + (uint32_t)n_boxes * 2 * KB_ROWS * 128);
+      for (int hf = 0; hf < 2; ++hf) ptx::tma_load_2d(sQ + hf * (QT * 128), &tmQ, bar_qk, h * DH + hf * 64, qrow);
+      for (int b = 0; b < n_boxes; ++b)
+        for (int hf = 0; hf < 2; ++hf)
+          ptx::tma_load_2d(sK + (uint32_t)(hf * ka + b * KB_ROWS) * 128, &tmKV, bar_qk, D + h * DH + hf * 64,
+                           (int)row0 + b * KB_ROWS);
+      ptx::mbar_arrive_expect_tx(bar_v, (uint32_t)n_boxes * 2 * KB_ROWS * 128);
+      for (int b = 0; b < n_boxes; ++b)
+        for (int hf = 0; hf < 2; ++hf)
+          ptx::tma_load_2d(sV + (uint32_t)(hf * ka + b * KB_ROWS) * 128, &tmKV, bar_v, 2 * D + h * DH + hf * 64,
+                           (int)row0 + b * KB_ROWS);
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && !skip) {
+      // ---------------- MMA issuer
+      bool ok = ptx::mbar_wait_bounded(bar_qk, 0, abort, WAIT_LIMIT_NS);
+      if (ok) {
+        ptx::tc_fence_after();
+        // S = Q K^T in N chunks of at most 256 key columns
+        for (int n0 = 0; n0 < n_cols; n0 += 256) {
+          const int nn = n_cols - n0 < 256 ? n_cols - n0 : 256;
+          const uint32_t idesc = ptx::idesc_bf16_f32(QT, nn);
+#pragma unroll
+          for (int kk = 0; kk < DH / 16; ++kk) {
+            const uint32_t a = sQ + (kk >> 2) * (QT * 128) + (kk & 3) * 32;
+            const uint32_t b = sK + (uint32_t)((kk >> 2) * ka + n0) * 128 + (kk & 3) * 32;
+            ptx::tc_mma_bf16(tmem_base + n0, ptx::smem_desc_sw128(a), ptx::smem_desc_sw128(b), idesc, kk != 0);
+          }
+        }
+        ptx::tc_commit(bar_s);
+        ok = ptx::mbar_wait_bounded(bar_p, 0, abort, WAIT_LIMIT_NS);
+      }
+      if (ok) {
+        ptx::tc_fence_after();
+        // O = P V: A = P (K-major, 64-key blocks of 16 KB), B = V (MN-major, dim halves ka*128 B apart)
+        const uint32_t idesc = ptx::idesc_bf16_f32(QT, DH) | (1u << 16);
+        for (int kk = 0; kk < n_cols / 16; ++kk) {
+          const uint32_t a = sK + (kk >> 2) * (QT * 128) + (kk & 3) * 32;
+          const uint32_t b = sV + (uint32_t)kk * 16 * 128;
+          ptx::tc_mma_bf16(tmem_base + O_COL, ptx::smem_desc_sw128(a), smem_desc_sw128_mn(b, (uint32_t)ka * 128),
+                           idesc, kk != 0);
+        }
+        ptx::tc_commit(bar_o);
+        volatile int never = 0;
+        if (!ptx::mbar_wait_bounded(bar_o, 0, &never, WAIT_LIMIT_NS)) ok = false;
+      }
+      if (!ok && !*abort) record_timeout(err, abort);
+    }
+  } else if (!skip) {
+    // ---------------- softmax and epilogue warps: lane quarter q, key half kh
+    const int ew = warp - 2;
+    const int q = warp & 3, kh = ew >> 2;
+    const int r = q * 32 + lane;                 // query row within the tile
+    const uint32_t lane_addr = (uint32_t)(q * 32) << 16;
+    const int half_cols = ((n_cols / 16 + 1) / 2) * 16;       // key columns of half 0
+    const int c_beg = kh == 0 ? 0 : half_cols;
+    const int c_end = kh == 0 ? half_cols : n_cols;
+    const float sc = 0.08838834764831845f * 1.4426950408889634f;   // log2(e) / sqrt(128)
+    bool ok = true;
+
+    // zero the value rows n_valid .. n_cols - 1 (inside O = P V's K range) once they land
+    ok = ptx::mbar_wait_bounded(bar_v, 0, abort, WAIT_LIMIT_NS);
+    if (ok && n_cols > n_valid) {
+      const int nz = n_cols - n_valid;
+      for (int i = ew * 32 + lane; i < nz * 2 * 8; i += SM_WARPS * 32) {
+        const int row = n_valid + i / 16, hf = (i / 8) & 1, c = i & 7;
+        *reinterpret_cast<uint4*>(smem + Q_BYTES + (size_t)ka * 256 + ((size_t)hf * ka + row) * 128 + c * 16) =
+            make_uint4(0u, 0u, 0u, 0u);
+      }
+    }
+    if (ok) ok = ptx::mbar_wait_bounded(bar_s, 0, abort, WAIT_LIMIT_NS);
+    float m = -INFINITY;
+    if (ok) {
+      ptx::tc_fence_after();
+      // pass 1: row maximum over this half's valid keys
+      for (int c0 = c_beg; c0 < c_end; c0 += 16) {
+        float v[16];
+        ptx::tmem_ld(tmem_base + lane_addr + c0, v);
+        ptx::tmem_ld_wait();
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+          if (c0 + j < n_valid) m = fmaxf(m, v[j]);
+      }
+    }
+    xmax[kh * QT + r] = m;
+    // the two warps of a lane quarter exchange their maxima (named barrier over the 8 softmax warps)
+    asm volatile("bar.sync 1, %0;" ::"n"(SM_WARPS * 32) : "memory");
+    m = fmaxf(xmax[r], xmax[QT + r]);
+    const float msc = m * sc;
+    float l = 0.f;
+    if (ok) {
+      // pass 2: p = 2^(s sc - m sc) on valid keys, 0 elsewhere; P row r into 64-key blocks (swizzled)
+      for (int c0 = c_beg; c0 < c_end; c0 += 16) {
+        float v[16];
+        ptx::tmem_ld(tmem_base + lane_addr + c0, v);
+        ptx::tmem_ld_wait();
+        uint32_t w[8];
+#pragma unroll
+        for (int j = 0; j < 16; j += 2) {
+          const float p0 = c0 + j < n_valid ? exp2f(fmaf(v[j], sc, -msc)) : 0.f;
+          const float p1 = c0 + j + 1 < n_valid ? exp2f(fmaf(v[j + 1], sc, -msc)) : 0.f;
+          l += p0 + p1;
+          w[j / 2] = bf16x2_bits(p0, p1);
+        }
+        // 16 keys = two 16-byte chunks of row r in block c0 / 64
+        uint8_t* blk = smem + Q_BYTES + (size_t)(c0 / 64) * (QT * 128) + (size_t)r * 128;
+        const int ch = (c0 % 64) / 8;
+        *reinterpret_cast<uint4*>(blk + (((ch) ^ (r & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+        *reinterpret_cast<uint4*>(blk + (((ch + 1) ^ (r & 7)) << 4)) = make_uint4(w[4], w[5], w[6], w[7]);
+      }
+    }
+    xsum[kh * QT + r] = l;
+    ptx::fence_proxy_async_smem();   // P and the zeroed value rows, before the MMA reads them
+    ptx::tc_fence_before();
+    __syncwarp();
+    if (lane == 0) ptx::mbar_arrive(bar_p);
+    asm volatile("bar.sync 1, %0;" ::"n"(SM_WARPS * 32) : "memory");
+    l = xsum[r] + xsum[QT + r];
+    if (ok) ok = ptx::mbar_wait_bounded(bar_o, 0, abort, WAIT_LIMIT_NS);
+    if (ok) {
+      ptx::tc_fence_after();
+      // O row r, dims [64 kh, 64 kh + 64): scale by 1 / l and store if the query exists
+      const float inv = 1.f / l;
+      const int qrow = qt * QT + r;
+      bf16* orow = out + (row0 + qrow) * D + h * DH + kh * 64;
+      for (int c0 = 0; c0 < 64; c0 += 16) {
+        float v[16];
+        ptx::tmem_ld(tmem_base + lane_addr + O_COL + kh * 64 + c0, v);
+        ptx::tmem_ld_wait();
+        if (qrow < S) {
+          uint4 w0 = make_uint4(bf16x2_bits(v[0] * inv, v[1] * inv), bf16x2_bits(v[2] * inv, v[3] * inv),
+                                bf16x2_bits(v[4] * inv, v[5] * inv), bf16x2_bits(v[6] * inv, v[7] * inv));
+          uint4 w1 = make_uint4(bf16x2_bits(v[8] * inv, v[9] * inv), bf16x2_bits(v[10] * inv, v[11] * inv),
+                                bf16x2_bits(v[12] * inv, v[13] * inv), bf16x2_bits(v[14] * inv, v[15] * inv));
+          *reinterpret_cast<uint4*>(orow + c0) = w0;
+          *reinterpret_cast<uint4*>(orow + c0 + 8) = w1;
+        }
+      }
+    }
+    if (!ok && !*abort) record_timeout(err, abort);
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+}  // namespace
+
+size_t attention_tc_smem(int S) {
+  const int ka = ((S + KB_ROWS - 1) / KB_ROWS) * KB_ROWS;
+  return smem_bytes(ka);
+}
+
+cudaError_t attention_tc_prepare() {
+  return cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              (int)smem_bytes(MAX_KA));
+}
+
+cudaError_t attention_tc(const bf16* qkv, bf16* out, int M, const int* lengths, int len_mod, int nseq, int S,
+                         DevError* err, cudaStream_t st, const int* tok0) {
+  if (nseq <= 0 || S <= 0 || M <= 0) return cudaSuccess;
+  if (S > MAX_FRAMES + 1) return cudaErrorInvalidValue;
+  CUtensorMap tq, tkv;
+  if (make_tmap_bf16(&tq, qkv, M, 3 * D, 3 * D, QT) || make_tmap_bf16(&tkv, qkv, M, 3 * D, 3 * D, KB_ROWS))
+    return cudaErrorInvalidValue;
+  const int ka = ((S + KB_ROWS - 1) / KB_ROWS) * KB_ROWS;
+  dim3 grid(H, nseq, (S + QT - 1) / QT);
+  return launch_kernel(attn_tc_kernel, grid, dim3(NUM_THREADS), smem_bytes(ka), st, tq, tkv, out, lengths, len_mod, S,
+                       ka, tok0, err);
+}
+
+}  // namespace kd

@@ -123,7 +123,8 @@ struct kimodo_ctx {
   long long last_launches = 0;
   Tokens tk;                    // token layout of the call being enqueued
   bool pair_gemm = true;   // 256-row CTA-pair GEMM tiles for the large projections (KIMODO_PAIR_GEMM=0 disables)
-  bool stream_k = true;    // stream-K shares for them (KIMODO_STREAM_K=0: one whole tile per pair and round)
+  bool stream_k = false;   // stream-K shares for them instead (KIMODO_STREAM_K=1; measured slower on the layer shapes)
+  bool attn_tc = false;    // tcgen05 attention (KIMODO_ATTN_TC=1) instead of the mma.sync kernel
   float* sk_partial = nullptr;   // stream-K partial accumulators
   int* sk_flags = nullptr;       // stream-K contributor counters (zero between launches)
   bool bf16() const { return precision == KIMODO_BF16; }
@@ -391,10 +392,17 @@ int run_net(kimodo_ctx* c, int net, int nseq, int T, int len_mod, const void* A_
     const double aflops = packed ? 4.0 * (double)M * S * DH * H : 4.0 * (double)nseq * S * S * DH * H;
     const double abytes = (double)M * 3 * D * eb + (double)M * D * eb;
     if (c->bf16()) {
-      KD_TRY(launch(c, CLS_ATTN, aflops, abytes, st, "attention_bf16", [&] {
-        return attention_bf16(static_cast<const bf16*>(w.qkv), static_cast<bf16*>(w.attn), w.lengths, len_mod,
-                              nseq, S, st, tok0);
-      }));
+      if (c->attn_tc) {
+        KD_TRY(launch(c, CLS_ATTN, aflops, abytes, st, "attention_tc", [&] {
+          return attention_tc(static_cast<const bf16*>(w.qkv), static_cast<bf16*>(w.attn), M, w.lengths, len_mod,
+                              nseq, S, c->derr, st, tok0);
+        }));
+      } else {
+        KD_TRY(launch(c, CLS_ATTN, aflops, abytes, st, "attention_bf16", [&] {
+          return attention_bf16(static_cast<const bf16*>(w.qkv), static_cast<bf16*>(w.attn), w.lengths, len_mod,
+                                nseq, S, st, tok0);
+        }));
+      }
     } else {
       KD_TRY(launch(c, CLS_ATTN, aflops, abytes, st, "attention_f32", [&] {
         return attention_f32(static_cast<const float*>(w.qkv), static_cast<float*>(w.attn), w.lengths, len_mod,
@@ -582,7 +590,7 @@ int kimodo_load_weights(kimodo_ctx** out_ctx, const float* host_blob, size_t n_f
     return set_error(KIMODO_EUNSUPPORTED, "cuTensorMapEncodeTiled is unavailable in this driver");
 
   if (gemm_tc_prepare() != cudaSuccess || gemm_tc2_prepare() != cudaSuccess || gemm_sk_prepare() != cudaSuccess ||
-      attention_prepare() != cudaSuccess) {
+      attention_prepare() != cudaSuccess || attention_tc_prepare() != cudaSuccess) {
     cudaGetLastError();
     return set_error(KIMODO_EUNSUPPORTED, "kernel attributes could not be set on device %d", device);
   }
@@ -591,6 +599,7 @@ int kimodo_load_weights(kimodo_ctx** out_ctx, const float* host_blob, size_t n_f
   c->precision = precision;
   if (const char* ev = getenv("KIMODO_PAIR_GEMM")) c->pair_gemm = ev[0] != '0';
   if (const char* ev = getenv("KIMODO_STREAM_K")) c->stream_k = ev[0] != '0';
+  if (const char* ev = getenv("KIMODO_ATTN_TC")) c->attn_tc = ev[0] != '0';
   c->num_sms = prop.multiProcessorCount;
   auto fail = [&](int code) {
     kimodo_free(c);
@@ -972,6 +981,7 @@ int prepared_device() {
     KD_CUDA(gemm_tc2_prepare());
     KD_CUDA(gemm_sk_prepare());
     KD_CUDA(attention_prepare());
+    KD_CUDA(attention_tc_prepare());
     done[dev] = true;
   }
   return KIMODO_OK;
@@ -1101,6 +1111,17 @@ int kimodo_attention_bf16(const void* qkv, void* out, const int* lengths, int ns
   KD_TRY(prepared_device());
   KD_CUDA(attention_bf16(static_cast<const bf16*>(qkv), static_cast<bf16*>(out), lengths, nseq, nseq, S,
                          static_cast<cudaStream_t>(stream)));
+  return KIMODO_OK;
+}
+
+int kimodo_attention_bf16_tc(const void* qkv, void* out, const int* lengths, int nseq, int S, void* stream) {
+  g_last_error.clear();
+  if (!qkv || !out || !lengths) return set_error(KIMODO_EINVAL, "NULL tensor argument");
+  if (nseq < 1 || S < 1 || S > MAX_FRAMES + 1) return set_error(KIMODO_EINVAL, "need nseq >= 1, 1 <= S <= 301");
+  if (reinterpret_cast<uintptr_t>(qkv) & 15) return set_error(KIMODO_EINVAL, "qkv must be 16-byte aligned");
+  KD_TRY(prepared_device());
+  KD_CUDA(attention_tc(static_cast<const bf16*>(qkv), static_cast<bf16*>(out), nseq * S, lengths, nseq, nseq, S,
+                       kernel_error_word(), static_cast<cudaStream_t>(stream)));
   return KIMODO_OK;
 }
 

@@ -41,6 +41,7 @@ enum DevErrWhere : int {
   WHERE_GEMM_MMA = 2,
   WHERE_GEMM_EPILOGUE = 3,
   WHERE_GEMM_DRAIN = 4,
+  WHERE_ATTENTION = 5,
 };
 
 }  // namespace kd

@@ -67,6 +67,14 @@ cudaError_t attention_bf16(const bf16* qkv, bf16* out, const int* lengths, int l
 cudaError_t attention_f32(const float* qkv, float* out, const int* lengths, int len_mod, int nseq, int S,
                           cudaStream_t st, const int* tok0 = nullptr);
 
+// The same attention on the tcgen05 tensor cores (bf16): one CTA per (head, sequence,
+// 128-query tile), exact softmax over all keys of the sequence at once.  qkv has M
+// rows (16-byte aligned, row stride 3*D); S <= MAX_FRAMES + 1.
+cudaError_t attention_tc(const bf16* qkv, bf16* out, int M, const int* lengths, int len_mod, int nseq, int S,
+                         DevError* err, cudaStream_t st, const int* tok0 = nullptr);
+cudaError_t attention_tc_prepare();
+size_t attention_tc_smem(int S);
+
 // Token layout of a batch: tok0[s] = sum over s' < s of (1 + lengths[s' % len_mod]) for
 // s <= nseq, and row_seq[r] = s for the rows r of sequence s (one CTA).
 cudaError_t build_token_map(const int* lengths, int len_mod, int nseq, int* tok0, int* row_seq, cudaStream_t st);
