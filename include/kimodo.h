@@ -175,17 +175,23 @@ KIMODO_API int kimodo_ddim_sample(kimodo_ctx* ctx, const float* text_emb, const 
  *   kimodo_ddim_step_ex.  Required when eta > 0, ignored when eta = 0.  Values at
  *   padded frames are never read into valid outputs.  A graph captured for a device
  *   step_noise pointer reads that pointer on every replay.
- * A NULL options pointer means { KIMODO_SCHEDULE_LINEAR, 0, NULL }.
+ * text_batch: 0 (text_emb has `batch` rows), or a divisor of batch for variations of
+ *   fewer prompts: text_emb then has text_batch rows and sequence b uses row
+ *   b / (batch / text_batch), each take with its own noise rows (the pages generate
+ *   several takes of one prompt in a batch).  null_emb keeps its own broadcast rule.
+ * A NULL options pointer means { KIMODO_SCHEDULE_LINEAR, 0, NULL, 0 }.
  */
 enum { KIMODO_SCHEDULE_LINEAR = 0, KIMODO_SCHEDULE_COSINE = 1 };
 typedef struct kimodo_sampler {
   int schedule;
   float eta;
   const float* step_noise;
+  int text_batch;
 } kimodo_sampler;
 
 /* kimodo_ddim_sample with sampler options (KIMODO_EINVAL on an unknown schedule,
- * eta outside [0, 1] or not finite, or eta > 0 without step_noise). */
+ * eta outside [0, 1] or not finite, eta > 0 without step_noise, or a text_batch that
+ * does not divide batch). */
 KIMODO_API int kimodo_ddim_sample_ex(kimodo_ctx* ctx, const float* text_emb, const float* null_emb,
                        int null_batch, const float* noise, const int* lengths, int batch,
                        int frames, int steps, float cfg_scale, const kimodo_sampler* options,

@@ -145,3 +145,37 @@ def test_sampler_option_errors(gpu_bf16, schedule, eta, noise, steps):
     rc = gpu_bf16._lib.kimodo_ddim_sample_ex(gpu_bf16._ctx, emb.ctypes.data, null.ctypes.data, 1, x.ctypes.data,
                                              L.ctypes.data, B, T, steps, 2.0, ctypes.byref(opts), out.ctypes.data, st)
     assert rc == -1, rc
+
+
+def test_variations_share_prompt_rows(gpu_bf16):
+    """Several takes of one prompt (text_batch < batch): sequence b uses prompt row
+    b // takes; the result equals the call with the rows repeated, and takes differ
+    only by their noise."""
+    B, T, L = 6, 20, np.full(6, 20, np.int32)
+    prompts = synth.text_embeddings(2, seed=471)
+    noise = synth.noise(B, T, seed=472)
+    null = np.zeros(4096, np.float32)
+    var = gpu_bf16.ddim_sample(prompts, null, noise, L, 4, 2.0)
+    rep = gpu_bf16.ddim_sample(np.repeat(prompts, 3, axis=0), null, noise, L, 4, 2.0)
+    np.testing.assert_array_equal(var, rep)
+    assert np.abs(var[0] - var[1]).max() > 1e-3
+    same = gpu_bf16.ddim_sample(prompts, null, np.repeat(noise[:1], B, axis=0), L, 4, 2.0)
+    np.testing.assert_array_equal(same[0], same[2])          # same prompt, same noise
+    assert np.abs(same[0] - same[3]).max() > 1e-3             # other prompt
+    vs = gpu_bf16.ddim_step(noise, prompts, null, L, 999, 749, 2.0)
+    rs = gpu_bf16.ddim_step(noise, np.repeat(prompts, 3, axis=0), null, L, 999, 749, 2.0)
+    np.testing.assert_array_equal(vs, rs)
+
+
+def test_text_batch_must_divide_batch(gpu_bf16):
+    B, T = 6, 8
+    x = synth.noise(B, T, seed=481)
+    emb = synth.text_embeddings(4, seed=482)
+    null = np.zeros(4096, np.float32)
+    L = np.full(B, T, np.int32)
+    opts = kb.SamplerOptions(0, 0.0, None, 4)
+    out = np.empty_like(x)
+    st = torch.cuda.current_stream().cuda_stream
+    rc = gpu_bf16._lib.kimodo_ddim_sample_ex(gpu_bf16._ctx, emb.ctypes.data, null.ctypes.data, 1, x.ctypes.data,
+                                             L.ctypes.data, B, T, 3, 2.0, ctypes.byref(opts), out.ctypes.data, st)
+    assert rc == -1, rc

@@ -57,7 +57,8 @@ SCHEDULES = {"linear": 0, "cosine": 1}
 
 class SamplerOptions(ctypes.Structure):
     """struct kimodo_sampler of include/kimodo.h."""
-    _fields_ = [("schedule", ctypes.c_int), ("eta", ctypes.c_float), ("step_noise", ctypes.c_void_p)]
+    _fields_ = [("schedule", ctypes.c_int), ("eta", ctypes.c_float), ("step_noise", ctypes.c_void_p),
+                ("text_batch", ctypes.c_int)]
 
 
 class KimodoError(RuntimeError):
@@ -253,12 +254,13 @@ class Kimodo:
         return out
 
     @staticmethod
-    def _options(schedule, eta, step_noise):
-        """kimodo_sampler for the _ex calls, or None for the defaults (linear, eta 0)."""
-        if schedule == "linear" and float(eta) == 0.0:
+    def _options(schedule, eta, step_noise, text_batch=0):
+        """kimodo_sampler for the _ex calls, or None for the defaults (linear, eta 0, one
+        text row per sequence)."""
+        if schedule == "linear" and float(eta) == 0.0 and not text_batch:
             return None, None
         z = None if step_noise is None else _f32(step_noise)
-        return SamplerOptions(SCHEDULES[schedule], float(eta), _ptr(z)), z
+        return SamplerOptions(SCHEDULES[schedule], float(eta), _ptr(z), int(text_batch)), z
 
     def ddim_step(self, x_t, text_emb, null_emb, lengths, t, t_prev, cfg_scale, out=None, stream=None,
                   schedule="linear", eta=0.0, step_noise=None):
@@ -266,7 +268,7 @@ class Kimodo:
         B, T = x_t.shape[0], x_t.shape[1]
         nb = 1 if null_emb.ndim == 1 else null_emb.shape[0]
         out = _like(x_t, (B, T, MOTION_DIM)) if out is None else out
-        opts, z = self._options(schedule, eta, step_noise)
+        opts, z = self._options(schedule, eta, step_noise, text_emb.shape[0] if text_emb.shape[0] != B else 0)
         if opts is None:
             _check(self._lib.kimodo_ddim_step(self._ctx, _ptr(x_t), _ptr(text_emb), _ptr(null_emb), nb,
                                               _ptr(lengths), B, T, int(t), int(t_prev), float(cfg_scale), _ptr(out),
@@ -280,12 +282,13 @@ class Kimodo:
     def ddim_sample(self, text_emb, null_emb, noise, lengths, steps, cfg_scale, out=None, stream=None,
                     schedule="linear", eta=0.0, step_noise=None):
         """Full sampler; schedule "linear" or "cosine", eta in [0, 1] with step_noise
-        [steps, B, T, 279] standard-normal draws when eta > 0."""
+        [steps, B, T, 279] standard-normal draws when eta > 0.  text_emb may have fewer
+        rows than the batch (a divisor of B): variations, row b // (B // rows) per sequence."""
         text_emb, null_emb, noise, lengths = _f32(text_emb), _f32(null_emb), _f32(noise), _i32(lengths)
         B, T = noise.shape[0], noise.shape[1]
         nb = 1 if null_emb.ndim == 1 else null_emb.shape[0]
         out = _like(noise, (B, T, MOTION_DIM)) if out is None else out
-        opts, z = self._options(schedule, eta, step_noise)
+        opts, z = self._options(schedule, eta, step_noise, text_emb.shape[0] if text_emb.shape[0] != B else 0)
         if opts is None:
             _check(self._lib.kimodo_ddim_sample(self._ctx, _ptr(text_emb), _ptr(null_emb), nb, _ptr(noise),
                                                 _ptr(lengths), B, T, int(steps), float(cfg_scale), _ptr(out),

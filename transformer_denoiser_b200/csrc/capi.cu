@@ -107,7 +107,7 @@ struct kimodo_ctx {
   double alphabar[2][N_TRAIN];   // [KIMODO_SCHEDULE_LINEAR / _COSINE][t]
   Workspace ws;
   cudaStream_t cap_stream = nullptr;
-  // sampler graphs keyed by (batch, frames, steps, null broadcast, cfg bits, schedule, eta bits, step noise,
+  // sampler graphs keyed by (batch, frames, steps, null broadcast | takes << 1, cfg bits, schedule, eta bits, step noise,
   // token rows: the packed layout's row count, or the padded one)
   std::map<std::tuple<int, int, int, int, uint32_t, int, uint32_t, const float*, int>,
            std::pair<cudaGraphExec_t, long long>>
@@ -450,6 +450,7 @@ struct Sampler {
   int schedule = KIMODO_SCHEDULE_LINEAR;
   float eta = 0.f;
   const float* z = nullptr;   // device draws for the call (eta > 0), step-major
+  int takes = 1;              // sequences per text-embedding row (variations of one prompt)
 };
 
 // One two-stage step for B prompts (cond rows 0..B-1, uncond rows B..2B-1).
@@ -727,9 +728,15 @@ int kimodo_denoiser_forward(kimodo_ctx* c, int net, const float* x, const float*
 }
 
 // Validates the sampler options; n_z = floats of step noise the call reads when eta > 0.
-static int check_sampler(kimodo_ctx* c, const kimodo_sampler* o, size_t n_z, Sampler* out, cudaStream_t st) {
+static int check_sampler(kimodo_ctx* c, const kimodo_sampler* o, int batch, size_t n_z, Sampler* out,
+                         cudaStream_t st) {
   *out = Sampler();
   if (!o) return KIMODO_OK;
+  if (o->text_batch != 0) {
+    if (o->text_batch < 1 || o->text_batch > batch || batch % o->text_batch)
+      return set_error(KIMODO_EINVAL, "text_batch must divide batch (got %d for batch %d)", o->text_batch, batch);
+    out->takes = batch / o->text_batch;
+  }
   if (o->schedule != KIMODO_SCHEDULE_LINEAR && o->schedule != KIMODO_SCHEDULE_COSINE)
     return set_error(KIMODO_EINVAL, "unknown schedule %d", o->schedule);
   if (!isfinite(o->eta) || o->eta < 0.f || o->eta > 1.f)
@@ -778,7 +785,7 @@ int kimodo_ddim_step_ex(kimodo_ctx* c, const float* x_t, const float* text_emb, 
     return set_error(KIMODO_EINVAL, "null_batch must be 1 or batch (got %d)", null_batch);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   Sampler smp;
-  KD_TRY(check_sampler(c, options, (size_t)batch * frames * MOTION_F, &smp, st));
+  KD_TRY(check_sampler(c, options, batch, (size_t)batch * frames * MOTION_F, &smp, st));
   KD_TRY(ensure_workspace(c, 2 * batch, frames, 1));
   const long long l0 = c->launches;
   Workspace& w = c->ws;
@@ -786,10 +793,10 @@ int kimodo_ddim_step_ex(kimodo_ctx* c, const float* x_t, const float* text_emb, 
   c->tk = plan_tokens(lengths, batch, 2 * batch, frames);
   KD_TRY(enqueue_token_map(c, batch, 2 * batch, st));
   KD_CUDA(cudaMemcpyAsync(w.x, x_t, (size_t)batch * frames * MOTION_F * 4, cudaMemcpyDefault, st));
-  KD_CUDA(cudaMemcpyAsync(w.st_text, text_emb, (size_t)batch * DTXT * 4, cudaMemcpyDefault, st));
+  KD_CUDA(cudaMemcpyAsync(w.st_text, text_emb, (size_t)(batch / smp.takes) * DTXT * 4, cudaMemcpyDefault, st));
   KD_CUDA(cudaMemcpyAsync(w.st_null, null_emb, (size_t)null_batch * DTXT * 4, cudaMemcpyDefault, st));
   KD_TRY(launch(c, CLS_SETUP, 0, (double)2 * batch * DTXT * 6, st, "pack_embeddings", [&] {
-    return pack_embeddings(w.st_text, batch, w.st_null, null_batch, batch, w.emb, c->bf16(), st);
+    return pack_embeddings(w.st_text, batch, w.st_null, null_batch, batch, w.emb, c->bf16(), st, smp.takes);
   }));
   KD_TRY(timestep_rows(c, t, 0, 1, st));
   KD_TRY(condition_setup(c, 0, 2 * batch, 1, st));
@@ -806,7 +813,7 @@ static int enqueue_sample(kimodo_ctx* c, int batch, int frames, int steps, float
   Workspace& w = c->ws;
   KD_TRY(enqueue_token_map(c, batch, 2 * batch, st));
   KD_TRY(launch(c, CLS_SETUP, 0, (double)2 * batch * DTXT * 6, st, "pack_embeddings", [&] {
-    return pack_embeddings(w.st_text, batch, w.st_null, null_batch, batch, w.emb, c->bf16(), st);
+    return pack_embeddings(w.st_text, batch, w.st_null, null_batch, batch, w.emb, c->bf16(), st, smp.takes);
   }));
   KD_TRY(timestep_rows(c, -1, steps, steps, st));
   KD_TRY(condition_setup(c, 0, 2 * batch, steps, st));
@@ -841,13 +848,13 @@ int kimodo_ddim_sample_ex(kimodo_ctx* c, const float* text_emb, const float* nul
     return set_error(KIMODO_EINVAL, "null_batch must be 1 or batch (got %d)", null_batch);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   Sampler smp;
-  KD_TRY(check_sampler(c, options, (size_t)steps * batch * frames * MOTION_F, &smp, st));
+  KD_TRY(check_sampler(c, options, batch, (size_t)steps * batch * frames * MOTION_F, &smp, st));
   KD_TRY(ensure_workspace(c, 2 * batch, frames, steps));
   Workspace& w = c->ws;
   KD_TRY(stage_lengths(c, lengths, batch, frames, st));
   c->tk = plan_tokens(lengths, batch, 2 * batch, frames);
   KD_CUDA(cudaMemcpyAsync(w.x, noise, (size_t)batch * frames * MOTION_F * 4, cudaMemcpyDefault, st));
-  KD_CUDA(cudaMemcpyAsync(w.st_text, text_emb, (size_t)batch * DTXT * 4, cudaMemcpyDefault, st));
+  KD_CUDA(cudaMemcpyAsync(w.st_text, text_emb, (size_t)(batch / smp.takes) * DTXT * 4, cudaMemcpyDefault, st));
   KD_CUDA(cudaMemcpyAsync(w.st_null, null_emb, (size_t)null_batch * DTXT * 4, cudaMemcpyDefault, st));
   const long long l0 = c->launches;
   if (c->profiling) {
@@ -878,8 +885,8 @@ int kimodo_ddim_sample_ex(kimodo_ctx* c, const float* text_emb, const float* nul
     uint32_t cfg_bits, eta_bits;
     memcpy(&cfg_bits, &cfg_scale, 4);
     memcpy(&eta_bits, &smp.eta, 4);
-    const auto key = std::make_tuple(batch, frames, steps, null_batch == 1 ? 1 : 0, cfg_bits, smp.schedule, eta_bits,
-                                     smp.z, c->tk.packed ? c->tk.M : -1);
+    const auto key = std::make_tuple(batch, frames, steps, (null_batch == 1 ? 1 : 0) | (smp.takes << 1), cfg_bits,
+                                     smp.schedule, eta_bits, smp.z, c->tk.packed ? c->tk.M : -1);
     auto it = c->graphs.find(key);
     if (it == c->graphs.end()) {
       KD_CUDA(cudaStreamBeginCapture(c->cap_stream, cudaStreamCaptureModeThreadLocal));

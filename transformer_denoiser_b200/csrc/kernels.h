@@ -108,10 +108,11 @@ cudaError_t cfg_ddim(const float* root_hat, const float* body_hat, float* x, con
                      float w, float c0, float c1, const float* z, float c2, void* A_next, bool a_bf16, int lda, int S,
                      cudaStream_t st, const int* tok0 = nullptr);
 
-// Condition inputs: rows [0, B) = text_emb, rows [B, B + nnull_rows) = null_emb
-// (row (r - B) % null_batch).  out (bf16 or fp32) [rows, DTXT].
+// Condition inputs: rows [0, B) = text_emb row r / takes (several takes of one prompt
+// share its row), rows [B, B + null_rows) = null_emb row (r - B) % null_batch.
+// out (bf16 or fp32) [rows, DTXT].
 cudaError_t pack_embeddings(const float* text_emb, int B, const float* null_emb, int null_batch, int null_rows,
-                            void* out, bool out_bf16, cudaStream_t st);
+                            void* out, bool out_bf16, cudaStream_t st, int takes = 1);
 
 // out[k, :] = pe[t_k, :] for k < n (sinusoid rows of the timesteps): t_k = t_single
 // when steps == 0, else the k-th trailing timestep of a `steps`-step sampler,

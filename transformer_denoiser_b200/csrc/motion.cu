@@ -153,14 +153,15 @@ __global__ void cfg_ddim_kernel(const float* __restrict__ root_hat, const float*
 }
 
 template <typename T>
-__global__ void pack_embeddings_kernel(const float* __restrict__ text, int B, const float* __restrict__ null_emb,
-                                       int null_batch, int null_rows, T* __restrict__ out) {
+__global__ void pack_embeddings_kernel(const float* __restrict__ text, int B, int takes,
+                                       const float* __restrict__ null_emb, int null_batch, int null_rows,
+                                       T* __restrict__ out) {
   ptx::pdl_wait();
   ptx::pdl_trigger();
   const long total = (long)(B + null_rows) * DTXT;
   for (long idx = blockIdx.x * (long)blockDim.x + threadIdx.x; idx < total; idx += (long)gridDim.x * blockDim.x) {
     const int r = idx / DTXT, c = idx % DTXT;
-    const float v = r < B ? text[(long)r * DTXT + c] : null_emb[(long)((r - B) % null_batch) * DTXT + c];
+    const float v = r < B ? text[(long)(r / takes) * DTXT + c] : null_emb[(long)((r - B) % null_batch) * DTXT + c];
     out[idx] = from_f<T>(v);
   }
 }
@@ -237,15 +238,15 @@ cudaError_t cfg_ddim(const float* root_hat, const float* body_hat, float* x, con
 }
 
 cudaError_t pack_embeddings(const float* text_emb, int B, const float* null_emb, int null_batch, int null_rows,
-                            void* out, bool out_bf16, cudaStream_t st) {
+                            void* out, bool out_bf16, cudaStream_t st, int takes) {
   const long n = (long)(B + null_rows) * DTXT;
   if (n <= 0) return cudaSuccess;
   if (out_bf16)
-    LAUNCHK(pack_embeddings_kernel<bf16>, blocks_for(n), 256, st, text_emb, B, null_emb, null_batch, null_rows,
+    LAUNCHK(pack_embeddings_kernel<bf16>, blocks_for(n), 256, st, text_emb, B, takes, null_emb, null_batch, null_rows,
                                                                 static_cast<bf16*>(out));
   else
-    LAUNCHK(pack_embeddings_kernel<float>, blocks_for(n), 256, st, text_emb, B, null_emb, null_batch, null_rows,
-                                                                 static_cast<float*>(out));
+    LAUNCHK(pack_embeddings_kernel<float>, blocks_for(n), 256, st, text_emb, B, takes, null_emb, null_batch,
+                                                                 null_rows, static_cast<float*>(out));
   return cudaGetLastError();
 }
 
