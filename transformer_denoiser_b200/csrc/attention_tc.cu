@@ -1,10 +1,12 @@
 // Masked multi-head self-attention on the tcgen05 tensor cores ("Kimodo WebGPU",
 // "WGSL compute shaders" table: multi-head self-attention with optional key masking).
 //
-// One CTA per (head, sequence, 128-query tile).  Every key of a sequence fits in
-// one pass (at most 301 tokens), so the softmax is exact, not online:
-//   1. TMA stages the query tile (128 x 128), and the keys and values of the
-//      sequence's rows rounded up to 64 (128-byte swizzle, no multicast).
+// One CTA per (head, sequence, 128-query tile), two CTAs per SM up to 256 keys.
+// Every key of a sequence fits in one pass (at most 301 tokens), so the softmax is
+// exact, not online:
+//   1. TMA stages the query tile (128 x 128), the keys and the upper half of the
+//      value dimensions of the sequence's rows rounded up to 32 (128-byte swizzle, no
+//      multicast); the lower value half goes into the query buffer once S is formed.
 //   2. One thread issues S = Q K^T (M = 128, N = valid keys rounded up to 16,
 //      K = 128) into TMEM.
 //   3. Eight softmax warps (two per TMEM lane quarter, one query row per thread,
@@ -14,9 +16,10 @@
 //      and write P in bf16 into the key buffer (dead once S is formed) in the
 //      K-major 128-byte-swizzle layout.  They zero the value rows past the valid
 //      keys inside the MMA's K range, so 0 * garbage cannot occur either.
-//   4. The same thread issues O = P V (M = 128, N = 128, K = keys) with V read in
-//      place as an MN-major operand; the softmax warps scale O by 1 / sum and store
-//      the valid query rows in bf16.
+//   4. The same thread issues O = P V as two N = 64 halves (K = keys) with each value
+//      half read in place as an MN-major operand, into the TMEM columns S occupied
+//      (up to 256 keys: a 256-column allocation); the softmax warps scale O by 1 / sum
+//      and store the valid query rows in bf16.
 // Rows of the key and value tiles past the sequence belong to other tokens or lie
 // outside the matrix (zero fill) and are masked as above.  Every wait is bounded.
 #include <cuda.h>
@@ -32,21 +35,24 @@ namespace kd {
 namespace {
 
 constexpr int QT = 128;                    // query rows per CTA
-constexpr int KB_ROWS = 64;                // key rows per TMA box
+constexpr int KB_ROWS = 32;                // key rows per TMA box
 constexpr int SM_WARPS = 8;                // softmax / epilogue warps
 constexpr int NUM_THREADS = 64 + 32 * SM_WARPS;
 constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;
 constexpr int KIMODO_ETIMEOUT_CODE = -5;
-constexpr uint32_t O_COL = 320;            // TMEM column of the O accumulator (S uses columns 0..303)
-constexpr uint32_t TMEM_COLS = 512;
-constexpr int MAX_KA = ((MAX_FRAMES + 1 + KB_ROWS - 1) / KB_ROWS) * KB_ROWS;   // 320 key rows
+constexpr int MAX_KA = ((MAX_FRAMES + 1 + KB_ROWS - 1) / KB_ROWS) * KB_ROWS;   // 304 key rows
 constexpr uint32_t Q_BYTES = QT * DH * 2;  // two 64-column halves of 16 KB
 
-// Shared memory: Q [2 halves][128 rows][128 B], K [2 halves][KA rows][128 B] (later P
-// [KA / 64 blocks][128 rows][128 B]), V [2 halves][KA rows][128 B], then barriers and
-// the row-statistics exchange.
-constexpr size_t smem_bytes(int ka) {
-  return 1024 + Q_BYTES + 2 * (size_t)ka * 256 + 8 * 8 + 2 * 2 * QT * 4 + 16;
+// Shared memory, with ka = key rows rounded up to 32 and kp = ka rounded up to 64:
+// Q [2 halves][128 rows][128 B] (later the lower value half V0 [ka rows][128 B] when
+// it fits), K [2 halves][ka rows][128 B] then P [kp / 64 blocks][128 rows][128 B] in a
+// region of kp * 256 B, the upper value half V1 [ka rows][128 B], V0 on its own when
+// it does not fit in the Q buffer, then barriers and the row-statistics exchange.
+__host__ __device__ constexpr bool v0_in_q(int ka) { return (uint32_t)ka * 128 <= Q_BYTES; }
+__host__ __device__ constexpr uint32_t kp_of(int ka) { return (uint32_t)((ka + 63) / 64) * 64; }
+__host__ __device__ constexpr size_t smem_bytes(int ka) {
+  return 1024 + Q_BYTES + (size_t)kp_of(ka) * 256 + (size_t)ka * 128 + (v0_in_q(ka) ? 0 : (size_t)ka * 128) +
+         8 * 8 + 2 * 2 * QT * 4 + 16;
 }
 
 __device__ __forceinline__ void record_timeout(DevError* err, volatile int* abort) {
@@ -69,18 +75,25 @@ __device__ __forceinline__ uint64_t smem_desc_sw128_mn(uint32_t saddr, uint32_t 
   return d;
 }
 
-__global__ void __launch_bounds__(NUM_THREADS, 1)
+__global__ void __launch_bounds__(NUM_THREADS, 2)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmKV,
                bf16* __restrict__ out, const int* __restrict__ lengths, int len_mod, int S_pad, int ka,
-               const int* __restrict__ tok0, DevError* err) {
+               uint32_t tmem_cols, uint32_t o_col, const int* __restrict__ tok0, DevError* err) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t kp = kp_of(ka);
+  const bool v0q = v0_in_q(ka);
   const uint32_t sQ = ptx::smem_u32(smem);
   const uint32_t sK = sQ + Q_BYTES;                       // also P
-  const uint32_t sV = sK + (uint32_t)ka * 256;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Q_BYTES + (size_t)ka * 512);
+  const uint32_t sV1 = sK + kp * 256;
+  const uint32_t sV0 = v0q ? sQ : sV1 + (uint32_t)ka * 128;
+  uint8_t* gV1 = smem + Q_BYTES + (size_t)kp * 256;       // generic addresses of the value halves
+  uint8_t* gV0 = v0q ? smem : gV1 + (size_t)ka * 128;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Q_BYTES + (size_t)kp * 256 + (size_t)ka * 128 +
+                                               (v0q ? 0 : (size_t)ka * 128));
   const uint32_t bar0 = ptx::smem_u32(bars);
-  const uint32_t bar_qk = bar0, bar_v = bar0 + 8, bar_s = bar0 + 16, bar_p = bar0 + 24, bar_o = bar0 + 32;
+  const uint32_t bar_qk = bar0, bar_v1 = bar0 + 8, bar_s = bar0 + 16, bar_p = bar0 + 24, bar_o = bar0 + 32,
+                 bar_v0 = bar0 + 40;
   float* xmax = reinterpret_cast<float*>(bars + 8);      // [2][QT] partial row maxima, then sums
   float* xsum = xmax + 2 * QT;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(xsum + 2 * QT);
@@ -96,11 +109,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   int n_valid = 1 + lengths[seq % len_mod];
   n_valid = n_valid < 1 ? 1 : (n_valid > S ? S : n_valid);
   const int n_cols = (n_valid + 15) & ~15;                 // MMA N for S = Q K^T, K range of O = P V
-  const int n_boxes = (n_valid + KB_ROWS - 1) / KB_ROWS;   // 64-row key / value boxes
+  const int n_boxes = (n_valid + KB_ROWS - 1) / KB_ROWS;   // 32-row key / value boxes
 
   if (threadIdx.x == 0) {
     ptx::mbar_init(bar_qk, 1);
-    ptx::mbar_init(bar_v, 1);
+    ptx::mbar_init(bar_v1, 1);
+    ptx::mbar_init(bar_v0, 1);
     ptx::mbar_init(bar_s, 1);
     ptx::mbar_init(bar_p, SM_WARPS);
     ptx::mbar_init(bar_o, 1);
@@ -108,7 +122,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     *abort = (err != nullptr && *reinterpret_cast<volatile int*>(&err->code) != 0) ? 1 : 0;
   }
   if (warp == 1) {
-    ptx::tmem_alloc(ptx::smem_u32(tmem_slot), TMEM_COLS);
+    ptx::tmem_alloc(ptx::smem_u32(tmem_slot), tmem_cols);
     ptx::tmem_relinquish();
   }
   ptx::tc_fence_before();
@@ -129,11 +143,18 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         for (int hf = 0; hf < 2; ++hf)
           ptx::tma_load_2d(sK + (uint32_t)(hf * ka + b * KB_ROWS) * 128, &tmKV, bar_qk, D + h * DH + hf * 64,
                            (int)row0 + b * KB_ROWS);
-      ptx::mbar_arrive_expect_tx(bar_v, (uint32_t)n_boxes * 2 * KB_ROWS * 128);
+      ptx::mbar_arrive_expect_tx(bar_v1, (uint32_t)n_boxes * KB_ROWS * 128);
       for (int b = 0; b < n_boxes; ++b)
-        for (int hf = 0; hf < 2; ++hf)
-          ptx::tma_load_2d(sV + (uint32_t)(hf * ka + b * KB_ROWS) * 128, &tmKV, bar_v, 2 * D + h * DH + hf * 64,
-                           (int)row0 + b * KB_ROWS);
+        ptx::tma_load_2d(sV1 + (uint32_t)(b * KB_ROWS) * 128, &tmKV, bar_v1, 2 * D + h * DH + 64, (int)row0 + b * KB_ROWS);
+      // the lower value half: into the query buffer once S = Q K^T no longer reads it
+      bool ok = v0q ? ptx::mbar_wait_bounded(bar_s, 0, abort, WAIT_LIMIT_NS) : true;
+      if (ok) {
+        ptx::mbar_arrive_expect_tx(bar_v0, (uint32_t)n_boxes * KB_ROWS * 128);
+        for (int b = 0; b < n_boxes; ++b)
+          ptx::tma_load_2d(sV0 + (uint32_t)(b * KB_ROWS) * 128, &tmKV, bar_v0, 2 * D + h * DH, (int)row0 + b * KB_ROWS);
+      } else if (!*abort) {
+        record_timeout(err, abort);
+      }
     }
   } else if (warp == 1) {
     if (lane == 0 && !skip) {
@@ -157,13 +178,17 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       }
       if (ok) {
         ptx::tc_fence_after();
-        // O = P V: A = P (K-major, 64-key blocks of 16 KB), B = V (MN-major, dim halves ka*128 B apart)
-        const uint32_t idesc = ptx::idesc_bf16_f32(QT, DH) | (1u << 16);
-        for (int kk = 0; kk < n_cols / 16; ++kk) {
-          const uint32_t a = sK + (kk >> 2) * (QT * 128) + (kk & 3) * 32;
-          const uint32_t b = sV + (uint32_t)kk * 16 * 128;
-          ptx::tc_mma_bf16(tmem_base + O_COL, ptx::smem_desc_sw128(a), smem_desc_sw128_mn(b, (uint32_t)ka * 128),
-                           idesc, kk != 0);
+        // O = P V per value half: A = P (K-major, 64-key blocks of 16 KB), B = V half (MN-major,
+        // one 64-dimension swizzle atom), D = TMEM columns o_col + 64 hf
+        const uint32_t idesc = ptx::idesc_bf16_f32(QT, 64) | (1u << 16);
+        for (int hf = 0; hf < 2; ++hf) {
+          const uint32_t vb = hf ? sV1 : sV0;
+          for (int kk = 0; kk < n_cols / 16; ++kk) {
+            const uint32_t a = sK + (kk >> 2) * (QT * 128) + (kk & 3) * 32;
+            const uint32_t b = vb + (uint32_t)kk * 16 * 128;
+            ptx::tc_mma_bf16(tmem_base + o_col + 64 * hf, ptx::smem_desc_sw128(a),
+                             smem_desc_sw128_mn(b, (uint32_t)ka * 128), idesc, kk != 0);
+          }
         }
         ptx::tc_commit(bar_o);
         volatile int never = 0;
@@ -184,15 +209,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     bool ok = true;
 
     // zero the value rows n_valid .. n_cols - 1 (inside O = P V's K range) once they land
-    ok = ptx::mbar_wait_bounded(bar_v, 0, abort, WAIT_LIMIT_NS);
-    if (ok && n_cols > n_valid) {
+    auto zero_rows = [&](uint8_t* vh) {
       const int nz = n_cols - n_valid;
-      for (int i = ew * 32 + lane; i < nz * 2 * 8; i += SM_WARPS * 32) {
-        const int row = n_valid + i / 16, hf = (i / 8) & 1, c = i & 7;
-        *reinterpret_cast<uint4*>(smem + Q_BYTES + (size_t)ka * 256 + ((size_t)hf * ka + row) * 128 + c * 16) =
-            make_uint4(0u, 0u, 0u, 0u);
-      }
-    }
+      for (int i = ew * 32 + lane; i < nz * 8; i += SM_WARPS * 32)
+        *reinterpret_cast<uint4*>(vh + (size_t)(n_valid + i / 8) * 128 + (i & 7) * 16) = make_uint4(0u, 0u, 0u, 0u);
+    };
+    ok = ptx::mbar_wait_bounded(bar_v1, 0, abort, WAIT_LIMIT_NS);
+    if (ok) zero_rows(gV1);
     if (ok) ok = ptx::mbar_wait_bounded(bar_s, 0, abort, WAIT_LIMIT_NS);
     float m = -INFINITY;
     if (ok) {
@@ -235,6 +258,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       }
     }
     xsum[kh * QT + r] = l;
+    if (ok) ok = ptx::mbar_wait_bounded(bar_v0, 0, abort, WAIT_LIMIT_NS);
+    if (ok) zero_rows(gV0);
     ptx::fence_proxy_async_smem();   // P and the zeroed value rows, before the MMA reads them
     ptx::tc_fence_before();
     __syncwarp();
@@ -250,7 +275,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       bf16* orow = out + (row0 + qrow) * D + h * DH + kh * 64;
       for (int c0 = 0; c0 < 64; c0 += 16) {
         float v[16];
-        ptx::tmem_ld(tmem_base + lane_addr + O_COL + kh * 64 + c0, v);
+        ptx::tmem_ld(tmem_base + lane_addr + o_col + kh * 64 + c0, v);
         ptx::tmem_ld_wait();
         if (qrow < S) {
           uint4 w0 = make_uint4(bf16x2_bits(v[0] * inv, v[1] * inv), bf16x2_bits(v[2] * inv, v[3] * inv),
@@ -268,7 +293,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   __syncthreads();
   if (warp == 1) {
     ptx::tc_fence_after();
-    ptx::tmem_dealloc(tmem_base, TMEM_COLS);
+    ptx::tmem_dealloc(tmem_base, tmem_cols);
   }
 }
 
@@ -292,9 +317,14 @@ cudaError_t attention_tc(const bf16* qkv, bf16* out, int M, const int* lengths, 
   if (make_tmap_bf16(&tq, qkv, M, 3 * D, 3 * D, QT) || make_tmap_bf16(&tkv, qkv, M, 3 * D, 3 * D, KB_ROWS))
     return cudaErrorInvalidValue;
   const int ka = ((S + KB_ROWS - 1) / KB_ROWS) * KB_ROWS;
+  // up to 256 keys S and then O share a 256-column TMEM allocation (two CTAs per SM);
+  // beyond, S takes columns 0..303 and O 320..447 of 512
+  const int n_cols_max = (S + 15) & ~15;
+  const uint32_t tmem_cols = n_cols_max <= 256 ? 256u : 512u;
+  const uint32_t o_col = n_cols_max <= 256 ? 0u : 320u;
   dim3 grid(H, nseq, (S + QT - 1) / QT);
   return launch_kernel(attn_tc_kernel, grid, dim3(NUM_THREADS), smem_bytes(ka), st, tq, tkv, out, lengths, len_mod, S,
-                       ka, tok0, err);
+                       ka, tmem_cols, o_col, tok0, err);
 }
 
 }  // namespace kd

@@ -124,7 +124,7 @@ struct kimodo_ctx {
   Tokens tk;                    // token layout of the call being enqueued
   bool pair_gemm = true;   // 256-row CTA-pair GEMM tiles for the large projections (KIMODO_PAIR_GEMM=0 disables)
   bool stream_k = false;   // stream-K shares for them instead (KIMODO_STREAM_K=1; measured slower on the layer shapes)
-  bool attn_tc = false;    // tcgen05 attention (KIMODO_ATTN_TC=1) instead of the mma.sync kernel
+  bool attn_tc = true;     // tcgen05 attention (KIMODO_ATTN_TC=0: the mma.sync kernel)
   float* sk_partial = nullptr;   // stream-K partial accumulators
   int* sk_flags = nullptr;       // stream-K contributor counters (zero between launches)
   bool bf16() const { return precision == KIMODO_BF16; }
