@@ -55,6 +55,12 @@ __host__ __device__ constexpr size_t smem_bytes(int ka) {
          8 * 8 + 2 * 2 * QT * 4 + 16;
 }
 
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 __device__ __forceinline__ void record_timeout(DevError* err, volatile int* abort) {
   *abort = 1;
   if (err && atomicCAS(&err->code, 0, KIMODO_ETIMEOUT_CODE) == 0) {
@@ -77,7 +83,7 @@ __device__ __forceinline__ uint64_t smem_desc_sw128_mn(uint32_t saddr, uint32_t 
 
 __global__ void __launch_bounds__(NUM_THREADS, 2)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmKV,
-               bf16* __restrict__ out, const int* __restrict__ lengths, int len_mod, int S_pad, int ka,
+               const __grid_constant__ CUtensorMap tmO, bf16* __restrict__ out, const int* __restrict__ lengths, int len_mod, int S_pad, int ka,
                uint32_t tmem_cols, uint32_t o_col, const int* __restrict__ tok0, DevError* err) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -85,10 +91,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   const bool v0q = v0_in_q(ka);
   const uint32_t sQ = ptx::smem_u32(smem);
   const uint32_t sK = sQ + Q_BYTES;                       // also P
-  const uint32_t sV1 = sK + kp * 256;
-  const uint32_t sV0 = v0q ? sQ : sV1 + (uint32_t)ka * 128;
-  uint8_t* gV1 = smem + Q_BYTES + (size_t)kp * 256;       // generic addresses of the value halves
-  uint8_t* gV0 = v0q ? smem : gV1 + (size_t)ka * 128;
+  // value halves: V0 in the Q buffer when it fits, else right after K; V1 after them, so
+  // that V1 - V0 is the (positive) stride between the two 64-dimension atoms of V
+  const uint32_t sV0 = v0q ? sQ : sK + kp * 256;
+  const uint32_t sV1 = sK + kp * 256 + (v0q ? 0u : (uint32_t)ka * 128);
+  uint8_t* gV0 = smem + (sV0 - sQ);                       // generic addresses of the value halves
+  uint8_t* gV1 = smem + (sV1 - sQ);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Q_BYTES + (size_t)kp * 256 + (size_t)ka * 128 +
                                                (v0q ? 0 : (size_t)ka * 128));
   const uint32_t bar0 = ptx::smem_u32(bars);
@@ -178,17 +186,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       }
       if (ok) {
         ptx::tc_fence_after();
-        // O = P V per value half: A = P (K-major, 64-key blocks of 16 KB), B = V half (MN-major,
-        // one 64-dimension swizzle atom), D = TMEM columns o_col + 64 hf
-        const uint32_t idesc = ptx::idesc_bf16_f32(QT, 64) | (1u << 16);
-        for (int hf = 0; hf < 2; ++hf) {
-          const uint32_t vb = hf ? sV1 : sV0;
-          for (int kk = 0; kk < n_cols / 16; ++kk) {
-            const uint32_t a = sK + (kk >> 2) * (QT * 128) + (kk & 3) * 32;
-            const uint32_t b = vb + (uint32_t)kk * 16 * 128;
-            ptx::tc_mma_bf16(tmem_base + o_col + 64 * hf, ptx::smem_desc_sw128(a),
-                             smem_desc_sw128_mn(b, (uint32_t)ka * 128), idesc, kk != 0);
-          }
+        // O = P V: A = P (K-major, 64-key blocks of 16 KB), B = V (MN-major, its two 64-dimension
+        // atoms V0 and V1 sV1 - sV0 bytes apart), D = TMEM columns o_col .. o_col + 127
+        const uint32_t idesc = ptx::idesc_bf16_f32(QT, DH) | (1u << 16);
+        for (int kk = 0; kk < n_cols / 16; ++kk) {
+          const uint32_t a = sK + (kk >> 2) * (QT * 128) + (kk & 3) * 32;
+          const uint32_t b = sV0 + (uint32_t)kk * 16 * 128;
+          ptx::tc_mma_bf16(tmem_base + o_col, ptx::smem_desc_sw128(a), smem_desc_sw128_mn(b, sV1 - sV0), idesc,
+                           kk != 0);
         }
         ptx::tc_commit(bar_o);
         volatile int never = 0;
@@ -206,6 +211,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     const int c_beg = kh == 0 ? 0 : half_cols;
     const int c_end = kh == 0 ? half_cols : n_cols;
     const float sc = 0.08838834764831845f * 1.4426950408889634f;   // log2(e) / sqrt(128)
+    // query rows of this tile that exist: whole warps past them skip the softmax and the
+    // epilogue (TMEM loads are warp-collective), single lanes skip their arithmetic
+    const int rows_valid = S - qt * QT < QT ? S - qt * QT : QT;
+    const bool warp_rows = q * 32 < rows_valid;
+    const bool row_ok = r < rows_valid;
     bool ok = true;
 
     // zero the value rows n_valid .. n_cols - 1 (inside O = P V's K range) once they land
@@ -218,7 +228,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     if (ok) zero_rows(gV1);
     if (ok) ok = ptx::mbar_wait_bounded(bar_s, 0, abort, WAIT_LIMIT_NS);
     float m = -INFINITY;
-    if (ok) {
+    if (ok && warp_rows) {
       ptx::tc_fence_after();
       // pass 1: row maximum over this half's valid keys
       for (int c0 = c_beg; c0 < c_end; c0 += 16) {
@@ -236,17 +246,18 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     m = fmaxf(xmax[r], xmax[QT + r]);
     const float msc = m * sc;
     float l = 0.f;
-    if (ok) {
+    if (ok && warp_rows) {
       // pass 2: p = 2^(s sc - m sc) on valid keys, 0 elsewhere; P row r into 64-key blocks (swizzled)
       for (int c0 = c_beg; c0 < c_end; c0 += 16) {
         float v[16];
         ptx::tmem_ld(tmem_base + lane_addr + c0, v);
         ptx::tmem_ld_wait();
+        if (!row_ok) continue;
         uint32_t w[8];
 #pragma unroll
         for (int j = 0; j < 16; j += 2) {
-          const float p0 = c0 + j < n_valid ? exp2f(fmaf(v[j], sc, -msc)) : 0.f;
-          const float p1 = c0 + j + 1 < n_valid ? exp2f(fmaf(v[j + 1], sc, -msc)) : 0.f;
+          const float p0 = c0 + j < n_valid ? ex2_approx(fmaf(v[j], sc, -msc)) : 0.f;
+          const float p1 = c0 + j + 1 < n_valid ? ex2_approx(fmaf(v[j + 1], sc, -msc)) : 0.f;
           l += p0 + p1;
           w[j / 2] = bf16x2_bits(p0, p1);
         }
@@ -267,24 +278,41 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     asm volatile("bar.sync 1, %0;" ::"n"(SM_WARPS * 32) : "memory");
     l = xsum[r] + xsum[QT + r];
     if (ok) ok = ptx::mbar_wait_bounded(bar_o, 0, abort, WAIT_LIMIT_NS);
-    if (ok) {
+    if (ok && warp_rows) {
       ptx::tc_fence_after();
-      // O row r, dims [64 kh, 64 kh + 64): scale by 1 / l and store if the query exists
+      // O row r, dims [64 kh, 64 kh + 64), scaled by 1 / l.  A warp whose 32 rows all exist
+      // stages them (128-byte swizzle) in the query buffer, dead since O = P V completed, and
+      // stores the 32 x 64 box by TMA; otherwise the existing rows are stored directly.
       const float inv = 1.f / l;
-      const int qrow = qt * QT + r;
-      bf16* orow = out + (row0 + qrow) * D + h * DH + kh * 64;
+      const bool full = q * 32 + 32 <= rows_valid;
+      uint8_t* stg = smem + (size_t)ew * 4096 + (size_t)lane * 128;
+      bf16* orow = out + (row0 + qt * QT + r) * D + h * DH + kh * 64;
       for (int c0 = 0; c0 < 64; c0 += 16) {
         float v[16];
         ptx::tmem_ld(tmem_base + lane_addr + o_col + kh * 64 + c0, v);
         ptx::tmem_ld_wait();
-        if (qrow < S) {
-          uint4 w0 = make_uint4(bf16x2_bits(v[0] * inv, v[1] * inv), bf16x2_bits(v[2] * inv, v[3] * inv),
-                                bf16x2_bits(v[4] * inv, v[5] * inv), bf16x2_bits(v[6] * inv, v[7] * inv));
-          uint4 w1 = make_uint4(bf16x2_bits(v[8] * inv, v[9] * inv), bf16x2_bits(v[10] * inv, v[11] * inv),
-                                bf16x2_bits(v[12] * inv, v[13] * inv), bf16x2_bits(v[14] * inv, v[15] * inv));
+        const uint4 w0 = make_uint4(bf16x2_bits(v[0] * inv, v[1] * inv), bf16x2_bits(v[2] * inv, v[3] * inv),
+                                    bf16x2_bits(v[4] * inv, v[5] * inv), bf16x2_bits(v[6] * inv, v[7] * inv));
+        const uint4 w1 = make_uint4(bf16x2_bits(v[8] * inv, v[9] * inv), bf16x2_bits(v[10] * inv, v[11] * inv),
+                                    bf16x2_bits(v[12] * inv, v[13] * inv), bf16x2_bits(v[14] * inv, v[15] * inv));
+        if (full) {
+          const int ch = c0 / 8;
+          *reinterpret_cast<uint4*>(stg + ((ch ^ (lane & 7)) << 4)) = w0;
+          *reinterpret_cast<uint4*>(stg + (((ch + 1) ^ (lane & 7)) << 4)) = w1;
+        } else if (row_ok) {
           *reinterpret_cast<uint4*>(orow + c0) = w0;
           *reinterpret_cast<uint4*>(orow + c0 + 8) = w1;
         }
+      }
+      if (full) {
+        ptx::fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          ptx::tma_store_2d(&tmO, sQ + (uint32_t)ew * 4096, h * DH + kh * 64, (int)row0 + qt * QT + q * 32);
+          ptx::bulk_commit();
+          ptx::bulk_wait_all();
+        }
+        __syncwarp();
       }
     }
     if (!ok && !*abort) record_timeout(err, abort);
@@ -313,8 +341,9 @@ cudaError_t attention_tc(const bf16* qkv, bf16* out, int M, const int* lengths, 
                          DevError* err, cudaStream_t st, const int* tok0) {
   if (nseq <= 0 || S <= 0 || M <= 0) return cudaSuccess;
   if (S > MAX_FRAMES + 1) return cudaErrorInvalidValue;
-  CUtensorMap tq, tkv;
-  if (make_tmap_bf16(&tq, qkv, M, 3 * D, 3 * D, QT) || make_tmap_bf16(&tkv, qkv, M, 3 * D, 3 * D, KB_ROWS))
+  CUtensorMap tq, tkv, to;
+  if (make_tmap_bf16(&tq, qkv, M, 3 * D, 3 * D, QT) || make_tmap_bf16(&tkv, qkv, M, 3 * D, 3 * D, KB_ROWS) ||
+      make_tmap_plain(&to, out, 2, M, D, D, 64, 32, 128))
     return cudaErrorInvalidValue;
   const int ka = ((S + KB_ROWS - 1) / KB_ROWS) * KB_ROWS;
   // up to 256 keys S and then O share a 256-column TMEM allocation (two CTAs per SM);
@@ -323,8 +352,8 @@ cudaError_t attention_tc(const bf16* qkv, bf16* out, int M, const int* lengths, 
   const uint32_t tmem_cols = n_cols_max <= 256 ? 256u : 512u;
   const uint32_t o_col = n_cols_max <= 256 ? 0u : 320u;
   dim3 grid(H, nseq, (S + QT - 1) / QT);
-  return launch_kernel(attn_tc_kernel, grid, dim3(NUM_THREADS), smem_bytes(ka), st, tq, tkv, out, lengths, len_mod, S,
-                       ka, tmem_cols, o_col, tok0, err);
+  return launch_kernel(attn_tc_kernel, grid, dim3(NUM_THREADS), smem_bytes(ka), st, tq, tkv, to, out, lengths, len_mod,
+                       S, ka, tmem_cols, o_col, tok0, err);
 }
 
 }  // namespace kd
