@@ -128,6 +128,22 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     ptx::mbar_init(bar_o, 1);
     ptx::fence_mbar_init();
     *abort = (err != nullptr && *reinterpret_cast<volatile int*>(&err->code) != 0) ? 1 : 0;
+    if (!*abort) {
+      // the query tile, the keys and the upper value half, issued before the TMEM allocation
+      // and the CTA barrier so that their latency overlaps the set-up
+      ptx::tma_prefetch_desc(&tmQ);
+      ptx::tma_prefetch_desc(&tmKV);
+      const int qrow = (int)row0 + qt * QT;
+      ptx::mbar_arrive_expect_tx(bar_qk, Q_BYTES + (uint32_t)n_boxes * 2 * KB_ROWS * 128);
+      for (int hf = 0; hf < 2; ++hf) ptx::tma_load_2d(sQ + hf * (QT * 128), &tmQ, bar_qk, h * DH + hf * 64, qrow);
+      for (int b = 0; b < n_boxes; ++b)
+        for (int hf = 0; hf < 2; ++hf)
+          ptx::tma_load_2d(sK + (uint32_t)(hf * ka + b * KB_ROWS) * 128, &tmKV, bar_qk, D + h * DH + hf * 64,
+                           (int)row0 + b * KB_ROWS);
+      ptx::mbar_arrive_expect_tx(bar_v1, (uint32_t)n_boxes * KB_ROWS * 128);
+      for (int b = 0; b < n_boxes; ++b)
+        ptx::tma_load_2d(sV1 + (uint32_t)(b * KB_ROWS) * 128, &tmKV, bar_v1, 2 * D + h * DH + 64, (int)row0 + b * KB_ROWS);
+    }
   }
   if (warp == 1) {
     ptx::tmem_alloc(ptx::smem_u32(tmem_slot), tmem_cols);
@@ -141,19 +157,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 
   if (warp == 0) {
     if (lane == 0 && !skip) {
-      // ---------------- TMA: Q tile and keys first (for S), then values
-      ptx::tma_prefetch_desc(&tmQ);
-      ptx::tma_prefetch_desc(&tmKV);
-      const int qrow = (int)row0 + qt * QT;
-      ptx::mbar_arrive_expect_tx(bar_qk, Q_BYTES + (uint32_t)n_boxes * 2 * KB_ROWS * 128);
-      for (int hf = 0; hf < 2; ++hf) ptx::tma_load_2d(sQ + hf * (QT * 128), &tmQ, bar_qk, h * DH + hf * 64, qrow);
-      for (int b = 0; b < n_boxes; ++b)
-        for (int hf = 0; hf < 2; ++hf)
-          ptx::tma_load_2d(sK + (uint32_t)(hf * ka + b * KB_ROWS) * 128, &tmKV, bar_qk, D + h * DH + hf * 64,
-                           (int)row0 + b * KB_ROWS);
-      ptx::mbar_arrive_expect_tx(bar_v1, (uint32_t)n_boxes * KB_ROWS * 128);
-      for (int b = 0; b < n_boxes; ++b)
-        ptx::tma_load_2d(sV1 + (uint32_t)(b * KB_ROWS) * 128, &tmKV, bar_v1, 2 * D + h * DH + 64, (int)row0 + b * KB_ROWS);
+      // ---------------- TMA (Q, K and V1 were issued at set-up)
       // the lower value half: into the query buffer once S = Q K^T no longer reads it
       bool ok = v0q ? ptx::mbar_wait_bounded(bar_s, 0, abort, WAIT_LIMIT_NS) : true;
       if (ok) {

@@ -78,6 +78,7 @@ struct Workspace {
   void* emb = nullptr; float* txt[2] = {}; void* tpe = nullptr; void* thid = nullptr; float* tmlp[2] = {};
   int* lengths = nullptr; float* st_text = nullptr; float* st_null = nullptr;
   int* tok0 = nullptr; int* row_seq = nullptr;   // packed token layout (valid tokens only)
+  float* stats[2] = {};                           // LayerNorm row statistics (mean, 1/std) [M][2]
 };
 
 // Token rows of a call: the padded layout (every sequence frames + 1 rows) or, when the
@@ -125,6 +126,7 @@ struct kimodo_ctx {
   bool pair_gemm = true;   // 256-row CTA-pair GEMM tiles for the large projections (KIMODO_PAIR_GEMM=0 disables)
   bool stream_k = false;   // stream-K shares for them instead (KIMODO_STREAM_K=1; measured slower on the layer shapes)
   bool attn_tc = true;     // tcgen05 attention (KIMODO_ATTN_TC=0: the mma.sync kernel)
+  bool ln_lite = true;     // LayerNorm writes row statistics, residual epilogues normalise (KIMODO_LN_LITE=0)
   float* sk_partial = nullptr;   // stream-K partial accumulators
   int* sk_flags = nullptr;       // stream-K contributor counters (zero between launches)
   bool bf16() const { return precision == KIMODO_BF16; }
@@ -181,7 +183,7 @@ int gemm(kimodo_ctx* c, const void* A, int lda, const void* W, int ldw, int M, i
   const double flops = 2.0 * M * N * K;
   const double bytes = (double)c->elem() * ((double)M * K + (double)N * K) +
                        (double)M * N * (out_f32 ? 4.0 : (double)c->elem()) +
-                       (kind == EPI_BIAS_RESID ? (double)M * N * 4.0 : 0.0);
+                       (kind == EPI_BIAS_RESID || kind == EPI_BIAS_RESID_LN ? (double)M * N * 4.0 : 0.0);
   if (c->bf16()) {
     if (c->pair_gemm && c->stream_k && M >= 1024 && N >= 256 && gemm_tc2_supports(kind, out_f32)) {
       return launch(c, cls_override >= 0 ? cls_override : CLS_GEMM_TC, flops, bytes, st, "gemm_sk",
@@ -307,7 +309,8 @@ int ensure_workspace(kimodo_ctx* c, int nseq, int frames, int steps) {
       {(void**)&w.tmlp[0], (size_t)ST * D * 4},            {(void**)&w.tmlp[1], (size_t)ST * D * 4},
       {(void**)&w.lengths, (size_t)NS * 4},                {(void**)&w.st_text, (size_t)NS * DTXT * 4},
       {(void**)&w.st_null, (size_t)NS * DTXT * 4},        {(void**)&w.tok0, (size_t)(NS + 1) * 4},
-      {(void**)&w.row_seq, (size_t)R2 * 4}};
+      {(void**)&w.row_seq, (size_t)R2 * 4},               {(void**)&w.stats[0], (size_t)R2 * 8},
+      {(void**)&w.stats[1], (size_t)R2 * 8}};
   for (auto& p : plan) off += align256(p.second);
   void* arena = nullptr;
   cudaError_t err = cudaMalloc(&arena, off);
@@ -385,6 +388,18 @@ int run_net(kimodo_ctx* c, int net, int nseq, int T, int len_mod, const void* A_
   const void* resid = c->bf16() ? static_cast<const void*>(w.y) : w.h;
   float* ln32 = c->bf16() ? w.y : nullptr;
   const double eb = (double)c->elem();
+  // Row-statistics residual (bf16 path): y keeps the un-normalised sums z;
+  // LayerNorm writes only the bf16 operand h and (mean, 1/std) per row, and the next
+  // residual epilogue adds gamma (z - mean) / std + beta itself (EPI_BIAS_RESID_LN).
+  const bool lite = c->bf16() && c->ln_lite && !c->stream_k && w.stats[0] != nullptr;
+  if (lite) ln32 = nullptr;
+  auto resid_epi = [&](EpiParams& e, int which, const float* g, const float* b) {
+    if (!lite || g == nullptr) return EPI_BIAS_RESID;
+    e.ln_stats = w.stats[which];
+    e.ln_g = g;
+    e.ln_b = b;
+    return EPI_BIAS_RESID_LN;
+  };
   for (int l = 0; l < L; ++l) {
     EpiParams e;
     e.bias = n.qkv_b[l]; e.out = w.qkv; e.ldo = 3 * D; e.N = 3 * D; e.M = M;
@@ -411,18 +426,23 @@ int run_net(kimodo_ctx* c, int net, int nseq, int T, int len_mod, const void* A_
     }
     EpiParams eo;
     eo.bias = n.o_b[l]; eo.out = w.y; eo.ldo = D; eo.resid = resid; eo.ldr = D; eo.N = D; eo.M = M;
-    KD_TRY(gemm(c, w.attn, D, n.o_W[l], D, M, D, D, EPI_BIAS_RESID, true, eo, st));
-    const double lnb = (double)M * D * (4.0 + eb + (c->bf16() ? 4.0 : 0.0));
-    KD_TRY(launch(c, CLS_LN, 0, lnb, st, "layernorm",
-                  [&] { return layernorm(w.y, w.h, c->bf16(), n.ln1_g[l], n.ln1_b[l], M, st, ln32); }));
+    // layer 0 adds the un-normalised input projection; later layers the previous LayerNorm 2
+    const int ko = resid_epi(eo, 1, l > 0 ? n.ln2_g[l - 1] : nullptr, l > 0 ? n.ln2_b[l - 1] : nullptr);
+    KD_TRY(gemm(c, w.attn, D, n.o_W[l], D, M, D, D, ko, true, eo, st));
+    const double lnb = lite ? (double)M * D * (4.0 + eb) + (double)M * 8 : (double)M * D * (4.0 + eb + (c->bf16() ? 4.0 : 0.0));
+    KD_TRY(launch(c, CLS_LN, 0, lnb, st, "layernorm", [&] {
+      return layernorm(w.y, w.h, c->bf16(), n.ln1_g[l], n.ln1_b[l], M, st, ln32, lite ? w.stats[0] : nullptr);
+    }));
     EpiParams e1;
     e1.bias = n.ff1_b[l]; e1.out = w.u; e1.ldo = F; e1.N = F; e1.M = M;
     KD_TRY(gemm(c, w.h, D, n.ff1_W[l], D, M, F, D, EPI_BIAS_GELU, act_f32, e1, st));
     EpiParams e2;
     e2.bias = n.ff2_b[l]; e2.out = w.y; e2.ldo = D; e2.resid = resid; e2.ldr = D; e2.N = D; e2.M = M;
-    KD_TRY(gemm(c, w.u, F, n.ff2_W[l], F, M, D, F, EPI_BIAS_RESID, true, e2, st));
-    KD_TRY(launch(c, CLS_LN, 0, lnb, st, "layernorm",
-                  [&] { return layernorm(w.y, w.h, c->bf16(), n.ln2_g[l], n.ln2_b[l], M, st, ln32); }));
+    const int kf = resid_epi(e2, 0, n.ln1_g[l], n.ln1_b[l]);
+    KD_TRY(gemm(c, w.u, F, n.ff2_W[l], F, M, D, F, kf, true, e2, st));
+    KD_TRY(launch(c, CLS_LN, 0, lnb, st, "layernorm", [&] {
+      return layernorm(w.y, w.h, c->bf16(), n.ln2_g[l], n.ln2_b[l], M, st, ln32, lite ? w.stats[1] : nullptr);
+    }));
   }
   EpiParams eo;
   eo.bias = n.out_b; eo.out = hat; eo.ldo = n.dout; eo.lengths = w.lengths; eo.len_mod = len_mod; eo.S = S;
@@ -601,6 +621,7 @@ int kimodo_load_weights(kimodo_ctx** out_ctx, const float* host_blob, size_t n_f
   if (const char* ev = getenv("KIMODO_PAIR_GEMM")) c->pair_gemm = ev[0] != '0';
   if (const char* ev = getenv("KIMODO_STREAM_K")) c->stream_k = ev[0] != '0';
   if (const char* ev = getenv("KIMODO_ATTN_TC")) c->attn_tc = ev[0] != '0';
+  if (const char* ev = getenv("KIMODO_LN_LITE")) c->ln_lite = ev[0] != '0';
   c->num_sms = prop.multiProcessorCount;
   auto fail = [&](int code) {
     kimodo_free(c);
@@ -1193,6 +1214,8 @@ constexpr size_t noalloc_layout(char* base, size_t e, size_t rows, size_t nseq, 
   char* tm1 = take(D * 4);
   char* len = take(nseq * 4);
   char* stt = take(nseq * DTXT * 4);
+  char* st0 = take(rows * 8);
+  char* st1 = take(rows * 8);
   if (w) {
     w->h = h; w->qkv = qkv; w->attn = attn; w->u = u; w->y = reinterpret_cast<float*>(y);
     w->A_root = ar; w->A_body = ab;
@@ -1202,6 +1225,7 @@ constexpr size_t noalloc_layout(char* base, size_t e, size_t rows, size_t nseq, 
     w->tpe = tpe; w->thid = thid;
     w->tmlp[0] = reinterpret_cast<float*>(tm0); w->tmlp[1] = reinterpret_cast<float*>(tm1);
     w->lengths = reinterpret_cast<int*>(len); w->st_text = reinterpret_cast<float*>(stt); w->st_null = nullptr;
+    w->stats[0] = reinterpret_cast<float*>(st0); w->stats[1] = reinterpret_cast<float*>(st1);
   }
   return off;
 }

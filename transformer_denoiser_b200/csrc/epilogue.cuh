@@ -19,6 +19,9 @@ enum EpiKind : int {
   EPI_BIAS_RESID = 3, // out = acc + b + resid          (attention out-proj, FFN2)
   EPI_INPROJ = 4,     // token 0: cond[seq] + tvec + pe[0];  token j: acc + b + pe[j]
   EPI_OUTPROJ = 5,    // frame tokens only, written as [seq, T, ldo]; padded frames 0
+  EPI_BIAS_RESID_LN = 6, // out = acc + b + LN(resid): the residual is the un-normalised sum
+                         // z of the previous sub-layer, normalised here from its row
+                         // statistics (mean, 1/std) and the LayerNorm's gamma / beta
 };
 
 struct EpiParams {
@@ -38,6 +41,10 @@ struct EpiParams {
   // row_seq[r] is the sequence of row r; both null for the padded layout (row = s * S + pos)
   const int* tok0 = nullptr;
   const int* row_seq = nullptr;
+  // EPI_BIAS_RESID_LN: row statistics [M][2] = (mean, 1/std) and the LayerNorm affine [N]
+  const float* ln_stats = nullptr;
+  const float* ln_g = nullptr;
+  const float* ln_b = nullptr;
   int T = 1;                     // frames per sequence (EPI_OUTPROJ)
   int N = 0;                     // valid output columns
   int M = 0;                     // valid rows
@@ -277,12 +284,19 @@ __device__ __forceinline__ void epilogue_prefetch(const EpiParams& e, int row0, 
     bias4.z = col + 2 < e.N ? e.bias[col + 2] : 0.f;
     bias4.w = col + 3 < e.N ? e.bias[col + 3] : 0.f;
   }
-  if constexpr (KIND == EPI_BIAS_RESID || KIND == EPI_INPROJ) {
+  if constexpr (KIND == EPI_BIAS_RESID_LN) {
+    // bias + beta, summed as the pair GEMM's epilogue sums them
+    if (col + 4 <= e.N) {
+      const float4 be = ld4(e.ln_b + col);
+      bias4.x += be.x; bias4.y += be.y; bias4.z += be.z; bias4.w += be.w;
+    }
+  }
+  if constexpr (KIND == EPI_BIAS_RESID || KIND == EPI_BIAS_RESID_LN || KIND == EPI_INPROJ) {
     if (col + 4 > e.N) return;
 #pragma unroll
     for (int p = 0; p < Ln::PASSES; ++p) {
       const int row = min(row0 + p * Ln::RPP + rsub, e.M - 1);
-      if constexpr (KIND == EPI_BIAS_RESID) {
+      if constexpr (KIND == EPI_BIAS_RESID || KIND == EPI_BIAS_RESID_LN) {
         pre[p] = ld4(reinterpret_cast<const float*>(e.resid) + (long)row * e.ldr + col);
       } else {
         int seq, pos;
@@ -356,6 +370,14 @@ __device__ __forceinline__ void epilogue_warp_tile(const EpiParams& e, const flo
         }
         if constexpr (KIND == EPI_BIAS_RESID) {
           v[0] += pre[p].x; v[1] += pre[p].y; v[2] += pre[p].z; v[3] += pre[p].w;
+        }
+        if constexpr (KIND == EPI_BIAS_RESID_LN) {
+          // the residual is the un-normalised sum z: add gamma (z - mean) / std (+ beta, in b4)
+          const float2 st2 = *reinterpret_cast<const float2*>(e.ln_stats + 2 * (long)min(row, e.M - 1));
+          const float ra = st2.y, rb = -st2.x * st2.y;
+          const float4 g4 = ld4(e.ln_g + col);
+          v[0] += fmaf(pre[p].x, ra, rb) * g4.x; v[1] += fmaf(pre[p].y, ra, rb) * g4.y;
+          v[2] += fmaf(pre[p].z, ra, rb) * g4.z; v[3] += fmaf(pre[p].w, ra, rb) * g4.w;
         }
       }
       if (in_rows) {

@@ -371,12 +371,14 @@ static cudaError_t dispatch(const GemmArgs& g, int bn, int kind, bool out_f32, c
   KD_TC(256, 4, EPI_BIAS, bf16)
   KD_TC(256, 4, EPI_BIAS_GELU, bf16)
   KD_TC(256, 4, EPI_BIAS_RESID, float)
+  KD_TC(256, 4, EPI_BIAS_RESID_LN, float)
   KD_TC(256, 4, EPI_INPROJ, bf16)
   KD_TC(128, 6, EPI_BIAS, bf16)
   KD_TC(128, 6, EPI_BIAS, float)
   KD_TC(128, 6, EPI_BIAS_GELU, bf16)
   KD_TC(128, 6, EPI_BIAS_SILU, bf16)
   KD_TC(128, 6, EPI_BIAS_RESID, float)
+  KD_TC(128, 6, EPI_BIAS_RESID_LN, float)
   KD_TC(128, 6, EPI_INPROJ, bf16)
   KD_TC(128, 6, EPI_OUTPROJ, float)
   KD_TC(16, 8, EPI_OUTPROJ, float)

@@ -50,10 +50,11 @@ struct Tc2Cfg {
   static constexpr int PART_CH = (NCH + 1) / 2;
   static constexpr uint32_t STG_BYTES = 32 * CW * 4;     // one 32-row staging tile (fp32 size)
   // bytes of one staging row of the stored type (fp32 64, bf16 32): also the TMA swizzle span
-  static constexpr int ROW_BYTES = CW * (KIND == EPI_BIAS_RESID ? 4 : 2);
+  static constexpr bool RES = KIND == EPI_BIAS_RESID || KIND == EPI_BIAS_RESID_LN;
+  static constexpr int ROW_BYTES = CW * (RES ? 4 : 2);
   // staging tiles per epilogue warp: two alternating ones, or, with a residual, one per
   // chunk of the warp's tile share so the whole residual share is loaded ahead of the MMA
-  static constexpr int NBUF = KIND == EPI_BIAS_RESID ? PART_CH : 2;
+  static constexpr int NBUF = RES ? PART_CH : 2;
   static constexpr uint32_t EPI_BYTES = EPI_WARPS * NBUF * STG_BYTES;
   static constexpr uint32_t NUM_BARS = 2 * STAGES + 5 + NBUF * EPI_WARPS;
   static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE_BYTES + EPI_BYTES + NUM_BARS * 8 + 16;
@@ -116,7 +117,7 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
     ptx::tma_prefetch_desc(&tmA);
     ptx::tma_prefetch_desc(&tmB);
     ptx::tma_prefetch_desc(&tmO);
-    if (KIND == EPI_BIAS_RESID) ptx::tma_prefetch_desc(&tmR);
+    if (C::RES) ptx::tma_prefetch_desc(&tmR);
   }
   if (warp == 1) {
     ptx::tmem_alloc_pair(ptx::smem_u32(tmem_slot), C::TMEM_COLS);
@@ -242,13 +243,32 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
       // chunk k of this tile is the warp's chunk number cc0 + k and uses staging tile (cc0 + k) % NBUF
       const int cc0 = cc;
       auto stage_tile = [&](int a) { return stg_base + (a % C::NBUF) * C::STG_BYTES; };
-      auto load_bias = [&](int k, float4 (&b4)[CW / 4]) {
+      // per-column operands of chunk k: bias, and for EPI_BIAS_RESID_LN the LayerNorm gamma and
+      // (bias + beta), so that x = acc + (bias + beta) + (z * rstd - mean * rstd) * gamma
+      auto load_bias = [&](int k, float4 (&b4)[CW / 4], float4 (&g4)[CW / 4]) {
 #pragma unroll
-        for (int j = 0; j < CW / 4; ++j) b4[j] = ld4(ep.bias + gcol + k * CW + 4 * j);
+        for (int j = 0; j < CW / 4; ++j) {
+          b4[j] = ld4(ep.bias + gcol + k * CW + 4 * j);
+          if constexpr (KIND == EPI_BIAS_RESID_LN) {
+            const float4 be = ld4(ep.ln_b + gcol + k * CW + 4 * j);
+            b4[j].x += be.x; b4[j].y += be.y; b4[j].z += be.z; b4[j].w += be.w;
+            g4[j] = ld4(ep.ln_g + gcol + k * CW + 4 * j);
+          }
+        }
       };
-      float4 ba[CW / 4], bb[CW / 4];
+      // this lane's row statistics for EPI_BIAS_RESID_LN: z * rs_a + rs_b = (z - mean) / std
+      float rs_a = 1.f, rs_b = 0.f;
+      if constexpr (KIND == EPI_BIAS_RESID_LN) {
+        const int row = row0 + lane;
+        if (nch > 0 && row < ep.M) {
+          const float2 st2 = *reinterpret_cast<const float2*>(ep.ln_stats + 2 * (long)row);
+          rs_a = st2.y;
+          rs_b = -st2.x * st2.y;
+        }
+      }
+      float4 ba[CW / 4], bb[CW / 4], ga[CW / 4], gb[CW / 4];
       if (nch > 0) {
-        if (KIND == EPI_BIAS_RESID && lane == 0) {
+        if (C::RES && lane == 0) {
           // the whole residual share of this tile, one staging tile per chunk, loaded while
           // the MMAs run; the previous tile's stores have read their staging tiles first
           ptx::bulk_wait_read<0>();
@@ -258,7 +278,7 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
             ptx::tma_load_2d(ptx::smem_u32(stage_tile(cc0 + k)), &tmR, res_bar(ew, b), gcol + k * CW, row0);
           }
         }
-        load_bias(0, ba);
+        load_bias(0, ba, ga);
       }
       if (!ptx::mbar_wait_bounded(tfull_bar(acc), acc_phase, abort, WAIT_LIMIT_NS)) {
         if (!*abort) record_timeout(err, WHERE_GEMM_EPILOGUE, abort);
@@ -277,7 +297,7 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
         continue;
       }
       // finish chunk k (the warp's chunk number cc == cc0 + k) from accumulator values v, bias b4
-      auto process = [&](float (&v)[CW], const float4 (&b4)[CW / 4], int k) -> bool {
+      auto process = [&](float (&v)[CW], const float4 (&b4)[CW / 4], const float4 (&g4)[CW / 4], int k) -> bool {
         uint8_t* st = stage_tile(cc);
         // this lane's row of the staging tile; its 16-byte unit u sits at unit u ^ swz
         // (the tile's TMA swizzle, so that the warp's row-per-lane accesses hit distinct banks)
@@ -299,12 +319,16 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
 #pragma unroll
           for (int j = 0; j < CW; ++j) x[j] = silu_f(x[j]);
         }
-        if constexpr (KIND == EPI_BIAS_RESID) {
+        if constexpr (C::RES) {
           if (!ptx::mbar_wait_bounded(res_bar(ew, cc % C::NBUF), (cc / C::NBUF) & 1, abort, WAIT_LIMIT_NS))
             return false;
 #pragma unroll
           for (int u = 0; u < CW / 4; ++u) {
-            const float4 r = *reinterpret_cast<const float4*>(srow + ((u ^ swz) << 4));
+            float4 r = *reinterpret_cast<const float4*>(srow + ((u ^ swz) << 4));
+            if constexpr (KIND == EPI_BIAS_RESID_LN) {
+              r.x = fmaf(r.x, rs_a, rs_b) * g4[u].x; r.y = fmaf(r.y, rs_a, rs_b) * g4[u].y;
+              r.z = fmaf(r.z, rs_a, rs_b) * g4[u].z; r.w = fmaf(r.w, rs_a, rs_b) * g4[u].w;
+            }
             x[4 * u] += r.x; x[4 * u + 1] += r.y; x[4 * u + 2] += r.z; x[4 * u + 3] += r.w;
           }
         } else {
@@ -340,17 +364,17 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
         if (c == nch - 1) release();
         if (c + 1 < nch) {
           ptx::tmem_ld(taddr + (c + 1) * CW, vb);
-          load_bias(c + 1, bb);
+          load_bias(c + 1, bb, gb);
         }
-        if (!process(va, ba, c)) { failed = true; break; }
+        if (!process(va, ba, ga, c)) { failed = true; break; }
         if (c + 1 >= nch) break;
         ptx::tmem_ld_wait();
         if (c + 1 == nch - 1) release();
         if (c + 2 < nch) {
           ptx::tmem_ld(taddr + (c + 2) * CW, va);
-          load_bias(c + 2, ba);
+          load_bias(c + 2, ba, ga);
         }
-        if (!process(vb, bb, c + 1)) { failed = true; break; }
+        if (!process(vb, bb, gb, c + 1)) { failed = true; break; }
       }
       if (failed && !*abort) record_timeout(err, WHERE_GEMM_EPILOGUE, abort);
     }
@@ -409,7 +433,7 @@ struct Tc2Launcher {
     static_assert(Cf::ROW_BYTES == Cf::CW * (int)sizeof(OutT), "staging row bytes");
     if (make_tmap_plain(&to, ep.out, (int)sizeof(OutT), g.M, g.N, ep.ldo, Cf::CW, 32, Cf::ROW_BYTES))
       return cudaErrorInvalidValue;
-    if (KIND == EPI_BIAS_RESID) {
+    if (Cf::RES) {
       if (make_tmap_plain(&tr, ep.resid, 4, g.M, g.N, ep.ldr, Cf::CW, 32, Cf::ROW_BYTES)) return cudaErrorInvalidValue;
     } else {
       tr = to;
@@ -445,7 +469,8 @@ int Tc2Launcher<BN, STAGES, KIND, OutT>::max_clusters = 0;
   X(160, 7, EPI_BIAS, bf16) X(144, 7, EPI_BIAS, bf16)   \
   X(256, 6, EPI_BIAS_GELU, bf16) X(208, 6, EPI_BIAS_GELU, bf16) \
   X(160, 7, EPI_BIAS_GELU, bf16) X(144, 7, EPI_BIAS_GELU, bf16) \
-  X(160, 5, EPI_BIAS_RESID, float) X(144, 5, EPI_BIAS_RESID, float)
+  X(160, 5, EPI_BIAS_RESID, float) X(144, 5, EPI_BIAS_RESID, float)   \
+  X(160, 5, EPI_BIAS_RESID_LN, float) X(144, 5, EPI_BIAS_RESID_LN, float)
 
 }  // namespace
 
@@ -462,7 +487,7 @@ cudaError_t gemm_tc2_prepare() {
 
 bool gemm_tc2_supports(int kind, bool out_f32) {
   return (kind == EPI_BIAS && !out_f32) || (kind == EPI_BIAS_GELU && !out_f32) ||
-         (kind == EPI_BIAS_RESID && out_f32);
+         ((kind == EPI_BIAS_RESID || kind == EPI_BIAS_RESID_LN) && out_f32);
 }
 
 // Tile N minimizing (rounds of pair tiles) x (N + per-tile overhead) over the available
@@ -471,8 +496,9 @@ bool gemm_tc2_supports(int kind, bool out_f32) {
 int gemm_tc2_pick_bn(int M, int N, int kind) {
   const int all[4] = {256, 208, 160, 144};
   const int resid[2] = {160, 144};
-  const int* cands = kind == EPI_BIAS_RESID ? resid : all;
-  const int ncand = kind == EPI_BIAS_RESID ? 2 : 4;
+  const bool res = kind == EPI_BIAS_RESID || kind == EPI_BIAS_RESID_LN;
+  const int* cands = res ? resid : all;
+  const int ncand = res ? 2 : 4;
   const int pairs = Tc2Launcher<256, 6, EPI_BIAS, bf16>::max_clusters > 0
                         ? Tc2Launcher<256, 6, EPI_BIAS, bf16>::max_clusters : 74;
   const long mt = (M + 2 * BMC - 1) / (2 * BMC);

@@ -80,9 +80,10 @@ size_t attention_tc_smem(int S);
 cudaError_t build_token_map(const int* lengths, int len_mod, int nseq, int* tok0, int* row_seq, cudaStream_t st);
 
 // Row LayerNorm over D features: y fp32 [M, D] -> out (bf16 or fp32) [M, D], and
-// optionally an fp32 copy into out32 (which may be y itself).
+// optionally an fp32 copy into out32 (which may be y itself) and the row statistics
+// (mean, 1/std) into stats [M][2].
 cudaError_t layernorm(const float* y, void* out, bool out_bf16, const float* gamma, const float* beta, int M,
-                      cudaStream_t st, float* out32 = nullptr);
+                      cudaStream_t st, float* out32 = nullptr, float* stats = nullptr);
 
 // ---- motion / sampler kernels (element type of the activation matrices: bf16 or fp32)
 

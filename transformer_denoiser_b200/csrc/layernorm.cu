@@ -4,7 +4,8 @@
 // and the biased variance are two warp-shuffle reductions (two passes over the
 // registers), eps = 1e-5; statistics in fp32, output bf16 or fp32, plus an
 // optional fp32 copy that may overwrite the input row in place (the row is read
-// completely into registers before any store).
+// completely into registers before any store) and optional row statistics, from
+// which a later residual epilogue rebuilds the normalised row instead of reading it.
 #include <cuda_runtime.h>
 
 #include "common.cuh"
@@ -28,7 +29,8 @@ __device__ __forceinline__ float warp_sum(float v) {
 template <typename OutT>
 __global__ void __launch_bounds__(LN_WARPS * 32, 18) layernorm_kernel(const float* y, OutT* __restrict__ out,
                                                         const float* __restrict__ gamma,
-                                                        const float* __restrict__ beta, int M, float* out32) {
+                                                        const float* __restrict__ beta, int M, float* out32,
+                                                        float* __restrict__ stats) {
   ptx::pdl_wait();
   ptx::pdl_trigger();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -52,6 +54,7 @@ __global__ void __launch_bounds__(LN_WARPS * 32, 18) layernorm_kernel(const floa
     q += d * d;
   }
   const float rstd = 1.0f / sqrtf(warp_sum(q) * (1.0f / D) + 1e-5f);
+  if (stats != nullptr && lane == 0) *reinterpret_cast<float2*>(stats + 2 * (long)row) = make_float2(mean, rstd);
   OutT* orow = out + (long)row * D;
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
@@ -78,14 +81,14 @@ __global__ void __launch_bounds__(LN_WARPS * 32, 18) layernorm_kernel(const floa
 }  // namespace
 
 cudaError_t layernorm(const float* y, void* out, bool out_bf16, const float* gamma, const float* beta, int M,
-                      cudaStream_t st, float* out32) {
+                      cudaStream_t st, float* out32, float* stats) {
   if (M <= 0) return cudaSuccess;
   const int grid = (M + LN_WARPS - 1) / LN_WARPS;
   if (out_bf16)
     return launch_kernel(layernorm_kernel<bf16>, dim3(grid), dim3(LN_WARPS * 32), 0, st, y, static_cast<bf16*>(out), gamma, beta,
-                         M, out32);
+                         M, out32, stats);
   return launch_kernel(layernorm_kernel<float>, dim3(grid), dim3(LN_WARPS * 32), 0, st, y, static_cast<float*>(out), gamma, beta,
-                       M, out32);
+                       M, out32, stats);
 }
 
 }  // namespace kd
