@@ -225,6 +225,51 @@ def oracle_sample(target_s: float = 12.0):
 
 # --------------------------------------------------------------------------- our arm
 
+def secondary_workloads(model, dev, flush, reps=3):
+    """The other two generation workloads, timed like the headline one (device inputs,
+    L2 flushed, CUDA events, warm graph): 50-step latency of one 180-frame prompt, and a
+    ragged batch of 64 prompts (lengths U{60..300} padded to 300 frames, CFG 2.5, garbage
+    in the padding) on the packed token layout (lengths in host memory) and on the padded
+    one (lengths in device memory)."""
+    import torch
+    import synth
+
+    def timed(fn):
+        fn()
+        torch.cuda.synchronize()
+        best = None
+        for _ in range(reps):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            torch.cuda.synchronize()
+            ms = e0.elapsed_time(e1)
+            best = ms if best is None else min(best, ms)
+        return best
+
+    emb1 = torch.from_numpy(synth.text_embeddings(1)).to(dev)
+    null = torch.zeros(4096, device=dev)
+    n1 = torch.from_numpy(synth.noise(1, 180)).to(dev)
+    l1 = torch.full((1,), 180, dtype=torch.int32, device=dev)
+    c3_ms = timed(lambda: model.ddim_sample(emb1, null, n1, l1, 50, 2.0))
+    B, T = 64, 300
+    lengths = synth.lengths_uniform(B, 60, 300)
+    emb = torch.from_numpy(synth.text_embeddings(B)).to(dev)
+    noise = torch.from_numpy(synth.fill_padding(synth.noise(B, T), lengths)).to(dev)
+    packed_ms = timed(lambda: model.ddim_sample(emb, null, noise, lengths, 50, 2.5))
+    d_len = torch.from_numpy(lengths).to(dev)
+    padded_ms = timed(lambda: model.ddim_sample(emb, null, noise, d_len, 50, 2.5))
+    valid_tokens = 2 * 2 * int((lengths + 1).sum()) * 50
+    return {"c3_latency": {"workload": "50-step DDIM, 1 prompt x 180 frames, CFG 2.0", "ms": round(c3_ms, 3)},
+            "c5_ragged": {"workload": "50-step DDIM, 64 prompts, lengths U{60..300} padded to 300 frames, CFG 2.5",
+                          "clips_per_min_packed": round(B * 60e3 / packed_ms, 2),
+                          "clips_per_min_padded": round(B * 60e3 / padded_ms, 2),
+                          "valid_tokens_per_s_packed": round(valid_tokens / (packed_ms / 1e3), 1),
+                          "ms_packed": round(packed_ms, 2), "ms_padded": round(padded_ms, 2)}}
+
+
 def run_ours(args, rank, world, local_rank):
     import torch
     import torch.distributed as dist
@@ -305,6 +350,10 @@ def run_ours(args, rank, world, local_rank):
     model.sync_status()
 
     ms_max, e2e_max = max_over_ranks([ms, e2e_ms], dev, world)
+    secondary = None
+    if world == 1 and not args.no_secondary and not args.ddim_steps:
+        secondary = secondary_workloads(model, dev, flush)
+        model.sync_status()
     model.close()
     if rank != 0:
         return None
@@ -323,6 +372,8 @@ def run_ours(args, rank, world, local_rank):
         "roofline": roofline(prof),
         "clocks": clk.summary(),
     }
+    if secondary is not None:
+        line["secondary"] = secondary
     if args.ddim_steps:
         line["note"] = (f"profiling case: {args.ddim_steps} DDIM steps per generation instead of "
                         f"{w['steps']}; not a benchmark number")
@@ -360,6 +411,8 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-secondary", action="store_true",
+                    help="skip the c3 latency and c5 ragged-batch measurements")
     ap.add_argument("--ddim-steps", type=int, default=0,
                     help="profiling only: DDIM steps per generation (default: the workload's 100)")
     args = ap.parse_args(argv)
