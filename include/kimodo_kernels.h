@@ -34,8 +34,9 @@ enum {
  * resid: fp32 [M, ldr] (KIMODO_EPI_BIAS_RESID only, else NULL); may equal out.
  * out: bf16 (out_f32 = 0) or fp32 (out_f32 = 1), row stride ldo.
  * out, resid, bias 16-byte aligned; ldo, ldr multiples of 4.
- * KIMODO_EPI_BIAS_RESID requires out_f32 = 1.  tile_n: 128 or 256 (output
- * columns per tile), or 0 to let the library choose.
+ * KIMODO_EPI_BIAS_RESID requires out_f32 = 1.  tile_n: 32, 64, 128 or 256
+ * (output columns per tile; 32 and 64 are built for the bias and GELU epilogues
+ * with bf16 output and the residual epilogue), or 0 to let the library choose.
  */
 KIMODO_API int kimodo_gemm_bf16(const void* A, int lda, const void* W, int ldw, const float* bias,
                                 const void* resid, int ldr, void* out, int ldo, int M, int N, int K,

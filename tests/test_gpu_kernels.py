@@ -43,6 +43,12 @@ GEMM_CASES = [
     (257, 1024, 279, 320, kb.EPI_BIAS, True, 128),         # body input width, ragged K
     (200, 274, 1024, 1024, kb.EPI_BIAS, True, 128),        # body output width, ragged N
     (100, 1024, 4096, 4096, kb.EPI_BIAS, True, 128),       # text projection
+    (362, 3072, 1024, 1024, kb.EPI_BIAS, False, 64),       # narrow tiles for a few hundred tokens
+    (362, 2048, 1024, 1024, kb.EPI_BIAS_GELU, False, 64),
+    (362, 1024, 2048, 2048, kb.EPI_BIAS_RESID, True, 32),
+    (300, 1040, 1024, 1024, kb.EPI_BIAS_RESID, True, 64),  # ragged last tile, partial epilogue parts
+    (130, 1008, 1024, 1024, kb.EPI_BIAS, False, 32),
+    (5, 2048, 1024, 1024, kb.EPI_BIAS_GELU, False, 32),
 ]
 
 

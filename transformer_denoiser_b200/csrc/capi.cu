@@ -57,6 +57,9 @@ int set_error(int code, const char* fmt, ...) {
     if (s_ != KIMODO_OK) return s_; \
   } while (0)
 
+// Folded LayerNorm: arrival counters for up to this many 32-row groups (2 M token rows).
+constexpr int PART_GROUPS_MAX = 1 << 16;
+
 enum LaunchClass { CLS_GEMM_TC = 0, CLS_ATTN = 1, CLS_LN = 2, CLS_MOTION = 3, CLS_GEMM_F32 = 4, CLS_SETUP = 5,
                    NUM_CLS = 8 };
 
@@ -66,6 +69,10 @@ struct NetW {
   float* txt_b = nullptr; float* t_b1 = nullptr; float* t_b2 = nullptr; float* in_b = nullptr; float* out_b = nullptr;
   float* qkv_b[L] = {}; float* o_b[L] = {}; float* ln1_g[L] = {}; float* ln1_b[L] = {};
   float* ff1_b[L] = {}; float* ff2_b[L] = {}; float* ln2_g[L] = {}; float* ln2_b[L] = {};
+  // folded LayerNorm (bf16 path): the projection after a LayerNorm stores W diag(gamma);
+  // *_g are the row sums of the stored weights, *_h = W beta + b (null when not folded)
+  float* qkv_g[L] = {}; float* qkv_h[L] = {}; float* ff1_g[L] = {}; float* ff1_h[L] = {};
+  float* out_g = nullptr; float* out_h = nullptr;
   int din = 0, dout = 0, in_ld = 0;
 };
 
@@ -79,6 +86,7 @@ struct Workspace {
   int* lengths = nullptr; float* st_text = nullptr; float* st_null = nullptr;
   int* tok0 = nullptr; int* row_seq = nullptr;   // packed token layout (valid tokens only)
   float* stats[2] = {};                           // LayerNorm row statistics (mean, 1/std) [M][2]
+  float2* part = nullptr;                         // folded LayerNorm: chunk statistics [D / 16][M]
 };
 
 // Token rows of a call: the padded layout (every sequence frames + 1 rows) or, when the
@@ -127,6 +135,9 @@ struct kimodo_ctx {
   bool stream_k = false;   // stream-K shares for them instead (KIMODO_STREAM_K=1; measured slower on the layer shapes)
   bool attn_tc = true;     // tcgen05 attention (KIMODO_ATTN_TC=0: the mma.sync kernel)
   bool ln_lite = true;     // LayerNorm writes row statistics, residual epilogues normalise (KIMODO_LN_LITE=0)
+  bool ln_fold = false;    // no LayerNorm launches: residual epilogues write the statistics, the next
+                           // projection folds the normalisation (KIMODO_LN_FOLD=1; measured slower)
+  int* part_cnt = nullptr; // folded LayerNorm: arrival counters per 32-row group (zero between launches)
   float* sk_partial = nullptr;   // stream-K partial accumulators
   int* sk_flags = nullptr;       // stream-K contributor counters (zero between launches)
   bool bf16() const { return precision == KIMODO_BF16; }
@@ -164,9 +175,20 @@ int launch(kimodo_ctx* c, int cls, double flops, double bytes, cudaStream_t st, 
   return KIMODO_OK;
 }
 
-int pick_bn(const kimodo_ctx* c, int M, int N) {
+int pick_bn(const kimodo_ctx* c, int M, int N, int kind, bool out_f32) {
   if (N <= 16) return 16;
   if (N < 1024) return 128;
+  // A few hundred tokens: every tile streams its full K extent of A and B, so the time is
+  // set by the bytes one SM loads; the narrowest tile whose grid still fits in one wave
+  // spreads the weights over the most SMs (the column split leaves each output
+  // element's summation order unchanged).
+  const bool narrow = (!out_f32 && (kind == EPI_BIAS || kind == EPI_BIAS_GELU)) ||
+                      (out_f32 && (kind == EPI_BIAS_RESID || kind == EPI_BIAS_RESID_LN));
+  if (narrow) {
+    const long mt = (M + 127) / 128;
+    for (int bn : {32, 64, 128})
+      if (mt * ((N + bn - 1) / bn) <= c->num_sms) return bn;
+  }
   auto eff = [&](int bn) {
     const long tiles = (long)((M + 127) / 128) * ((N + bn - 1) / bn);
     const long waves = (tiles + c->num_sms - 1) / c->num_sms;
@@ -194,7 +216,7 @@ int gemm(kimodo_ctx* c, const void* A, int lda, const void* W, int ldw, int M, i
       return launch(c, cls_override >= 0 ? cls_override : CLS_GEMM_TC, flops, bytes, st, "gemm_tc2",
                     [&] { return gemm_tc2(g, bn, kind, out_f32, ep, c->derr, st); });
     }
-    const int bn = pick_bn(c, M, N);
+    const int bn = pick_bn(c, M, N, kind, out_f32);
     return launch(c, cls_override >= 0 ? cls_override : CLS_GEMM_TC, flops, bytes, st, "gemm_tc",
                   [&] { return gemm_tc(g, bn, kind, out_f32, ep, c->derr, st, c->num_sms); });
   }
@@ -219,6 +241,41 @@ __global__ void convert_matrix_kernel(const float* __restrict__ src, int rows, i
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
+// LayerNorm (gamma, beta) folded into the projection W [rows, cols] (fp32) that follows
+// it: dst [rows, ld] = bf16(W diag(gamma)), g[j] = sum over k of the stored dst[j][k],
+// h[j] = b[j] + sum over k of W[j][k] beta[k] (double accumulation).  One CTA per row.
+__global__ void fold_layernorm_kernel(const float* __restrict__ W, int cols, const float* __restrict__ gamma,
+                                      const float* __restrict__ beta, const float* __restrict__ b, bf16* dst,
+                                      int ld, float* g, float* h) {
+  const int j = blockIdx.x;
+  double gs = 0.0, hs = 0.0;
+  for (int k = threadIdx.x; k < ld; k += blockDim.x) {
+    bf16 wf = __float2bfloat16_rn(0.f);
+    if (k < cols) {
+      const float w = W[(long)j * cols + k];
+      wf = __float2bfloat16_rn(__fmul_rn(w, gamma[k]));
+      gs += (double)__bfloat162float(wf);
+      hs += (double)w * (double)beta[k];
+    }
+    dst[(long)j * ld + k] = wf;
+  }
+  __shared__ double rg[256], rh[256];
+  rg[threadIdx.x] = gs;
+  rh[threadIdx.x] = hs;
+  __syncthreads();
+  for (int o = 128; o > 0; o >>= 1) {
+    if ((int)threadIdx.x < o) {
+      rg[threadIdx.x] += rg[threadIdx.x + o];
+      rh[threadIdx.x] += rh[threadIdx.x + o];
+    }
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    g[j] = (float)rg[0];
+    h[j] = (float)((double)b[j] + rh[0]);
+  }
+}
+
 // Walks the canonical blob order; in "plan" mode only sizes the arena.
 struct WeightWalker {
   kimodo_ctx* c;
@@ -228,6 +285,28 @@ struct WeightWalker {
   size_t arena_off = 0;
   cudaStream_t st;
   int err = 0;
+  size_t last_matrix = 0;   // blob offset of the latest matrix, and of the latest vector
+  size_t last_vec = 0;
+
+  bool fold() const { return c->bf16() && c->ln_fold; }
+  // arena space for a vector that is not in the blob
+  float* extra(int n) {
+    float* dst = arena ? reinterpret_cast<float*>(arena + arena_off) : nullptr;
+    arena_off += align256((size_t)n * 4);
+    return dst;
+  }
+  // fold the LayerNorm whose gamma / beta sit at blob offsets (go, bo) into the matrix just
+  // walked (rows x cols, stored at dst with row stride ld) and its bias (blob offset bias_off)
+  void fold_into(void* dst, int rows, int cols, int ld, size_t go, size_t bo, size_t bias_off, float** g,
+                 float** h) {
+    *g = extra(rows);
+    *h = extra(rows);
+    if (arena && !err) {
+      fold_layernorm_kernel<<<rows, 256, 0, st>>>(src + last_matrix, cols, src + go, src + bo, src + bias_off,
+                                                  static_cast<bf16*>(dst), ld, *g, *h);
+      if (cudaGetLastError() != cudaSuccess) err = 1;
+    }
+  }
 
   void* matrix(int rows, int cols, int ld) {
     const size_t bytes = align256((size_t)rows * ld * c->elem());
@@ -240,10 +319,12 @@ struct WeightWalker {
       if (cudaGetLastError() != cudaSuccess) err = 1;
     }
     arena_off += bytes;
+    last_matrix = src_off;
     src_off += (size_t)rows * cols;
     return dst;
   }
   float* vec(int n) {
+    last_vec = src_off;
     const size_t bytes = align256((size_t)n * 4);
     float* dst = arena ? reinterpret_cast<float*>(arena + arena_off) : nullptr;
     if (arena && !err && cudaMemcpyAsync(dst, src + src_off, (size_t)n * 4, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
@@ -258,15 +339,22 @@ struct WeightWalker {
     n.t_W1 = matrix(D, D, D); n.t_b1 = vec(D);
     n.t_W2 = matrix(D, D, D); n.t_b2 = vec(D);
     n.in_W = matrix(D, din, in_ld); n.in_b = vec(D);
+    size_t ln_g = 0, ln_b = 0;   // blob offsets of the latest LayerNorm's gamma and beta
     for (int l = 0; l < L; ++l) {
       n.qkv_W[l] = matrix(3 * D, D, D); n.qkv_b[l] = vec(3 * D);
+      if (fold() && l > 0)
+        fold_into(n.qkv_W[l], 3 * D, D, D, ln_g, ln_b, last_vec, &n.qkv_g[l], &n.qkv_h[l]);
       n.o_W[l] = matrix(D, D, D); n.o_b[l] = vec(D);
-      n.ln1_g[l] = vec(D); n.ln1_b[l] = vec(D);
+      n.ln1_g[l] = vec(D); ln_g = last_vec;
+      n.ln1_b[l] = vec(D); ln_b = last_vec;
       n.ff1_W[l] = matrix(F, D, D); n.ff1_b[l] = vec(F);
+      if (fold()) fold_into(n.ff1_W[l], F, D, D, ln_g, ln_b, last_vec, &n.ff1_g[l], &n.ff1_h[l]);
       n.ff2_W[l] = matrix(D, F, F); n.ff2_b[l] = vec(D);
-      n.ln2_g[l] = vec(D); n.ln2_b[l] = vec(D);
+      n.ln2_g[l] = vec(D); ln_g = last_vec;
+      n.ln2_b[l] = vec(D); ln_b = last_vec;
     }
     n.out_W = matrix(dout, D, D); n.out_b = vec(dout);
+    if (fold()) fold_into(n.out_W, dout, D, D, ln_g, ln_b, last_vec, &n.out_g, &n.out_h);
   }
   void all() {
     net(c->net[0], ROOT_F, ROOT_F, ROOT_IN_LD);
@@ -310,7 +398,7 @@ int ensure_workspace(kimodo_ctx* c, int nseq, int frames, int steps) {
       {(void**)&w.lengths, (size_t)NS * 4},                {(void**)&w.st_text, (size_t)NS * DTXT * 4},
       {(void**)&w.st_null, (size_t)NS * DTXT * 4},        {(void**)&w.tok0, (size_t)(NS + 1) * 4},
       {(void**)&w.row_seq, (size_t)R2 * 4},               {(void**)&w.stats[0], (size_t)R2 * 8},
-      {(void**)&w.stats[1], (size_t)R2 * 8}};
+      {(void**)&w.stats[1], (size_t)R2 * 8},              {(void**)&w.part, (size_t)R2 * (D / 16) * 8}};
   for (auto& p : plan) off += align256(p.second);
   void* arena = nullptr;
   cudaError_t err = cudaMalloc(&arena, off);
@@ -391,18 +479,39 @@ int run_net(kimodo_ctx* c, int net, int nseq, int T, int len_mod, const void* A_
   // Row-statistics residual (bf16 path): y keeps the un-normalised sums z;
   // LayerNorm writes only the bf16 operand h and (mean, 1/std) per row, and the next
   // residual epilogue adds gamma (z - mean) / std + beta itself (EPI_BIAS_RESID_LN).
-  const bool lite = c->bf16() && c->ln_lite && !c->stream_k && w.stats[0] != nullptr;
-  if (lite) ln32 = nullptr;
+  // Folded LayerNorm (bf16 path): no LayerNorm launches.  The residual epilogues also write
+  // bf16(y) into h and the row statistics of y (stats[0] after the attention block,
+  // stats[1] after the FFN); the projection that follows a LayerNorm runs on bf16(y)
+  // with W diag(gamma) and normalises in its epilogue.
+  const bool fold = c->bf16() && c->ln_fold && !c->stream_k && w.part != nullptr && n.ff1_g[0] != nullptr &&
+                    (M + 31) / 32 <= PART_GROUPS_MAX;
+  const bool lite = !fold && c->bf16() && c->ln_lite && !c->stream_k && w.stats[0] != nullptr;
+  if (lite || fold) ln32 = nullptr;
   auto resid_epi = [&](EpiParams& e, int which, const float* g, const float* b) {
-    if (!lite || g == nullptr) return EPI_BIAS_RESID;
+    if (fold) {
+      e.part = w.part;
+      e.part_cnt = c->part_cnt;
+      e.stats_out = w.stats[1 - which];
+      e.out16 = static_cast<bf16*>(w.h);
+      e.ldo16 = D;
+    }
+    if ((!lite && !fold) || g == nullptr) return EPI_BIAS_RESID;
     e.ln_stats = w.stats[which];
     e.ln_g = g;
     e.ln_b = b;
     return EPI_BIAS_RESID_LN;
   };
+  // consumer side of a folded LayerNorm whose statistics are in stats[which]
+  auto fold_epi = [&](EpiParams& e, const float* g, const float* h, int which) {
+    if (!fold || g == nullptr) return;
+    e.fold_g = g;
+    e.bias = h;
+    e.ln_stats = w.stats[which];
+  };
   for (int l = 0; l < L; ++l) {
     EpiParams e;
     e.bias = n.qkv_b[l]; e.out = w.qkv; e.ldo = 3 * D; e.N = 3 * D; e.M = M;
+    fold_epi(e, n.qkv_g[l], n.qkv_h[l], 1);
     KD_TRY(gemm(c, w.h, D, n.qkv_W[l], D, M, 3 * D, D, EPI_BIAS, act_f32, e, st));
     const double aflops = packed ? 4.0 * (double)M * S * DH * H : 4.0 * (double)nseq * S * S * DH * H;
     const double abytes = (double)M * 3 * D * eb + (double)M * D * eb;
@@ -430,23 +539,29 @@ int run_net(kimodo_ctx* c, int net, int nseq, int T, int len_mod, const void* A_
     const int ko = resid_epi(eo, 1, l > 0 ? n.ln2_g[l - 1] : nullptr, l > 0 ? n.ln2_b[l - 1] : nullptr);
     KD_TRY(gemm(c, w.attn, D, n.o_W[l], D, M, D, D, ko, true, eo, st));
     const double lnb = lite ? (double)M * D * (4.0 + eb) + (double)M * 8 : (double)M * D * (4.0 + eb + (c->bf16() ? 4.0 : 0.0));
-    KD_TRY(launch(c, CLS_LN, 0, lnb, st, "layernorm", [&] {
-      return layernorm(w.y, w.h, c->bf16(), n.ln1_g[l], n.ln1_b[l], M, st, ln32, lite ? w.stats[0] : nullptr);
-    }));
+    if (!fold) {
+      KD_TRY(launch(c, CLS_LN, 0, lnb, st, "layernorm", [&] {
+        return layernorm(w.y, w.h, c->bf16(), n.ln1_g[l], n.ln1_b[l], M, st, ln32, lite ? w.stats[0] : nullptr);
+      }));
+    }
     EpiParams e1;
     e1.bias = n.ff1_b[l]; e1.out = w.u; e1.ldo = F; e1.N = F; e1.M = M;
+    fold_epi(e1, n.ff1_g[l], n.ff1_h[l], 0);
     KD_TRY(gemm(c, w.h, D, n.ff1_W[l], D, M, F, D, EPI_BIAS_GELU, act_f32, e1, st));
     EpiParams e2;
     e2.bias = n.ff2_b[l]; e2.out = w.y; e2.ldo = D; e2.resid = resid; e2.ldr = D; e2.N = D; e2.M = M;
     const int kf = resid_epi(e2, 0, n.ln1_g[l], n.ln1_b[l]);
     KD_TRY(gemm(c, w.u, F, n.ff2_W[l], F, M, D, F, kf, true, e2, st));
-    KD_TRY(launch(c, CLS_LN, 0, lnb, st, "layernorm", [&] {
-      return layernorm(w.y, w.h, c->bf16(), n.ln2_g[l], n.ln2_b[l], M, st, ln32, lite ? w.stats[1] : nullptr);
-    }));
+    if (!fold) {
+      KD_TRY(launch(c, CLS_LN, 0, lnb, st, "layernorm", [&] {
+        return layernorm(w.y, w.h, c->bf16(), n.ln2_g[l], n.ln2_b[l], M, st, ln32, lite ? w.stats[1] : nullptr);
+      }));
+    }
   }
   EpiParams eo;
   eo.bias = n.out_b; eo.out = hat; eo.ldo = n.dout; eo.lengths = w.lengths; eo.len_mod = len_mod; eo.S = S;
   eo.T = T; eo.N = n.dout; eo.M = M; eo.tok0 = tok0; eo.row_seq = row_seq;
+  fold_epi(eo, n.out_g, n.out_h, 1);
   return gemm(c, w.h, D, n.out_W, D, M, n.dout, D, EPI_OUTPROJ, true, eo, st);
 }
 
@@ -622,6 +737,8 @@ int kimodo_load_weights(kimodo_ctx** out_ctx, const float* host_blob, size_t n_f
   if (const char* ev = getenv("KIMODO_STREAM_K")) c->stream_k = ev[0] != '0';
   if (const char* ev = getenv("KIMODO_ATTN_TC")) c->attn_tc = ev[0] != '0';
   if (const char* ev = getenv("KIMODO_LN_LITE")) c->ln_lite = ev[0] != '0';
+  if (const char* ev = getenv("KIMODO_LN_FOLD")) c->ln_fold = ev[0] != '0';
+  if (precision != KIMODO_BF16) c->ln_fold = false;
   c->num_sms = prop.multiProcessorCount;
   auto fail = [&](int code) {
     kimodo_free(c);
@@ -667,6 +784,9 @@ int kimodo_load_weights(kimodo_ctx** out_ctx, const float* host_blob, size_t n_f
         cudaMalloc(&c->sk_flags, 2 * GEMM_SK_MAX_PAIRS * sizeof(int)) != cudaSuccess)
       return fail(set_error(KIMODO_ENOMEM, "stream-K workspace"));
     cudaMemset(c->sk_flags, 0, 2 * GEMM_SK_MAX_PAIRS * sizeof(int));
+    if (cudaMalloc(&c->part_cnt, PART_GROUPS_MAX * sizeof(int)) != cudaSuccess)
+      return fail(set_error(KIMODO_ENOMEM, "LayerNorm statistics counters"));
+    cudaMemset(c->part_cnt, 0, PART_GROUPS_MAX * sizeof(int));
   }
 
   // weights: plan the arena, stage the fp32 blob on the device, convert
@@ -703,6 +823,7 @@ void kimodo_free(kimodo_ctx* c) {
   if (c->zbuf) cudaFree(c->zbuf);
   if (c->sk_partial) cudaFree(c->sk_partial);
   if (c->sk_flags) cudaFree(c->sk_flags);
+  if (c->part_cnt) cudaFree(c->part_cnt);
   if (c->warena) cudaFree(c->warena);
   if (c->pe) cudaFree(c->pe);
   if (c->derr) cudaFree(c->derr);
@@ -941,8 +1062,10 @@ int kimodo_sync_status(kimodo_ctx* c, void* stream) {
   KD_CUDA(cudaMemcpy(&h, c->derr, sizeof(h), cudaMemcpyDeviceToHost));
   if (h.code != 0) {
     KD_CUDA(cudaMemset(c->derr, 0, sizeof(DevError)));
-    // an interrupted stream-K launch may leave contributor counters raised
+    // an interrupted stream-K launch may leave contributor counters raised, and an interrupted
+    // residual GEMM its LayerNorm-statistics arrival counters
     KD_CUDA(cudaMemset(c->sk_flags, 0, 2 * GEMM_SK_MAX_PAIRS * sizeof(int)));
+    KD_CUDA(cudaMemset(c->part_cnt, 0, PART_GROUPS_MAX * sizeof(int)));
     return set_error(h.code, "device wait timed out in kernel stage %d (block %d)", h.where, h.block);
   }
   return KIMODO_OK;
@@ -1040,9 +1163,12 @@ int kimodo_gemm_bf16(const void* A, int lda, const void* W, int ldw, const float
     return set_error(KIMODO_EINVAL, "out, resid and bias need 16-byte alignment and ldo, ldr multiples of 4");
   if (epilogue == 3 && !out_f32) return set_error(KIMODO_EINVAL, "residual epilogue writes fp32");
   if ((epilogue == 1 || epilogue == 2) && out_f32) return set_error(KIMODO_EINVAL, "GELU/SiLU epilogues write bf16");
-  if (tile_n != 0 && tile_n != 128 && tile_n != 256) return set_error(KIMODO_EINVAL, "tile_n must be 0, 128 or 256");
+  if (tile_n != 0 && tile_n != 32 && tile_n != 64 && tile_n != 128 && tile_n != 256)
+    return set_error(KIMODO_EINVAL, "tile_n must be 0, 32, 64, 128 or 256");
   if (tile_n == 256 && (epilogue == KIMODO_EPI_BIAS_SILU || (out_f32 && epilogue == KIMODO_EPI_BIAS)))
     return set_error(KIMODO_EINVAL, "tile_n 256 is not built for this epilogue");
+  if ((tile_n == 32 || tile_n == 64) && (epilogue == KIMODO_EPI_BIAS_SILU || (out_f32 && epilogue == KIMODO_EPI_BIAS)))
+    return set_error(KIMODO_EINVAL, "tile_n 32 and 64 are not built for this epilogue");
   KD_TRY(prepared_device());
   int dev = 0, sms = 148;
   KD_CUDA(cudaGetDevice(&dev));
@@ -1216,6 +1342,7 @@ constexpr size_t noalloc_layout(char* base, size_t e, size_t rows, size_t nseq, 
   char* stt = take(nseq * DTXT * 4);
   char* st0 = take(rows * 8);
   char* st1 = take(rows * 8);
+  char* prt = take(rows * (D / 16) * 8);
   if (w) {
     w->h = h; w->qkv = qkv; w->attn = attn; w->u = u; w->y = reinterpret_cast<float*>(y);
     w->A_root = ar; w->A_body = ab;
@@ -1226,6 +1353,7 @@ constexpr size_t noalloc_layout(char* base, size_t e, size_t rows, size_t nseq, 
     w->tmlp[0] = reinterpret_cast<float*>(tm0); w->tmlp[1] = reinterpret_cast<float*>(tm1);
     w->lengths = reinterpret_cast<int*>(len); w->st_text = reinterpret_cast<float*>(stt); w->st_null = nullptr;
     w->stats[0] = reinterpret_cast<float*>(st0); w->stats[1] = reinterpret_cast<float*>(st1);
+    w->part = reinterpret_cast<float2*>(prt);
   }
   return off;
 }

@@ -205,6 +205,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     constexpr int CW = C::CW;
     constexpr int PASSES = EpiLanes<CW>::PASSES;
     float* st = epi_smem + (warp - 2) * 32 * (CW + 4);
+    // folded LayerNorm statistics produced by the residual epilogues
+    const bool stats = (KIND == EPI_BIAS_RESID || KIND == EPI_BIAS_RESID_LN) && ep.part != nullptr;
     int local = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++local) {
       const int acc = local & 1;
@@ -226,6 +228,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         ptx::tc_fence_before();
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive(tempty_bar(acc));
+        if (stats) part_arrive(ep, m_blk * BM + quarter * 32, lane);
         continue;
       }
       // two register buffers: the TMEM load and global prefetch of chunk c + 1 are in
@@ -268,6 +271,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         }
         process(vb, pb, bb, c + 1);
       }
+      if (stats) part_arrive(ep, m_blk * BM + quarter * 32, lane);
     }
   }
 
@@ -313,7 +317,9 @@ cudaError_t launch_impl(const GemmArgs& g, const EpiParams& ep, DevError* err, c
   const int tiles = mt * nt;
   const int grid = tiles < num_sms ? tiles : num_sms;
   const int kb = (g.K + BK - 1) / BK;
-  return launch_kernel(kern, dim3(grid), dim3(NUM_THREADS), Cf::SMEM, st, ta, tb, mt, nt, kb, ep, err);
+  EpiParams e = ep;
+  e.part_arrivals = EPI_PARTS * nt;   // every epilogue warp of a lane quarter, for every column tile
+  return launch_kernel(kern, dim3(grid), dim3(NUM_THREADS), Cf::SMEM, st, ta, tb, mt, nt, kb, e, err);
 }
 
 }  // namespace
@@ -381,6 +387,14 @@ static cudaError_t dispatch(const GemmArgs& g, int bn, int kind, bool out_f32, c
   KD_TC(128, 6, EPI_BIAS_RESID_LN, float)
   KD_TC(128, 6, EPI_INPROJ, bf16)
   KD_TC(128, 6, EPI_OUTPROJ, float)
+  KD_TC(64, 8, EPI_BIAS, bf16)
+  KD_TC(64, 8, EPI_BIAS_GELU, bf16)
+  KD_TC(64, 8, EPI_BIAS_RESID, float)
+  KD_TC(64, 8, EPI_BIAS_RESID_LN, float)
+  KD_TC(32, 8, EPI_BIAS, bf16)
+  KD_TC(32, 8, EPI_BIAS_GELU, bf16)
+  KD_TC(32, 8, EPI_BIAS_RESID, float)
+  KD_TC(32, 8, EPI_BIAS_RESID_LN, float)
   KD_TC(16, 8, EPI_OUTPROJ, float)
 #undef KD_TC
   return prep ? cudaSuccess : cudaErrorInvalidValue;

@@ -229,6 +229,10 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
     int cc = 0;   // chunks processed by this warp so far: staging tile cc & 1
     int local = 0;
     bool failed = false;
+    // folded LayerNorm: the bias / GELU epilogues consume it, the residual ones produce it
+    constexpr bool FOLDABLE = KIND == EPI_BIAS || KIND == EPI_BIAS_GELU;
+    const bool fold = FOLDABLE && ep.fold_g != nullptr;
+    const bool stats = C::RES && ep.part != nullptr;
     for (int tile = pair; tile < num_tiles && !failed; tile += npairs, ++local) {
       const int acc = local & 1;
       const uint32_t acc_phase = (local >> 1) & 1;
@@ -244,7 +248,8 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
       const int cc0 = cc;
       auto stage_tile = [&](int a) { return stg_base + (a % C::NBUF) * C::STG_BYTES; };
       // per-column operands of chunk k: bias, and for EPI_BIAS_RESID_LN the LayerNorm gamma and
-      // (bias + beta), so that x = acc + (bias + beta) + (z * rstd - mean * rstd) * gamma
+      // (bias + beta), so that x = acc + (bias + beta) + (z * rstd - mean * rstd) * gamma; with
+      // a folded LayerNorm (fold) the row sums of the folded weights
       auto load_bias = [&](int k, float4 (&b4)[CW / 4], float4 (&g4)[CW / 4]) {
 #pragma unroll
         for (int j = 0; j < CW / 4; ++j) {
@@ -254,11 +259,15 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
             b4[j].x += be.x; b4[j].y += be.y; b4[j].z += be.z; b4[j].w += be.w;
             g4[j] = ld4(ep.ln_g + gcol + k * CW + 4 * j);
           }
+          if constexpr (FOLDABLE) {
+            if (fold) g4[j] = ld4(ep.fold_g + gcol + k * CW + 4 * j);
+          }
         }
       };
-      // this lane's row statistics for EPI_BIAS_RESID_LN: z * rs_a + rs_b = (z - mean) / std
+      // this lane's row statistics for EPI_BIAS_RESID_LN and a folded LayerNorm:
+      // z * rs_a + rs_b = (z - mean) / std
       float rs_a = 1.f, rs_b = 0.f;
-      if constexpr (KIND == EPI_BIAS_RESID_LN) {
+      if (KIND == EPI_BIAS_RESID_LN || fold) {
         const int row = row0 + lane;
         if (nch > 0 && row < ep.M) {
           const float2 st2 = *reinterpret_cast<const float2*>(ep.ln_stats + 2 * (long)row);
@@ -294,6 +303,7 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
       };
       if (nch == 0) {
         release();
+        if (stats) part_arrive(ep, row0, lane);
         continue;
       }
       // finish chunk k (the warp's chunk number cc == cc0 + k) from accumulator values v, bias b4
@@ -304,12 +314,23 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
         uint8_t* srow = st + lane * C::ROW_BYTES;
         const int swz = C::ROW_BYTES == 64 ? (lane >> 1) & 3 : (lane >> 2) & 1;
         float x[CW];
+        if (FOLDABLE && fold) {
+          // folded LayerNorm: acc / std - (mean / std) g + (W beta + b)
 #pragma unroll
-        for (int j = 0; j < CW / 4; ++j) {
-          x[4 * j] = v[4 * j] + b4[j].x;
-          x[4 * j + 1] = v[4 * j + 1] + b4[j].y;
-          x[4 * j + 2] = v[4 * j + 2] + b4[j].z;
-          x[4 * j + 3] = v[4 * j + 3] + b4[j].w;
+          for (int j = 0; j < CW / 4; ++j) {
+            x[4 * j] = fmaf(v[4 * j], rs_a, fmaf(rs_b, g4[j].x, b4[j].x));
+            x[4 * j + 1] = fmaf(v[4 * j + 1], rs_a, fmaf(rs_b, g4[j].y, b4[j].y));
+            x[4 * j + 2] = fmaf(v[4 * j + 2], rs_a, fmaf(rs_b, g4[j].z, b4[j].z));
+            x[4 * j + 3] = fmaf(v[4 * j + 3], rs_a, fmaf(rs_b, g4[j].w, b4[j].w));
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < CW / 4; ++j) {
+            x[4 * j] = v[4 * j] + b4[j].x;
+            x[4 * j + 1] = v[4 * j + 1] + b4[j].y;
+            x[4 * j + 2] = v[4 * j + 2] + b4[j].z;
+            x[4 * j + 3] = v[4 * j + 3] + b4[j].w;
+          }
         }
         if constexpr (KIND == EPI_BIAS_GELU) {
 #pragma unroll
@@ -330,6 +351,19 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
               r.z = fmaf(r.z, rs_a, rs_b) * g4[u].z; r.w = fmaf(r.w, rs_a, rs_b) * g4[u].w;
             }
             x[4 * u] += r.x; x[4 * u + 1] += r.y; x[4 * u + 2] += r.z; x[4 * u + 3] += r.w;
+          }
+          if (stats) {
+            // the new sum's bf16 copy (the next GEMM's operand) and its chunk statistics
+            const int row = row0 + lane;
+            if (row < ep.M) {
+              const int col = gcol + k * CW;
+              ep.part[(long)(col >> 4) * ep.M + row] = chunk_stats16(x);
+              uint4* o16 = reinterpret_cast<uint4*>(ep.out16 + (long)row * ep.ldo16 + col);
+              o16[0] = make_uint4(bf16x2_bits(x[0], x[1]), bf16x2_bits(x[2], x[3]), bf16x2_bits(x[4], x[5]),
+                                  bf16x2_bits(x[6], x[7]));
+              o16[1] = make_uint4(bf16x2_bits(x[8], x[9]), bf16x2_bits(x[10], x[11]), bf16x2_bits(x[12], x[13]),
+                                  bf16x2_bits(x[14], x[15]));
+            }
           }
         } else {
           if (lane == 0) ptx::bulk_wait_read<1>();   // store of chunk cc - 2 has read this tile
@@ -377,6 +411,7 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
         if (!process(vb, bb, gb, c + 1)) { failed = true; break; }
       }
       if (failed && !*abort) record_timeout(err, WHERE_GEMM_EPILOGUE, abort);
+      if (stats && !failed) part_arrive(ep, row0, lane);
     }
     if (lane == 0) ptx::bulk_wait_all();
     __syncwarp();
@@ -455,8 +490,10 @@ struct Tc2Launcher {
     cfg.stream = st;
     cfg.attrs = attr;
     cfg.numAttrs = pdl_enabled() ? 2 : 1;
+    EpiParams e = ep;
+    e.part_arrivals = 2 * nt;   // both epilogue warps of a lane quarter, for every column tile
     return cudaLaunchKernelEx(&cfg, gemm_tc2_kernel<BN, STAGES, KIND, OutT>, ta, tb, to, tr, mt, nt,
-                              (g.K + BK - 1) / BK, ep, err);
+                              (g.K + BK - 1) / BK, e, err);
   }
 };
 template <int BN, int STAGES, int KIND, typename OutT>
