@@ -426,7 +426,9 @@ __device__ __forceinline__ void epilogue_prefetch(const EpiParams& e, int row0, 
   }
 }
 
-template <int KIND, typename OutT, int CW>
+// FOLD: the folded-LayerNorm form (bias / GELU / output projection consume the row
+// statistics, the residual kinds produce them).
+template <int KIND, typename OutT, int CW, bool FOLD = false>
 __device__ __forceinline__ void epilogue_warp_tile(const EpiParams& e, const float* st, int row0, int col0,
                                                    int lane, const float4 (&pre)[EpiLanes<CW>::PASSES],
                                                    const float4 bias4) {
@@ -451,7 +453,7 @@ __device__ __forceinline__ void epilogue_warp_tile(const EpiParams& e, const flo
         const int frame = pos - 1;
         const bool valid = frame < e.lengths[seq % e.len_mod];
         OutT* o = reinterpret_cast<OutT*>(e.out) + ((long)seq * e.T + frame) * e.ldo + col;
-        if (e.fold_g != nullptr) {
+        if constexpr (FOLD) {
           // folded LayerNorm: acc / std - (mean / std) g + (W beta + b)
           const float2 st2 = *reinterpret_cast<const float2*>(e.ln_stats + 2 * (long)row);
           const float ra = st2.y, rb = -st2.x * st2.y;
@@ -480,7 +482,7 @@ __device__ __forceinline__ void epilogue_warp_tile(const EpiParams& e, const flo
         }
         if (in_rows && e.out32 != nullptr) store4<float>(e.out32 + (long)row * e.ldo + col, v[0], v[1], v[2], v[3]);
       } else {
-        if ((KIND == EPI_BIAS || KIND == EPI_BIAS_GELU) && e.fold_g != nullptr) {
+        if constexpr ((KIND == EPI_BIAS || KIND == EPI_BIAS_GELU) && FOLD) {
           // folded LayerNorm: acc / std - (mean / std) g + (W beta + b), as the pair GEMM forms it
           const float2 st2 = *reinterpret_cast<const float2*>(e.ln_stats + 2 * (long)min(row, e.M - 1));
           const float ra = st2.y, rb = -st2.x * st2.y;
@@ -517,7 +519,7 @@ __device__ __forceinline__ void epilogue_warp_tile(const EpiParams& e, const flo
           v[2] += fmaf(pre[p].z, ra, rb) * g4.z; v[3] += fmaf(pre[p].w, ra, rb) * g4.w;
         }
         if constexpr (KIND == EPI_BIAS_RESID || KIND == EPI_BIAS_RESID_LN) {
-          if (e.part != nullptr) {
+          if constexpr (FOLD) {
             // folded LayerNorm producer: chunk statistics of the new sum (the four lanes of
             // this row hold its 16 columns; N % 16 == 0, so every lane is here) and its bf16 copy
             static_assert(CW == 16, "four lanes per 16-column chunk");
