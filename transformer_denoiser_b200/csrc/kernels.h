@@ -16,8 +16,9 @@ struct GemmArgs {
   int lda = 0, ldb = 0;
 };
 
-// tcgen05 bf16 GEMM.  bn in {16, 128, 256}; returns cudaErrorInvalidValue for an
-// unsupported (bn, kind, output type) combination.
+// tcgen05 bf16 GEMM.  bn in {16, 32, 64, 128, 256}; returns cudaErrorInvalidValue for an
+// unsupported (bn, kind, output type) combination.  A launch whose EpiParams carry
+// folded-LayerNorm row statistics (fold_g or part set) runs the folded instantiation.
 cudaError_t gemm_tc(const GemmArgs& g, int bn, int kind, bool out_f32, const EpiParams& ep, DevError* err,
                     cudaStream_t st, int num_sms);
 bool gemm_tc_available();
@@ -42,7 +43,8 @@ cudaError_t gemm_sk(const GemmArgs& g, int kind, bool out_f32, const EpiParams& 
                     DevError* err, cudaStream_t st);
 
 // tcgen05 GEMM on CTA pairs (256-row tiles).  bn in {144, 160, 208, 256} for EPI_BIAS /
-// EPI_BIAS_GELU with bf16 output, {144, 160} for EPI_BIAS_RESID with fp32 output.
+// EPI_BIAS_GELU with bf16 output, {144, 160} for EPI_BIAS_RESID / EPI_BIAS_RESID_LN with
+// fp32 output; folded-LayerNorm launches as for gemm_tc.
 cudaError_t gemm_tc2(const GemmArgs& g, int bn, int kind, bool out_f32, const EpiParams& ep, DevError* err,
                      cudaStream_t st);
 cudaError_t gemm_tc2_prepare();
