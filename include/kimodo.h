@@ -81,6 +81,16 @@ enum { KIMODO_NET_ROOT = 0, KIMODO_NET_BODY = 1 };
  * precision: KIMODO_BF16 (tensor-core path: bf16 operands, fp32 accumulation,
  *   fp32 LayerNorm/softmax/DDIM) or KIMODO_FP32 (fp32 everywhere).
  * On success *ctx receives a context owned by the caller (kimodo_free).
+ *
+ * Kernel choices, read from the environment when the context is created (bf16 path;
+ * every choice computes the same function, within the bf16 tolerances):
+ *   KIMODO_PAIR_GEMM=0  single-CTA GEMM tiles instead of CTA-pair tiles at >= 1024 tokens;
+ *   KIMODO_STREAM_K=1   stream-K work sharing for the layer projections;
+ *   KIMODO_ATTN_TC=0    the mma.sync attention kernel instead of the tcgen05 one;
+ *   KIMODO_LN_LITE=0    LayerNorm rewrites the fp32 residual stream (no row statistics);
+ *   KIMODO_LN_FOLD=1    no LayerNorm launches: the residual GEMM epilogues produce the
+ *                       row statistics and the next projection folds the normalisation
+ *                       (the weights are folded at load; measured slower, off by default).
  */
 KIMODO_API int kimodo_load_weights(kimodo_ctx** ctx, const float* host_blob, size_t n_floats,
                         int precision, int device);
