@@ -168,6 +168,32 @@ def _ncu_traffic():
         return None
 
 
+# Algorithmic work of one denoiser step (both networks; projections per token per
+# network forward, activation bytes per token per layer: QKV 8192, attention 8192,
+# attention output 10240, FFN1 6144, FFN2 12288, two LayerNorms 6144 each).
+PROJ_FLOP_PER_TOKEN = 268435456
+ACT_BYTES_PER_TOKEN_LAYER = 57344
+WEIGHT_BYTES_PER_STEP = 2 * 16 * 8388608 * 2
+
+
+def step_roofline(nseq, tokens_per_seq, ms_per_step):
+    """Roofline of one DDIM step of the two-stage denoiser at nseq sequences (cond and
+    uncond counted) of tokens_per_seq tokens: the slower of its FLOPs at the measured
+    burst bf16 peak and its weight-plus-activation bytes at the measured HBM peak, and
+    the fraction of it that ms_per_step achieves."""
+    peaks, kind = _measured_peaks()
+    tokens = nseq * tokens_per_seq
+    flops = 2 * (tokens * PROJ_FLOP_PER_TOKEN + 16 * nseq * 4 * tokens_per_seq ** 2 * 1024)
+    nbytes = WEIGHT_BYTES_PER_STEP + 2 * 16 * ACT_BYTES_PER_TOKEN_LAYER * tokens
+    t_flop = flops / (float(peaks["bf16_tflops"]) * 1e12)
+    t_byte = nbytes / (float(peaks["hbm_gbs"]) * 1e9)
+    floor = max(t_flop, t_byte)
+    return {"bound": "tensor" if t_flop >= t_byte else "hbm", "floor_us": round(floor * 1e6, 2),
+            "flop": flops, "bytes": nbytes, "achieved_us": round(ms_per_step * 1e3, 2),
+            "frac": round(floor / (ms_per_step * 1e-3), 4),
+            "peaks": f"{kind} burst bf16 {peaks['bf16_tflops']} TFLOP/s, HBM {peaks['hbm_gbs']} GB/s"}
+
+
 def roofline(prof):
     peaks, kind = _measured_peaks()
     g = prof["gemm_tc"]
@@ -262,7 +288,8 @@ def secondary_workloads(model, dev, flush, reps=3):
     d_len = torch.from_numpy(lengths).to(dev)
     padded_ms = timed(lambda: model.ddim_sample(emb, null, noise, d_len, 50, 2.5))
     valid_tokens = 2 * 2 * int((lengths + 1).sum()) * 50
-    return {"c3_latency": {"workload": "50-step DDIM, 1 prompt x 180 frames, CFG 2.0", "ms": round(c3_ms, 3)},
+    return {"c3_latency": {"workload": "50-step DDIM, 1 prompt x 180 frames, CFG 2.0", "ms": round(c3_ms, 3),
+                           "step_roofline": step_roofline(2, 181, c3_ms / 50)},
             "c5_ragged": {"workload": "50-step DDIM, 64 prompts, lengths U{60..300} padded to 300 frames, CFG 2.5",
                           "clips_per_min_packed": round(B * 60e3 / packed_ms, 2),
                           "clips_per_min_padded": round(B * 60e3 / padded_ms, 2),

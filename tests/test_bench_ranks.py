@@ -68,3 +68,21 @@ def test_whole_job_throughput_scales_with_ranks(n):
     per_rank = bench.clips_per_min(1, 10, 5.0)
     assert bench.clips_per_min(n, 10, 5.0) == pytest.approx(n * per_rank)
     assert bench.workload_config(n)["global_batch"] == n * bench.WORKLOAD["batch"]
+
+
+def test_step_roofline_counts():
+    """One prompt with CFG at 180 frames: 2 x 181 tokens per network forward."""
+    r = bench.step_roofline(2, 181, 1.0)
+    tokens = 2 * 181
+    # projections: QKV 3, O 1, FFN 2 + 2 (x 1024^2 MACs) per token, 16 layers, 2 FLOP per MAC
+    assert bench.PROJ_FLOP_PER_TOKEN == 16 * 2 * (3 + 1 + 2 + 2) * 1024 * 1024
+    # attention per sequence and layer: QK^T and PV, 2 x 2 x S^2 x 1024 FLOP
+    assert r["flop"] == 2 * (tokens * bench.PROJ_FLOP_PER_TOKEN + 16 * 2 * 4 * 181 * 181 * 1024)
+    assert r["bytes"] == 2 * 16 * (8 * 1024 * 1024) * 2 + 2 * 16 * 57344 * tokens
+    peaks, _ = bench._measured_peaks()
+    t_flop = r["flop"] / (float(peaks["bf16_tflops"]) * 1e12)
+    t_byte = r["bytes"] / (float(peaks["hbm_gbs"]) * 1e9)
+    assert r["floor_us"] == round(max(t_flop, t_byte) * 1e6, 2)
+    assert r["bound"] == ("tensor" if t_flop >= t_byte else "hbm")
+    assert r["frac"] == round(max(t_flop, t_byte) / 1e-3, 4)
+    assert abs(bench.step_roofline(2, 181, 2.0)["frac"] - r["frac"] / 2) < 1e-4
