@@ -74,6 +74,13 @@ def test_kernel_entry_argument_checks(lib):
     assert lib.kimodo_gemm_bf16(p, 60, p, 64, p, None, 0, p, 64, 1, 1, 60, 0, 0, 0, None) == -1
     assert lib.kimodo_gemm_bf16(p, 64, p, 64, p, None, 0, p, 64, 1, 1, 64, 3, 1, 0, None) == -1  # resid missing
     assert lib.kimodo_gemm_f32(p, 64, p, 64, p, None, 0, p, 64, 1, 1, 40, 0, None) == -1       # K % 16
+    # output tiles: 32, 64, 128, 256 or 0; the narrow ones exist for bias / GELU (bf16) and residual only
+    assert lib.kimodo_gemm_bf16(p, 64, p, 64, p, None, 0, p, 64, 1, 64, 64, 0, 0, 48, None) == -1
+    assert b"tile_n must be" in lib.kimodo_last_error()
+    assert lib.kimodo_gemm_bf16(p, 64, p, 64, p, None, 0, p, 64, 1, 64, 64, 2, 0, 32, None) == -1  # SiLU
+    assert b"not built" in lib.kimodo_last_error()
+    assert lib.kimodo_gemm_bf16(p, 64, p, 64, p, None, 0, p, 64, 1, 64, 64, 0, 1, 64, None) == -1  # fp32 bias
+    assert b"not built" in lib.kimodo_last_error()
     assert lib.kimodo_attention_bf16(p, p, p, 1, 302, None) == -1
     assert lib.kimodo_layernorm(p, p, 1, p, p, 0, None) == -1
 
