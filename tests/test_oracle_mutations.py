@@ -149,3 +149,38 @@ def test_timestep_rounding_down_is_caught(monkeypatch):
         return [(ts[k], ts[k + 1] if k + 1 < steps else -1) for k in range(steps)]
     monkeypatch.setattr(ko, "ddim_timesteps_trailing", floor_only)
     _expect_fail(pins.test_trailing_timesteps_any_count)
+
+
+def test_sinusoid_sin_cos_swapped_is_caught(monkeypatch):
+    def swapped(positions, d):
+        p = np.asarray(positions, dtype=np.float64).reshape(-1, 1)
+        w = np.power(10000.0, -2.0 * np.arange(d // 2, dtype=np.float64) / d)
+        out = np.empty((p.shape[0], d))
+        out[:, 0::2] = np.cos(p * w)
+        out[:, 1::2] = np.sin(p * w)
+        return out
+    monkeypatch.setattr(ko, "sinusoid", swapped)
+    _expect_fail(pins.test_sinusoid_closed_forms)
+
+
+def test_timestep_mlp_without_silu_is_caught(monkeypatch):
+    def no_silu(net, t):
+        e = ko.sinusoid([t], net["t_W1"].shape[1])[0]
+        return ko.linear(ko.linear(e, net["t_W1"], net["t_b1"]), net["t_W2"], net["t_b2"])
+    monkeypatch.setattr(ko, "timestep_mlp", no_silu)
+    _expect_fail(pins.test_denoiser_forward_vs_torch_modules, "root")
+
+
+def test_condition_without_timestep_is_caught(monkeypatch):
+    monkeypatch.setattr(ko, "condition_vector",
+                        lambda net, emb, t: ko.linear(np.asarray(emb, np.float64), net["txt_W"], net["txt_b"]))
+    _expect_fail(pins.test_denoiser_forward_vs_torch_modules, "body")
+
+
+def test_condition_key_masked_out_is_caught(monkeypatch):
+    real = ko.attention
+
+    def skip_condition_key(q, k, v, n):
+        return real(q, k[1:], v[1:], n - 1) if n > 1 else real(q, k, v, n)
+    monkeypatch.setattr(ko, "attention", skip_condition_key)
+    _expect_fail(pins.test_attention_brute_force, 5, 5)
