@@ -81,16 +81,6 @@ enum { KIMODO_NET_ROOT = 0, KIMODO_NET_BODY = 1 };
  * precision: KIMODO_BF16 (tensor-core path: bf16 operands, fp32 accumulation,
  *   fp32 LayerNorm/softmax/DDIM) or KIMODO_FP32 (fp32 everywhere).
  * On success *ctx receives a context owned by the caller (kimodo_free).
- *
- * Kernel choices, read from the environment when the context is created (bf16 path;
- * every choice computes the same function, within the bf16 tolerances):
- *   KIMODO_PAIR_GEMM=0  single-CTA GEMM tiles instead of CTA-pair tiles at >= 1024 tokens;
- *   KIMODO_STREAM_K=1   stream-K work sharing for the layer projections;
- *   KIMODO_ATTN_TC=0    the mma.sync attention kernel instead of the tcgen05 one;
- *   KIMODO_LN_LITE=0    LayerNorm rewrites the fp32 residual stream (no row statistics);
- *   KIMODO_LN_FOLD=1    no LayerNorm launches: the residual GEMM epilogues produce the
- *                       row statistics and the next projection folds the normalisation
- *                       (the weights are folded at load; measured slower, off by default).
  */
 KIMODO_API int kimodo_load_weights(kimodo_ctx** ctx, const float* host_blob, size_t n_floats,
                         int precision, int device);
@@ -122,14 +112,19 @@ KIMODO_API int kimodo_denoiser_forward(kimodo_ctx* ctx, int net, const float* x,
  * routine.  The context itself is created, with its weights, by
  * kimodo_load_weights.
  *
- * Arguments, layouts and results are those of kimodo_denoiser_forward, within
- * these limits: batch <= 16 and batch * (frames + 1) <= 512 tokens, else
- * KIMODO_EINVAL (use kimodo_denoiser_forward for larger calls).
- * The first call on a device looks up the array's device address (set-up); make
- * that first call before any stream capture.  Every call on a device shares the
- * one array and overwrites the previous call's contents: calls whose work can
- * overlap on the GPU (other streams, other contexts, other threads) race and
- * must be ordered by the caller.
+ * Arguments and output layout are those of kimodo_denoiser_forward, within these
+ * limits: batch <= 16 and batch * (frames + 1) <= 512 tokens, else KIMODO_EINVAL
+ * (use kimodo_denoiser_forward for larger calls).  The scratch always holds the
+ * padded token layout (every sequence frames + 1 rows, padded rows computed and
+ * discarded), where kimodo_denoiser_forward packs the valid tokens when host lengths
+ * are shorter than frames; the results agree within the path's tolerances (bf16:
+ * relative L2 2e-2; fp32: max-abs relative 1e-4), not necessarily bit for bit.
+ * The first call on a device looks up the array's device address (set-up, cached per
+ * device for the life of the process; a cudaDeviceReset invalidates it together with
+ * every context); make that first call before any stream capture.  Every call on a
+ * device shares the one array and overwrites the previous call's contents: calls
+ * whose work can overlap on the GPU (other streams, other contexts, other threads)
+ * race and must be ordered by the caller.
  */
 KIMODO_API int kimodo_denoiser_forward_noalloc(kimodo_ctx* ctx, int net, const float* x, const float* emb,
                                                int t, const int* lengths, int batch, int frames,

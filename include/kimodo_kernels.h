@@ -55,18 +55,6 @@ KIMODO_API int kimodo_gemm_bf16_pair(const void* A, int lda, const void* W, int 
                                      const void* resid, int ldr, void* out, int ldo, int M, int N, int K,
                                      int epilogue, int out_f32, int tile_n, void* stream);
 
-/*
- * The same product with stream-K work sharing (the denoiser's kernel for its large
- * projections): 256 x 256 pair tiles, every SM pair takes an equal contiguous share
- * of the (tile, 64-deep k-block) units; a tile split between pairs is summed in fp32
- * by the pair that holds its last k-block.  Arguments and epilogues as
- * kimodo_gemm_bf16_pair (no tile choice).  The call allocates and frees its
- * partial-sum workspace in stream order (cudaMallocAsync on `stream`).
- */
-KIMODO_API int kimodo_gemm_bf16_streamk(const void* A, int lda, const void* W, int ldw, const float* bias,
-                                        const void* resid, int ldr, void* out, int ldo, int M, int N, int K,
-                                        int epilogue, int out_f32, void* stream);
-
 /* fp32 SIMT GEMM with the same epilogues; all operands fp32; K % 16 == 0,
  * lda, ldw multiples of 4. */
 KIMODO_API int kimodo_gemm_f32(const float* A, int lda, const float* W, int ldw, const float* bias,
@@ -79,19 +67,16 @@ KIMODO_API int kimodo_gemm_f32(const float* A, int lda, const float* W, int ldw,
  * qkv: [nseq * S, 3072] with columns Q | K | V (head h at h * 128 inside each).
  * Sequence s attends to keys 0 .. lengths[s] (the condition token plus
  * lengths[s] frames; clamped to [1, S] keys).  out: [nseq * S, 1024].
- * bf16 variant: bf16 qkv/out, fp32 softmax; f32 variant: fp32 throughout.
  * 1 <= S <= 301.
+ * bf16 variant: bf16 qkv/out (qkv 16-byte aligned), on the tcgen05 tensor cores:
+ *   one CTA per (head, sequence, 128-query tile), S = Q K^T and O = P V in TMEM,
+ *   exact fp32 softmax over all keys of a sequence.
+ * f32 variant: fp32 throughout (SIMT, one warp per query).
  */
 KIMODO_API int kimodo_attention_bf16(const void* qkv, void* out, const int* lengths, int nseq, int S,
                                      void* stream);
 KIMODO_API int kimodo_attention_f32(const float* qkv, float* out, const int* lengths, int nseq, int S,
                                     void* stream);
-
-/* The bf16 attention on the tcgen05 tensor cores: one CTA per (head, sequence,
- * 128-query tile), S = Q K^T and O = P V in TMEM, exact softmax over all keys of a
- * sequence.  Arguments as kimodo_attention_bf16; qkv 16-byte aligned. */
-KIMODO_API int kimodo_attention_bf16_tc(const void* qkv, void* out, const int* lengths, int nseq, int S,
-                                        void* stream);
 
 /* LayerNorm over 1024 features, eps 1e-5, biased variance: y fp32 [M, 1024] ->
  * out bf16 (out_bf16 = 1) or fp32 [M, 1024]; gamma, beta fp32 [1024]. */

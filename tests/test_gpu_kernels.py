@@ -110,56 +110,6 @@ def test_gemm_tcgen05_pair_vs_oracle(M, N, K, epi, out_f32, tile):
         np.testing.assert_allclose(got, ref, rtol=2 ** -8, atol=1e-5 * scale)
 
 
-STREAMK_CASES = [
-    # M, N, K, epilogue, out_f32 (stream-K pair kernel: 256 x 256 tiles, equal k-block shares)
-    (4832, 3072, 1024, kb.EPI_BIAS, False),        # QKV: shares of 3.08 tiles, tail and head pieces
-    (4832, 2048, 1024, kb.EPI_BIAS_GELU, False),
-    (4832, 1024, 1024, kb.EPI_BIAS_RESID, True),   # 76 tiles on the pairs: about one tile each
-    (4832, 1024, 2048, kb.EPI_BIAS_RESID, True),
-    (1283, 2048, 1024, kb.EPI_BIAS_GELU, False),   # shares shorter than a tile: several contributors
-    (300, 1024, 1024, kb.EPI_BIAS, False),         # 8 tiles over all pairs; second CTA of a pair out of range
-    (611, 1024, 2048, kb.EPI_BIAS_RESID, True),
-]
-
-
-@pytest.mark.parametrize("M,N,K,epi,out_f32", STREAMK_CASES)
-def test_gemm_tcgen05_streamk_vs_oracle(M, N, K, epi, out_f32):
-    require_cuda()
-    seed = M * 3 + N * 11 + K
-    A = _bf16(synth.random_vectors((M, K), seed))
-    W = _bf16(synth.random_vectors((N, K), seed + 1, 0.05))
-    bias = torch.from_numpy(synth.random_vectors((N,), seed + 2, 0.1))
-    resid = torch.from_numpy(synth.random_vectors((M, N), seed + 3)) if epi == kb.EPI_BIAS_RESID else None
-    out = kb.gemm_bf16(A.cuda(), W.cuda(), bias.cuda(), epi, out_f32, None if resid is None else resid.cuda(),
-                       stream_k=True)
-    torch.cuda.synchronize()
-    ref = _epi_ref(epi, ko.linear(_f64(A), _f64(W), bias.double().numpy()),
-                   None if resid is None else resid.double().numpy())
-    got = out.float().cpu().double().numpy()
-    scale = np.abs(ref).max()
-    if out_f32:
-        np.testing.assert_allclose(got, ref, rtol=0, atol=2e-5 * scale)
-    else:
-        np.testing.assert_allclose(got, ref, rtol=2 ** -8, atol=1e-5 * scale)
-
-
-def test_gemm_streamk_residual_in_place_and_repeatable():
-    """The stream-K residual epilogue may read and write the same fp32 buffer, and the
-    split-tile sums do not depend on the run."""
-    require_cuda()
-    M, N, K = 4832, 1024, 1024
-    A = _bf16(synth.random_vectors((M, K), 95)).cuda()
-    W = _bf16(synth.random_vectors((N, K), 96, 0.05)).cuda()
-    bias = torch.from_numpy(synth.random_vectors((N,), 97, 0.1)).cuda()
-    y = torch.from_numpy(synth.random_vectors((M, N), 98)).cuda()
-    want = kb.gemm_bf16(A, W, bias, kb.EPI_BIAS_RESID, True, y.clone(), stream_k=True)
-    again = kb.gemm_bf16(A, W, bias, kb.EPI_BIAS_RESID, True, y.clone(), stream_k=True)
-    kb.gemm_bf16(A, W, bias, kb.EPI_BIAS_RESID, True, y, out=y, stream_k=True)
-    torch.cuda.synchronize()
-    assert torch.equal(want, again)
-    assert torch.equal(want, y)
-
-
 def test_gemm_residual_in_place():
     """The residual epilogue may read and write the same fp32 buffer."""
     require_cuda()
@@ -248,14 +198,13 @@ def _attention_ref(qkv, lengths, S):
 
 
 @pytest.mark.parametrize("S,lengths", [(31, [30]), (151, [150, 60, 0]), (301, [300, 123]), (64, [63, 64])])
-@pytest.mark.parametrize("tc", [False, True])
-def test_attention_bf16_vs_oracle(S, lengths, tc):
+def test_attention_bf16_vs_oracle(S, lengths):
     require_cuda()
     lengths = [min(n, S - 1) for n in lengths]
     nseq = len(lengths)
     qkv = _bf16(synth.random_vectors((nseq * S, 3072), S + 100))
     L = torch.tensor(lengths, dtype=torch.int32)
-    out = kb.attention(qkv.cuda(), L.cuda(), nseq, S, tc=tc)
+    out = kb.attention(qkv.cuda(), L.cuda(), nseq, S)
     ref = _attention_ref(_f64(qkv), lengths, S)
     got = out.float().cpu().double().numpy()
     err = np.linalg.norm(got - ref) / np.linalg.norm(ref)
@@ -263,17 +212,16 @@ def test_attention_bf16_vs_oracle(S, lengths, tc):
     assert np.abs(got - ref).max() < 3e-2 * np.abs(ref).max()
 
 
-@pytest.mark.parametrize("tc", [False, True])
-def test_attention_bf16_masked_keys_never_read(tc):
+def test_attention_bf16_masked_keys_never_read():
     require_cuda()
     S, lengths = 151, [40, 150]
     qkv = _bf16(synth.random_vectors((2 * S, 3072), 77)).cuda()
     L = torch.tensor(lengths, dtype=torch.int32).cuda()
-    base = kb.attention(qkv, L, 2, S, tc=tc)
+    base = kb.attention(qkv, L, 2, S)
     poisoned = qkv.clone()
     for s, n in enumerate(lengths):
         poisoned[s * S + 1 + n:(s + 1) * S, 1024:] = float("nan")
-    again = kb.attention(poisoned, L, 2, S, tc=tc)
+    again = kb.attention(poisoned, L, 2, S)
     torch.cuda.synchronize()
     assert torch.equal(base, again)
 

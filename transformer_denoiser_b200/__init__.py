@@ -42,11 +42,9 @@ SIGNATURES = [
     # include/kimodo_kernels.h
     ("kimodo_gemm_bf16", _I, [_P, _I, _P, _I, _P, _P, _I, _P, _I, _I, _I, _I, _I, _I, _I, _P]),
     ("kimodo_gemm_bf16_pair", _I, [_P, _I, _P, _I, _P, _P, _I, _P, _I, _I, _I, _I, _I, _I, _I, _P]),
-    ("kimodo_gemm_bf16_streamk", _I, [_P, _I, _P, _I, _P, _P, _I, _P, _I, _I, _I, _I, _I, _I, _P]),
     ("kimodo_gemm_f32", _I, [_P, _I, _P, _I, _P, _P, _I, _P, _I, _I, _I, _I, _I, _P]),
     ("kimodo_attention_bf16", _I, [_P, _P, _P, _I, _I, _P]),
     ("kimodo_attention_f32", _I, [_P, _P, _P, _I, _I, _P]),
-    ("kimodo_attention_bf16_tc", _I, [_P, _P, _P, _I, _I, _P]),
     ("kimodo_layernorm", _I, [_P, _P, _I, _P, _P, _I, _P]),
 ]
 EPI_BIAS, EPI_BIAS_GELU, EPI_BIAS_SILU, EPI_BIAS_RESID = 0, 1, 2, 3
@@ -153,10 +151,9 @@ def _cur_stream():
 
 # ------------------------------------------------------------ kernel-level calls (torch CUDA tensors)
 
-def gemm_bf16(A, W, bias, epilogue=EPI_BIAS, out_f32=False, resid=None, out=None, K=None, tile_n=0, pair=False,
-              stream_k=False):
+def gemm_bf16(A, W, bias, epilogue=EPI_BIAS, out_f32=False, resid=None, out=None, K=None, tile_n=0, pair=False):
     """out = epilogue(A[:, :K] W[:, :K]^T + bias) on the tcgen05 GEMM (A, W bf16 CUDA tensors);
-    pair=True runs the CTA-pair kernel (256-row tiles), stream_k=True its stream-K variant."""
+    pair=True runs the CTA-pair kernel (256-row tiles)."""
     import torch
     lib = load_library()
     M, N = A.shape[0], W.shape[0]
@@ -166,11 +163,8 @@ def gemm_bf16(A, W, bias, epilogue=EPI_BIAS, out_f32=False, resid=None, out=None
     args = [_ptr_rows(A), A.stride(0), _ptr_rows(W), W.stride(0), _ptr(bias), _ptr_rows(resid),
             0 if resid is None else resid.stride(0), _ptr_rows(out), out.stride(0), M, N, K,
             int(epilogue), int(bool(out_f32))]
-    if stream_k:
-        _check(lib.kimodo_gemm_bf16_streamk(*args, _cur_stream()))
-    else:
-        fn = lib.kimodo_gemm_bf16_pair if pair else lib.kimodo_gemm_bf16
-        _check(fn(*args, int(tile_n), _cur_stream()))
+    fn = lib.kimodo_gemm_bf16_pair if pair else lib.kimodo_gemm_bf16
+    _check(fn(*args, int(tile_n), _cur_stream()))
     return out
 
 
@@ -186,16 +180,13 @@ def gemm_f32(A, W, bias, epilogue=EPI_BIAS, resid=None, out=None, K=None):
     return out
 
 
-def attention(qkv, lengths, nseq, S, tc=False):
-    """Masked attention over qkv [nseq*S, 3072] (bf16 or fp32 CUDA tensor); tc=True runs
-    the tcgen05 kernel (bf16)."""
+def attention(qkv, lengths, nseq, S):
+    """Masked attention over qkv [nseq*S, 3072] (CUDA tensor): bf16 runs the tcgen05
+    kernel, fp32 the fp32 one."""
     import torch
     lib = load_library()
     out = torch.empty((nseq * S, 1024), dtype=qkv.dtype, device=qkv.device)
-    if tc:
-        fn = lib.kimodo_attention_bf16_tc
-    else:
-        fn = lib.kimodo_attention_bf16 if qkv.dtype == torch.bfloat16 else lib.kimodo_attention_f32
+    fn = lib.kimodo_attention_bf16 if qkv.dtype == torch.bfloat16 else lib.kimodo_attention_f32
     _check(fn(_ptr(qkv), _ptr(out), _ptr(lengths), nseq, S, _cur_stream()))
     return out
 

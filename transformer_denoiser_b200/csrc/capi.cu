@@ -17,6 +17,7 @@
 #include <string.h>
 
 #include <map>
+#include <mutex>
 #include <string>
 #include <tuple>
 #include <vector>
@@ -57,9 +58,6 @@ int set_error(int code, const char* fmt, ...) {
     if (s_ != KIMODO_OK) return s_; \
   } while (0)
 
-// Folded LayerNorm: arrival counters for up to this many 32-row groups (2 M token rows).
-constexpr int PART_GROUPS_MAX = 1 << 16;
-
 enum LaunchClass { CLS_GEMM_TC = 0, CLS_ATTN = 1, CLS_LN = 2, CLS_MOTION = 3, CLS_GEMM_F32 = 4, CLS_SETUP = 5,
                    NUM_CLS = 8 };
 
@@ -69,10 +67,6 @@ struct NetW {
   float* txt_b = nullptr; float* t_b1 = nullptr; float* t_b2 = nullptr; float* in_b = nullptr; float* out_b = nullptr;
   float* qkv_b[L] = {}; float* o_b[L] = {}; float* ln1_g[L] = {}; float* ln1_b[L] = {};
   float* ff1_b[L] = {}; float* ff2_b[L] = {}; float* ln2_g[L] = {}; float* ln2_b[L] = {};
-  // folded LayerNorm (bf16 path): the projection after a LayerNorm stores W diag(gamma);
-  // *_g are the row sums of the stored weights, *_h = W beta + b (null when not folded)
-  float* qkv_g[L] = {}; float* qkv_h[L] = {}; float* ff1_g[L] = {}; float* ff1_h[L] = {};
-  float* out_g = nullptr; float* out_h = nullptr;
   int din = 0, dout = 0, in_ld = 0;
 };
 
@@ -86,7 +80,6 @@ struct Workspace {
   int* lengths = nullptr; float* st_text = nullptr; float* st_null = nullptr;
   int* tok0 = nullptr; int* row_seq = nullptr;   // packed token layout (valid tokens only)
   float* stats[2] = {};                           // LayerNorm row statistics (mean, 1/std) [M][2]
-  float2* part = nullptr;                         // folded LayerNorm: chunk statistics [D / 16][M]
 };
 
 // Token rows of a call: the padded layout (every sequence frames + 1 rows) or, when the
@@ -131,15 +124,6 @@ struct kimodo_ctx {
   long long launches = 0;
   long long last_launches = 0;
   Tokens tk;                    // token layout of the call being enqueued
-  bool pair_gemm = true;   // 256-row CTA-pair GEMM tiles for the large projections (KIMODO_PAIR_GEMM=0 disables)
-  bool stream_k = false;   // stream-K shares for them instead (KIMODO_STREAM_K=1; measured slower on the layer shapes)
-  bool attn_tc = true;     // tcgen05 attention (KIMODO_ATTN_TC=0: the mma.sync kernel)
-  bool ln_lite = true;     // LayerNorm writes row statistics, residual epilogues normalise (KIMODO_LN_LITE=0)
-  bool ln_fold = false;    // no LayerNorm launches: residual epilogues write the statistics, the next
-                           // projection folds the normalisation (KIMODO_LN_FOLD=1; measured slower)
-  int* part_cnt = nullptr; // folded LayerNorm: arrival counters per 32-row group (zero between launches)
-  float* sk_partial = nullptr;   // stream-K partial accumulators
-  int* sk_flags = nullptr;       // stream-K contributor counters (zero between launches)
   bool bf16() const { return precision == KIMODO_BF16; }
   size_t elem() const { return bf16() ? 2 : 4; }
 };
@@ -207,11 +191,7 @@ int gemm(kimodo_ctx* c, const void* A, int lda, const void* W, int ldw, int M, i
                        (double)M * N * (out_f32 ? 4.0 : (double)c->elem()) +
                        (kind == EPI_BIAS_RESID || kind == EPI_BIAS_RESID_LN ? (double)M * N * 4.0 : 0.0);
   if (c->bf16()) {
-    if (c->pair_gemm && c->stream_k && M >= 1024 && N >= 256 && gemm_tc2_supports(kind, out_f32)) {
-      return launch(c, cls_override >= 0 ? cls_override : CLS_GEMM_TC, flops, bytes, st, "gemm_sk",
-                    [&] { return gemm_sk(g, kind, out_f32, ep, c->sk_partial, c->sk_flags, c->derr, st); });
-    }
-    if (c->pair_gemm && M >= 1024 && N >= 256 && gemm_tc2_supports(kind, out_f32)) {
+    if (M >= 1024 && N >= 256 && gemm_tc2_supports(kind, out_f32)) {
       const int bn = gemm_tc2_pick_bn(M, N, kind);
       return launch(c, cls_override >= 0 ? cls_override : CLS_GEMM_TC, flops, bytes, st, "gemm_tc2",
                     [&] { return gemm_tc2(g, bn, kind, out_f32, ep, c->derr, st); });
@@ -241,41 +221,6 @@ __global__ void convert_matrix_kernel(const float* __restrict__ src, int rows, i
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-// LayerNorm (gamma, beta) folded into the projection W [rows, cols] (fp32) that follows
-// it: dst [rows, ld] = bf16(W diag(gamma)), g[j] = sum over k of the stored dst[j][k],
-// h[j] = b[j] + sum over k of W[j][k] beta[k] (double accumulation).  One CTA per row.
-__global__ void fold_layernorm_kernel(const float* __restrict__ W, int cols, const float* __restrict__ gamma,
-                                      const float* __restrict__ beta, const float* __restrict__ b, bf16* dst,
-                                      int ld, float* g, float* h) {
-  const int j = blockIdx.x;
-  double gs = 0.0, hs = 0.0;
-  for (int k = threadIdx.x; k < ld; k += blockDim.x) {
-    bf16 wf = __float2bfloat16_rn(0.f);
-    if (k < cols) {
-      const float w = W[(long)j * cols + k];
-      wf = __float2bfloat16_rn(__fmul_rn(w, gamma[k]));
-      gs += (double)__bfloat162float(wf);
-      hs += (double)w * (double)beta[k];
-    }
-    dst[(long)j * ld + k] = wf;
-  }
-  __shared__ double rg[256], rh[256];
-  rg[threadIdx.x] = gs;
-  rh[threadIdx.x] = hs;
-  __syncthreads();
-  for (int o = 128; o > 0; o >>= 1) {
-    if ((int)threadIdx.x < o) {
-      rg[threadIdx.x] += rg[threadIdx.x + o];
-      rh[threadIdx.x] += rh[threadIdx.x + o];
-    }
-    __syncthreads();
-  }
-  if (threadIdx.x == 0) {
-    g[j] = (float)rg[0];
-    h[j] = (float)((double)b[j] + rh[0]);
-  }
-}
-
 // Walks the canonical blob order; in "plan" mode only sizes the arena.
 struct WeightWalker {
   kimodo_ctx* c;
@@ -285,28 +230,6 @@ struct WeightWalker {
   size_t arena_off = 0;
   cudaStream_t st;
   int err = 0;
-  size_t last_matrix = 0;   // blob offset of the latest matrix, and of the latest vector
-  size_t last_vec = 0;
-
-  bool fold() const { return c->bf16() && c->ln_fold; }
-  // arena space for a vector that is not in the blob
-  float* extra(int n) {
-    float* dst = arena ? reinterpret_cast<float*>(arena + arena_off) : nullptr;
-    arena_off += align256((size_t)n * 4);
-    return dst;
-  }
-  // fold the LayerNorm whose gamma / beta sit at blob offsets (go, bo) into the matrix just
-  // walked (rows x cols, stored at dst with row stride ld) and its bias (blob offset bias_off)
-  void fold_into(void* dst, int rows, int cols, int ld, size_t go, size_t bo, size_t bias_off, float** g,
-                 float** h) {
-    *g = extra(rows);
-    *h = extra(rows);
-    if (arena && !err) {
-      fold_layernorm_kernel<<<rows, 256, 0, st>>>(src + last_matrix, cols, src + go, src + bo, src + bias_off,
-                                                  static_cast<bf16*>(dst), ld, *g, *h);
-      if (cudaGetLastError() != cudaSuccess) err = 1;
-    }
-  }
 
   void* matrix(int rows, int cols, int ld) {
     const size_t bytes = align256((size_t)rows * ld * c->elem());
@@ -319,12 +242,10 @@ struct WeightWalker {
       if (cudaGetLastError() != cudaSuccess) err = 1;
     }
     arena_off += bytes;
-    last_matrix = src_off;
     src_off += (size_t)rows * cols;
     return dst;
   }
   float* vec(int n) {
-    last_vec = src_off;
     const size_t bytes = align256((size_t)n * 4);
     float* dst = arena ? reinterpret_cast<float*>(arena + arena_off) : nullptr;
     if (arena && !err && cudaMemcpyAsync(dst, src + src_off, (size_t)n * 4, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
@@ -339,22 +260,17 @@ struct WeightWalker {
     n.t_W1 = matrix(D, D, D); n.t_b1 = vec(D);
     n.t_W2 = matrix(D, D, D); n.t_b2 = vec(D);
     n.in_W = matrix(D, din, in_ld); n.in_b = vec(D);
-    size_t ln_g = 0, ln_b = 0;   // blob offsets of the latest LayerNorm's gamma and beta
     for (int l = 0; l < L; ++l) {
       n.qkv_W[l] = matrix(3 * D, D, D); n.qkv_b[l] = vec(3 * D);
-      if (fold() && l > 0)
-        fold_into(n.qkv_W[l], 3 * D, D, D, ln_g, ln_b, last_vec, &n.qkv_g[l], &n.qkv_h[l]);
       n.o_W[l] = matrix(D, D, D); n.o_b[l] = vec(D);
-      n.ln1_g[l] = vec(D); ln_g = last_vec;
-      n.ln1_b[l] = vec(D); ln_b = last_vec;
+      n.ln1_g[l] = vec(D);
+      n.ln1_b[l] = vec(D);
       n.ff1_W[l] = matrix(F, D, D); n.ff1_b[l] = vec(F);
-      if (fold()) fold_into(n.ff1_W[l], F, D, D, ln_g, ln_b, last_vec, &n.ff1_g[l], &n.ff1_h[l]);
       n.ff2_W[l] = matrix(D, F, F); n.ff2_b[l] = vec(D);
-      n.ln2_g[l] = vec(D); ln_g = last_vec;
-      n.ln2_b[l] = vec(D); ln_b = last_vec;
+      n.ln2_g[l] = vec(D);
+      n.ln2_b[l] = vec(D);
     }
     n.out_W = matrix(dout, D, D); n.out_b = vec(dout);
-    if (fold()) fold_into(n.out_W, dout, D, D, ln_g, ln_b, last_vec, &n.out_g, &n.out_h);
   }
   void all() {
     net(c->net[0], ROOT_F, ROOT_F, ROOT_IN_LD);
@@ -398,7 +314,7 @@ int ensure_workspace(kimodo_ctx* c, int nseq, int frames, int steps) {
       {(void**)&w.lengths, (size_t)NS * 4},                {(void**)&w.st_text, (size_t)NS * DTXT * 4},
       {(void**)&w.st_null, (size_t)NS * DTXT * 4},        {(void**)&w.tok0, (size_t)(NS + 1) * 4},
       {(void**)&w.row_seq, (size_t)R2 * 4},               {(void**)&w.stats[0], (size_t)R2 * 8},
-      {(void**)&w.stats[1], (size_t)R2 * 8},              {(void**)&w.part, (size_t)R2 * (D / 16) * 8}};
+      {(void**)&w.stats[1], (size_t)R2 * 8}};
   for (auto& p : plan) off += align256(p.second);
   void* arena = nullptr;
   cudaError_t err = cudaMalloc(&arena, off);
@@ -469,64 +385,32 @@ int run_net(kimodo_ctx* c, int net, int nseq, int T, int len_mod, const void* A_
     if (c->bf16()) e.out32 = w.y;   // fp32 residual stream
     KD_TRY(gemm(c, A_in, n.in_ld, n.in_W, n.in_ld, M, D, n.in_ld, EPI_INPROJ, act_f32, e, st));
   }
-  // Residual stream: on the bf16 path the fp32 buffer y carries the layer input
-  // (LayerNorm output) and is updated in place by the residual epilogues and by
-  // LayerNorm; h holds its bf16 copy, the GEMM operand.  On the fp32 path the
-  // residual is h itself.
-  const void* resid = c->bf16() ? static_cast<const void*>(w.y) : w.h;
-  float* ln32 = c->bf16() ? w.y : nullptr;
+  // Residual stream.  The residual epilogues write the sub-layer sums z into the fp32
+  // buffer y.  bf16 path: y also serves as the residual, holding the un-normalised sums;
+  // LayerNorm writes only the bf16 GEMM operand h and (mean, 1/std) per row, and the
+  // next residual epilogue adds gamma (z - mean) / std + beta itself (EPI_BIAS_RESID_LN).
+  // fp32 path: LayerNorm writes the normalised fp32 rows into h, which is the residual.
+  const bool bf = c->bf16();
+  const void* resid = bf ? static_cast<const void*>(w.y) : w.h;
   const double eb = (double)c->elem();
-  // Row-statistics residual (bf16 path): y keeps the un-normalised sums z;
-  // LayerNorm writes only the bf16 operand h and (mean, 1/std) per row, and the next
-  // residual epilogue adds gamma (z - mean) / std + beta itself (EPI_BIAS_RESID_LN).
-  // Folded LayerNorm (bf16 path): no LayerNorm launches.  The residual epilogues also write
-  // bf16(y) into h and the row statistics of y (stats[0] after the attention block,
-  // stats[1] after the FFN); the projection that follows a LayerNorm runs on bf16(y)
-  // with W diag(gamma) and normalises in its epilogue.
-  const bool fold = c->bf16() && c->ln_fold && !c->stream_k && w.part != nullptr && n.ff1_g[0] != nullptr &&
-                    (M + 31) / 32 <= PART_GROUPS_MAX;
-  const bool lite = !fold && c->bf16() && c->ln_lite && !c->stream_k && w.stats[0] != nullptr;
-  if (lite || fold) ln32 = nullptr;
   auto resid_epi = [&](EpiParams& e, int which, const float* g, const float* b) {
-    if (fold) {
-      e.part = w.part;
-      e.part_cnt = c->part_cnt;
-      e.stats_out = w.stats[1 - which];
-      e.out16 = static_cast<bf16*>(w.h);
-      e.ldo16 = D;
-    }
-    if ((!lite && !fold) || g == nullptr) return EPI_BIAS_RESID;
+    if (!bf || g == nullptr) return EPI_BIAS_RESID;
     e.ln_stats = w.stats[which];
     e.ln_g = g;
     e.ln_b = b;
     return EPI_BIAS_RESID_LN;
   };
-  // consumer side of a folded LayerNorm whose statistics are in stats[which]
-  auto fold_epi = [&](EpiParams& e, const float* g, const float* h, int which) {
-    if (!fold || g == nullptr) return;
-    e.fold_g = g;
-    e.bias = h;
-    e.ln_stats = w.stats[which];
-  };
   for (int l = 0; l < L; ++l) {
     EpiParams e;
     e.bias = n.qkv_b[l]; e.out = w.qkv; e.ldo = 3 * D; e.N = 3 * D; e.M = M;
-    fold_epi(e, n.qkv_g[l], n.qkv_h[l], 1);
     KD_TRY(gemm(c, w.h, D, n.qkv_W[l], D, M, 3 * D, D, EPI_BIAS, act_f32, e, st));
     const double aflops = packed ? 4.0 * (double)M * S * DH * H : 4.0 * (double)nseq * S * S * DH * H;
     const double abytes = (double)M * 3 * D * eb + (double)M * D * eb;
-    if (c->bf16()) {
-      if (c->attn_tc) {
-        KD_TRY(launch(c, CLS_ATTN, aflops, abytes, st, "attention_tc", [&] {
-          return attention_tc(static_cast<const bf16*>(w.qkv), static_cast<bf16*>(w.attn), M, w.lengths, len_mod,
-                              nseq, S, c->derr, st, tok0);
-        }));
-      } else {
-        KD_TRY(launch(c, CLS_ATTN, aflops, abytes, st, "attention_bf16", [&] {
-          return attention_bf16(static_cast<const bf16*>(w.qkv), static_cast<bf16*>(w.attn), w.lengths, len_mod,
-                                nseq, S, st, tok0);
-        }));
-      }
+    if (bf) {
+      KD_TRY(launch(c, CLS_ATTN, aflops, abytes, st, "attention_tc", [&] {
+        return attention_tc(static_cast<const bf16*>(w.qkv), static_cast<bf16*>(w.attn), M, w.lengths, len_mod,
+                            nseq, S, c->derr, st, tok0);
+      }));
     } else {
       KD_TRY(launch(c, CLS_ATTN, aflops, abytes, st, "attention_f32", [&] {
         return attention_f32(static_cast<const float*>(w.qkv), static_cast<float*>(w.attn), w.lengths, len_mod,
@@ -534,34 +418,30 @@ int run_net(kimodo_ctx* c, int net, int nseq, int T, int len_mod, const void* A_
       }));
     }
     EpiParams eo;
-    eo.bias = n.o_b[l]; eo.out = w.y; eo.ldo = D; eo.resid = resid; eo.ldr = D; eo.N = D; eo.M = M;
+    eo.bias = n.o_b[l]; eo.out = w.y; eo.ldo = D; eo.resid = resid; eo.ldr = D;
+    eo.N = D; eo.M = M;
     // layer 0 adds the un-normalised input projection; later layers the previous LayerNorm 2
     const int ko = resid_epi(eo, 1, l > 0 ? n.ln2_g[l - 1] : nullptr, l > 0 ? n.ln2_b[l - 1] : nullptr);
     KD_TRY(gemm(c, w.attn, D, n.o_W[l], D, M, D, D, ko, true, eo, st));
-    const double lnb = lite ? (double)M * D * (4.0 + eb) + (double)M * 8 : (double)M * D * (4.0 + eb + (c->bf16() ? 4.0 : 0.0));
-    if (!fold) {
-      KD_TRY(launch(c, CLS_LN, 0, lnb, st, "layernorm", [&] {
-        return layernorm(w.y, w.h, c->bf16(), n.ln1_g[l], n.ln1_b[l], M, st, ln32, lite ? w.stats[0] : nullptr);
-      }));
-    }
+    const double lnb = bf ? (double)M * D * (4.0 + eb) + (double)M * 8 : (double)M * D * 8.0;
+    KD_TRY(launch(c, CLS_LN, 0, lnb, st, "layernorm", [&] {
+      return layernorm(w.y, w.h, bf, n.ln1_g[l], n.ln1_b[l], M, st, bf ? w.stats[0] : nullptr);
+    }));
     EpiParams e1;
     e1.bias = n.ff1_b[l]; e1.out = w.u; e1.ldo = F; e1.N = F; e1.M = M;
-    fold_epi(e1, n.ff1_g[l], n.ff1_h[l], 0);
     KD_TRY(gemm(c, w.h, D, n.ff1_W[l], D, M, F, D, EPI_BIAS_GELU, act_f32, e1, st));
     EpiParams e2;
-    e2.bias = n.ff2_b[l]; e2.out = w.y; e2.ldo = D; e2.resid = resid; e2.ldr = D; e2.N = D; e2.M = M;
+    e2.bias = n.ff2_b[l]; e2.out = w.y; e2.ldo = D; e2.resid = resid; e2.ldr = D;
+    e2.N = D; e2.M = M;
     const int kf = resid_epi(e2, 0, n.ln1_g[l], n.ln1_b[l]);
     KD_TRY(gemm(c, w.u, F, n.ff2_W[l], F, M, D, F, kf, true, e2, st));
-    if (!fold) {
-      KD_TRY(launch(c, CLS_LN, 0, lnb, st, "layernorm", [&] {
-        return layernorm(w.y, w.h, c->bf16(), n.ln2_g[l], n.ln2_b[l], M, st, ln32, lite ? w.stats[1] : nullptr);
-      }));
-    }
+    KD_TRY(launch(c, CLS_LN, 0, lnb, st, "layernorm", [&] {
+      return layernorm(w.y, w.h, bf, n.ln2_g[l], n.ln2_b[l], M, st, bf ? w.stats[1] : nullptr);
+    }));
   }
   EpiParams eo;
   eo.bias = n.out_b; eo.out = hat; eo.ldo = n.dout; eo.lengths = w.lengths; eo.len_mod = len_mod; eo.S = S;
   eo.T = T; eo.N = n.dout; eo.M = M; eo.tok0 = tok0; eo.row_seq = row_seq;
-  fold_epi(eo, n.out_g, n.out_h, 1);
   return gemm(c, w.h, D, n.out_W, D, M, n.dout, D, EPI_OUTPROJ, true, eo, st);
 }
 
@@ -725,20 +605,13 @@ int kimodo_load_weights(kimodo_ctx** out_ctx, const float* host_blob, size_t n_f
   if (precision == KIMODO_BF16 && !gemm_tc_available())
     return set_error(KIMODO_EUNSUPPORTED, "cuTensorMapEncodeTiled is unavailable in this driver");
 
-  if (gemm_tc_prepare() != cudaSuccess || gemm_tc2_prepare() != cudaSuccess || gemm_sk_prepare() != cudaSuccess ||
-      attention_prepare() != cudaSuccess || attention_tc_prepare() != cudaSuccess) {
+  if (gemm_tc_prepare() != cudaSuccess || gemm_tc2_prepare() != cudaSuccess || attention_tc_prepare() != cudaSuccess) {
     cudaGetLastError();
     return set_error(KIMODO_EUNSUPPORTED, "kernel attributes could not be set on device %d", device);
   }
   kimodo_ctx* c = new kimodo_ctx();
   c->device = device;
   c->precision = precision;
-  if (const char* ev = getenv("KIMODO_PAIR_GEMM")) c->pair_gemm = ev[0] != '0';
-  if (const char* ev = getenv("KIMODO_STREAM_K")) c->stream_k = ev[0] != '0';
-  if (const char* ev = getenv("KIMODO_ATTN_TC")) c->attn_tc = ev[0] != '0';
-  if (const char* ev = getenv("KIMODO_LN_LITE")) c->ln_lite = ev[0] != '0';
-  if (const char* ev = getenv("KIMODO_LN_FOLD")) c->ln_fold = ev[0] != '0';
-  if (precision != KIMODO_BF16) c->ln_fold = false;
   c->num_sms = prop.multiProcessorCount;
   auto fail = [&](int code) {
     kimodo_free(c);
@@ -780,13 +653,6 @@ int kimodo_load_weights(kimodo_ctx** out_ctx, const float* host_blob, size_t n_f
       return fail(set_error(KIMODO_ECUDA, "pe upload"));
     if (cudaMalloc(&c->derr, sizeof(DevError)) != cudaSuccess) return fail(set_error(KIMODO_ENOMEM, "error word"));
     cudaMemset(c->derr, 0, sizeof(DevError));
-    if (cudaMalloc(&c->sk_partial, gemm_sk_workspace_floats() * 4) != cudaSuccess ||
-        cudaMalloc(&c->sk_flags, 2 * GEMM_SK_MAX_PAIRS * sizeof(int)) != cudaSuccess)
-      return fail(set_error(KIMODO_ENOMEM, "stream-K workspace"));
-    cudaMemset(c->sk_flags, 0, 2 * GEMM_SK_MAX_PAIRS * sizeof(int));
-    if (cudaMalloc(&c->part_cnt, PART_GROUPS_MAX * sizeof(int)) != cudaSuccess)
-      return fail(set_error(KIMODO_ENOMEM, "LayerNorm statistics counters"));
-    cudaMemset(c->part_cnt, 0, PART_GROUPS_MAX * sizeof(int));
   }
 
   // weights: plan the arena, stage the fp32 blob on the device, convert
@@ -821,9 +687,6 @@ void kimodo_free(kimodo_ctx* c) {
   for (auto e : c->ev_pool) cudaEventDestroy(e);
   if (c->ws.arena) cudaFree(c->ws.arena);
   if (c->zbuf) cudaFree(c->zbuf);
-  if (c->sk_partial) cudaFree(c->sk_partial);
-  if (c->sk_flags) cudaFree(c->sk_flags);
-  if (c->part_cnt) cudaFree(c->part_cnt);
   if (c->warena) cudaFree(c->warena);
   if (c->pe) cudaFree(c->pe);
   if (c->derr) cudaFree(c->derr);
@@ -1062,10 +925,6 @@ int kimodo_sync_status(kimodo_ctx* c, void* stream) {
   KD_CUDA(cudaMemcpy(&h, c->derr, sizeof(h), cudaMemcpyDeviceToHost));
   if (h.code != 0) {
     KD_CUDA(cudaMemset(c->derr, 0, sizeof(DevError)));
-    // an interrupted stream-K launch may leave contributor counters raised, and an interrupted
-    // residual GEMM its LayerNorm-statistics arrival counters
-    KD_CUDA(cudaMemset(c->sk_flags, 0, 2 * GEMM_SK_MAX_PAIRS * sizeof(int)));
-    KD_CUDA(cudaMemset(c->part_cnt, 0, PART_GROUPS_MAX * sizeof(int)));
     return set_error(h.code, "device wait timed out in kernel stage %d (block %d)", h.where, h.block);
   }
   return KIMODO_OK;
@@ -1130,8 +989,6 @@ int prepared_device() {
   if (!done[dev]) {
     KD_CUDA(gemm_tc_prepare());
     KD_CUDA(gemm_tc2_prepare());
-    KD_CUDA(gemm_sk_prepare());
-    KD_CUDA(attention_prepare());
     KD_CUDA(attention_tc_prepare());
     done[dev] = true;
   }
@@ -1210,41 +1067,6 @@ int kimodo_gemm_bf16_pair(const void* A, int lda, const void* W, int ldw, const 
   return KIMODO_OK;
 }
 
-int kimodo_gemm_bf16_streamk(const void* A, int lda, const void* W, int ldw, const float* bias, const void* resid,
-                             int ldr, void* out, int ldo, int M, int N, int K, int epilogue, int out_f32,
-                             void* stream) {
-  g_last_error.clear();
-  KD_TRY(check_gemm_args(A, lda, W, ldw, bias, resid, out, ldo, M, N, K, epilogue));
-  if (lda % 8 || ldw % 8 || (reinterpret_cast<uintptr_t>(A) & 15) || (reinterpret_cast<uintptr_t>(W) & 15))
-    return set_error(KIMODO_EINVAL, "bf16 operands need 16-byte aligned rows (lda, ldw multiples of 8)");
-  if (ldo % 4 || (reinterpret_cast<uintptr_t>(out) & 15) || (epilogue == 3 && (ldr % 4 ||
-      (reinterpret_cast<uintptr_t>(resid) & 15))) || (reinterpret_cast<uintptr_t>(bias) & 15))
-    return set_error(KIMODO_EINVAL, "out, resid and bias need 16-byte alignment and ldo, ldr multiples of 4");
-  if (!gemm_tc2_supports(epilogue, out_f32 != 0))
-    return set_error(KIMODO_EINVAL, "pair GEMM epilogues: bias or GELU with bf16 output, residual with fp32 output");
-  if (N % 16 || ((long)ldo * (out_f32 ? 4 : 2)) % 16)
-    return set_error(KIMODO_EINVAL, "pair GEMM needs N % 16 == 0 and 16-byte output rows");
-  KD_TRY(prepared_device());
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  // a workspace of its own for this call, stream-ordered
-  float* partial = nullptr;
-  int* flags = nullptr;
-  KD_CUDA(cudaMallocAsync(reinterpret_cast<void**>(&partial), gemm_sk_workspace_floats() * 4, st));
-  cudaError_t e = cudaMallocAsync(reinterpret_cast<void**>(&flags), 2 * GEMM_SK_MAX_PAIRS * sizeof(int), st);
-  if (e == cudaSuccess) e = cudaMemsetAsync(flags, 0, 2 * GEMM_SK_MAX_PAIRS * sizeof(int), st);
-  if (e == cudaSuccess) {
-    GemmArgs g;
-    g.A = A; g.B = W; g.M = M; g.N = N; g.K = K; g.lda = lda; g.ldb = ldw;
-    EpiParams ep;
-    ep.bias = bias; ep.out = out; ep.ldo = ldo; ep.resid = resid; ep.ldr = ldr; ep.N = N; ep.M = M;
-    e = gemm_sk(g, epilogue, out_f32 != 0, ep, partial, flags, kernel_error_word(), st);
-  }
-  if (flags) cudaFreeAsync(flags, st);
-  cudaFreeAsync(partial, st);
-  KD_CUDA(e);
-  return KIMODO_OK;
-}
-
 int kimodo_gemm_f32(const float* A, int lda, const float* W, int ldw, const float* bias, const float* resid, int ldr,
                     float* out, int ldo, int M, int N, int K, int epilogue, void* stream) {
   g_last_error.clear();
@@ -1259,16 +1081,6 @@ int kimodo_gemm_f32(const float* A, int lda, const float* W, int ldw, const floa
 }
 
 int kimodo_attention_bf16(const void* qkv, void* out, const int* lengths, int nseq, int S, void* stream) {
-  g_last_error.clear();
-  if (!qkv || !out || !lengths) return set_error(KIMODO_EINVAL, "NULL tensor argument");
-  if (nseq < 1 || S < 1 || S > MAX_FRAMES + 1) return set_error(KIMODO_EINVAL, "need nseq >= 1, 1 <= S <= 301");
-  KD_TRY(prepared_device());
-  KD_CUDA(attention_bf16(static_cast<const bf16*>(qkv), static_cast<bf16*>(out), lengths, nseq, nseq, S,
-                         static_cast<cudaStream_t>(stream)));
-  return KIMODO_OK;
-}
-
-int kimodo_attention_bf16_tc(const void* qkv, void* out, const int* lengths, int nseq, int S, void* stream) {
   g_last_error.clear();
   if (!qkv || !out || !lengths) return set_error(KIMODO_EINVAL, "NULL tensor argument");
   if (nseq < 1 || S < 1 || S > MAX_FRAMES + 1) return set_error(KIMODO_EINVAL, "need nseq >= 1, 1 <= S <= 301");
@@ -1342,7 +1154,6 @@ constexpr size_t noalloc_layout(char* base, size_t e, size_t rows, size_t nseq, 
   char* stt = take(nseq * DTXT * 4);
   char* st0 = take(rows * 8);
   char* st1 = take(rows * 8);
-  char* prt = take(rows * (D / 16) * 8);
   if (w) {
     w->h = h; w->qkv = qkv; w->attn = attn; w->u = u; w->y = reinterpret_cast<float*>(y);
     w->A_root = ar; w->A_body = ab;
@@ -1353,7 +1164,6 @@ constexpr size_t noalloc_layout(char* base, size_t e, size_t rows, size_t nseq, 
     w->tmlp[0] = reinterpret_cast<float*>(tm0); w->tmlp[1] = reinterpret_cast<float*>(tm1);
     w->lengths = reinterpret_cast<int*>(len); w->st_text = reinterpret_cast<float*>(stt); w->st_null = nullptr;
     w->stats[0] = reinterpret_cast<float*>(st0); w->stats[1] = reinterpret_cast<float*>(st1);
-    w->part = reinterpret_cast<float2*>(prt);
   }
   return off;
 }
@@ -1367,17 +1177,24 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[NOALLOC_BYTES];
 
 namespace {
 
-// Device address of g_noalloc_scratch on the current device (set-up on first use).
+// Device address of g_noalloc_scratch on the current device.  In host code the array's
+// name stands for a host-side shadow, not the device memory, so the address is looked up
+// once per device (set-up, with that device current) and cached; the lookup is serialised
+// so that threads making their first call at the same time agree on it.
 int noalloc_scratch(char** out) {
+  static std::mutex mu;
   static void* addr[64] = {};
   int dev = 0;
   KD_CUDA(cudaGetDevice(&dev));
   if (dev < 0 || dev >= 64) return set_error(KIMODO_EINVAL, "device index %d", dev);
+  std::lock_guard<std::mutex> lock(mu);
   if (!addr[dev]) {
     void* p = nullptr;
     cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-    if (e != cudaSuccess || !p)
+    if (e != cudaSuccess || !p) {
+      cudaGetLastError();
       return set_error(KIMODO_ECUDA, "cudaGetSymbolAddress of the static scratch failed: %s", cudaGetErrorString(e));
+    }
     addr[dev] = p;
   }
   *out = static_cast<char*>(addr[dev]);

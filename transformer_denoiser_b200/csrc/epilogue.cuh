@@ -48,24 +48,6 @@ struct EpiParams {
   int T = 1;                     // frames per sequence (EPI_OUTPROJ)
   int N = 0;                     // valid output columns
   int M = 0;                     // valid rows
-  // LayerNorm folded into the GEMMs (bf16 path, N == D for the producers).
-  // Producer (EPI_BIAS_RESID / EPI_BIAS_RESID_LN with part != nullptr): besides the fp32
-  // sum y it writes bf16(y) to out16 [M, ldo16] and, per row and 16-column chunk c, the
-  // chunk's (mean, sum of squared deviations) to part[c * M + row]; the last of the
-  // part_arrivals warps that cover a 32-row group (counted in part_cnt[row / 32], zero
-  // before the launch and left zero) merges the row's D / 16 chunks and writes
-  // (mean, 1/std) to stats_out [M][2].
-  bf16* out16 = nullptr;
-  long ldo16 = 0;
-  float2* part = nullptr;
-  int* part_cnt = nullptr;
-  float* stats_out = nullptr;
-  int part_arrivals = 0;         // set by the GEMM launcher: n tiles x epilogue warps per row group
-  // Consumer (EPI_BIAS, EPI_BIAS_GELU, EPI_OUTPROJ with fold_g != nullptr): A holds the
-  // un-normalised rows y, B = W diag(gamma), and the epilogue forms
-  // acc / std - (mean / std) fold_g + bias with (mean, 1/std) from ln_stats, where
-  // fold_g = B 1 (row sums of the stored bf16 B) and bias = W beta + b.
-  const float* fold_g = nullptr;
 };
 
 // erf by Abramowitz & Stegun, Handbook of Mathematical Functions, formula 7.1.26:
@@ -277,107 +259,6 @@ __device__ __forceinline__ uint32_t bf16x2_bits(float a, float b) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
-// ---------------------------------------------------------------------------
-// Row statistics of the folded LayerNorm, computed piecewise in the residual GEMMs.
-// Every sum below has a fixed association order (no contraction), so the single-CTA
-// and the CTA-pair kernels produce the same bits for the same row.
-
-__device__ __forceinline__ float sum4_tree(float a, float b, float c, float d) {
-  return __fadd_rn(__fadd_rn(a, b), __fadd_rn(c, d));
-}
-
-// (mean, sum of squared deviations) of 16 values: quads summed as (x0 + x1) + (x2 + x3),
-// then the four quad sums the same way; the squared deviations likewise.
-__device__ __forceinline__ float2 chunk_stats16(const float (&x)[16]) {
-  const float mean = __fmul_rn(sum4_tree(sum4_tree(x[0], x[1], x[2], x[3]), sum4_tree(x[4], x[5], x[6], x[7]),
-                                         sum4_tree(x[8], x[9], x[10], x[11]), sum4_tree(x[12], x[13], x[14], x[15])),
-                               0.0625f);
-  float q[4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const float d0 = __fsub_rn(x[4 * i], mean), d1 = __fsub_rn(x[4 * i + 1], mean);
-    const float d2 = __fsub_rn(x[4 * i + 2], mean), d3 = __fsub_rn(x[4 * i + 3], mean);
-    q[i] = sum4_tree(__fmul_rn(d0, d0), __fmul_rn(d1, d1), __fmul_rn(d2, d2), __fmul_rn(d3, d3));
-  }
-  return make_float2(mean, sum4_tree(q[0], q[1], q[2], q[3]));
-}
-
-// The same statistics when four consecutive lanes hold the chunk, four values each
-// (lane 4r + i holds values 4i .. 4i + 3): the xor-1 and xor-2 exchanges reproduce the
-// association order of chunk_stats16 exactly (IEEE addition is commutative).
-__device__ __forceinline__ float2 chunk_stats16_quad(float v0, float v1, float v2, float v3) {
-  float t = sum4_tree(v0, v1, v2, v3);
-  t = __fadd_rn(t, __shfl_xor_sync(0xffffffffu, t, 1));
-  t = __fadd_rn(t, __shfl_xor_sync(0xffffffffu, t, 2));
-  const float mean = __fmul_rn(t, 0.0625f);
-  const float d0 = __fsub_rn(v0, mean), d1 = __fsub_rn(v1, mean), d2 = __fsub_rn(v2, mean), d3 = __fsub_rn(v3, mean);
-  float q = sum4_tree(__fmul_rn(d0, d0), __fmul_rn(d1, d1), __fmul_rn(d2, d2), __fmul_rn(d3, d3));
-  q = __fadd_rn(q, __shfl_xor_sync(0xffffffffu, q, 1));
-  q = __fadd_rn(q, __shfl_xor_sync(0xffffffffu, q, 2));
-  return make_float2(mean, q);
-}
-
-// Merge of two blocks of n values each (Chan, Golub & LeVeque's pairwise update with
-// equal counts): mean = (ma + mb) / 2, M2 = M2a + M2b + (mb - ma)^2 n / 2.
-__device__ __forceinline__ void merge_equal(float& ma, float& qa, float mb, float qb, float half_n) {
-  const float d = __fsub_rn(mb, ma);
-  ma = __fmul_rn(__fadd_rn(ma, mb), 0.5f);
-  qa = __fadd_rn(__fadd_rn(qa, qb), __fmul_rn(__fmul_rn(d, d), half_n));
-}
-
-// (mean, 1/std) of row `row` from its D / 16 chunk statistics, merged pairwise
-// (chunks 2i and 2i + 1, then pairs of pairs, ...); biased variance, eps = 1e-5.
-__device__ __forceinline__ float2 row_stats_from_chunks(const float2* part, long M, int row) {
-  constexpr int NCH = D / 16;
-  static_assert((NCH & (NCH - 1)) == 0 && NCH <= 128, "chunk count must be a power of two");
-  // every load is issued before the first merge, so their latencies overlap
-  float2 p[NCH];
-#pragma unroll
-  for (int i = 0; i < NCH; ++i) p[i] = __ldcg(part + (long)i * M + row);
-  float sm[8], sq[8];   // sm[l], sq[l]: a merged block of 16 * 2^l values awaiting its partner
-#pragma unroll
-  for (int i = 0; i < NCH; ++i) {
-    float m = p[i].x, q = p[i].y;
-#pragma unroll
-    for (int l = 0; l < 8; ++l) {
-      if (!((i >> l) & 1)) {
-        sm[l] = m;
-        sq[l] = q;
-        break;
-      }
-      merge_equal(sm[l], sq[l], m, q, (float)(8 << l));
-      m = sm[l];
-      q = sq[l];
-    }
-  }
-  constexpr int TOP = NCH == 1 ? 0 : NCH == 2 ? 1 : NCH == 4 ? 2 : NCH == 8 ? 3 : NCH == 16 ? 4 : NCH == 32 ? 5
-                    : NCH == 64 ? 6 : 7;
-  const float var = __fmul_rn(sq[TOP], 1.0f / (float)D);
-  return make_float2(sm[TOP], __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(var, 1e-5f))));
-}
-
-// Called by all 32 lanes of an epilogue warp after it wrote its chunk statistics for
-// rows [row0, row0 + 32) of one output tile (row0 a multiple of 32).  Counts the warp's
-// arrival; the group's last warp resets the counter and writes the 32 rows' statistics.
-__device__ __forceinline__ void part_arrive(const EpiParams& e, int row0, int lane) {
-  if (row0 >= e.M) return;
-  __syncwarp();
-  int last = 0;
-  if (lane == 0) {
-    __threadfence();
-    int* cnt = e.part_cnt + (row0 >> 5);
-    last = atomicAdd(cnt, 1) == e.part_arrivals - 1;
-    if (last) {
-      *cnt = 0;
-      __threadfence();
-    }
-  }
-  last = __shfl_sync(0xffffffffu, last, 0);
-  if (!last) return;
-  const int row = row0 + lane;
-  if (row < e.M) *reinterpret_cast<float2*>(e.stats_out + 2 * (long)row) = row_stats_from_chunks(e.part, e.M, row);
-}
-
 template <int CW>
 struct EpiLanes {
   static constexpr int LDE = CW + 4;
@@ -426,9 +307,7 @@ __device__ __forceinline__ void epilogue_prefetch(const EpiParams& e, int row0, 
   }
 }
 
-// FOLD: the folded-LayerNorm form (bias / GELU / output projection consume the row
-// statistics, the residual kinds produce them).
-template <int KIND, typename OutT, int CW, bool FOLD = false>
+template <int KIND, typename OutT, int CW>
 __device__ __forceinline__ void epilogue_warp_tile(const EpiParams& e, const float* st, int row0, int col0,
                                                    int lane, const float4 (&pre)[EpiLanes<CW>::PASSES],
                                                    const float4 bias4) {
@@ -453,18 +332,9 @@ __device__ __forceinline__ void epilogue_warp_tile(const EpiParams& e, const flo
         const int frame = pos - 1;
         const bool valid = frame < e.lengths[seq % e.len_mod];
         OutT* o = reinterpret_cast<OutT*>(e.out) + ((long)seq * e.T + frame) * e.ldo + col;
-        if constexpr (FOLD) {
-          // folded LayerNorm: acc / std - (mean / std) g + (W beta + b)
-          const float2 st2 = *reinterpret_cast<const float2*>(e.ln_stats + 2 * (long)row);
-          const float ra = st2.y, rb = -st2.x * st2.y;
 #pragma unroll
-          for (int j = 0; j < 4; ++j)
-            if (col + j < e.N) o[j] = from_f<OutT>(valid ? fmaf(v[j], ra, fmaf(rb, e.fold_g[col + j], b4[j])) : 0.f);
-        } else {
-#pragma unroll
-          for (int j = 0; j < 4; ++j)
-            if (col + j < e.N) o[j] = from_f<OutT>(valid ? v[j] + b4[j] : 0.f);
-        }
+        for (int j = 0; j < 4; ++j)
+          if (col + j < e.N) o[j] = from_f<OutT>(valid ? v[j] + b4[j] : 0.f);
       }
     } else {
       if constexpr (KIND == EPI_INPROJ) {
@@ -482,20 +352,11 @@ __device__ __forceinline__ void epilogue_warp_tile(const EpiParams& e, const flo
         }
         if (in_rows && e.out32 != nullptr) store4<float>(e.out32 + (long)row * e.ldo + col, v[0], v[1], v[2], v[3]);
       } else {
-        if constexpr ((KIND == EPI_BIAS || KIND == EPI_BIAS_GELU) && FOLD) {
-          // folded LayerNorm: acc / std - (mean / std) g + (W beta + b), as the pair GEMM forms it
-          const float2 st2 = *reinterpret_cast<const float2*>(e.ln_stats + 2 * (long)min(row, e.M - 1));
-          const float ra = st2.y, rb = -st2.x * st2.y;
-          const float4 g4 = ld4(e.fold_g + col);
-          v[0] = fmaf(v[0], ra, fmaf(rb, g4.x, b4[0])); v[1] = fmaf(v[1], ra, fmaf(rb, g4.y, b4[1]));
-          v[2] = fmaf(v[2], ra, fmaf(rb, g4.z, b4[2])); v[3] = fmaf(v[3], ra, fmaf(rb, g4.w, b4[3]));
-        } else {
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            float x = v[j] + b4[j];
-            if constexpr (KIND == EPI_BIAS_SILU) x = silu_f(x);
-            v[j] = x;
-          }
+        for (int j = 0; j < 4; ++j) {
+          float x = v[j] + b4[j];
+          if constexpr (KIND == EPI_BIAS_SILU) x = silu_f(x);
+          v[j] = x;
         }
         if constexpr (KIND == EPI_BIAS_GELU) {
           // bf16 outputs take the packed GELU of the pair GEMM, fp32 outputs the A&S 7.1.26 one
@@ -517,18 +378,6 @@ __device__ __forceinline__ void epilogue_warp_tile(const EpiParams& e, const flo
           const float4 g4 = ld4(e.ln_g + col);
           v[0] += fmaf(pre[p].x, ra, rb) * g4.x; v[1] += fmaf(pre[p].y, ra, rb) * g4.y;
           v[2] += fmaf(pre[p].z, ra, rb) * g4.z; v[3] += fmaf(pre[p].w, ra, rb) * g4.w;
-        }
-        if constexpr (KIND == EPI_BIAS_RESID || KIND == EPI_BIAS_RESID_LN) {
-          if constexpr (FOLD) {
-            // folded LayerNorm producer: chunk statistics of the new sum (the four lanes of
-            // this row hold its 16 columns; N % 16 == 0, so every lane is here) and its bf16 copy
-            static_assert(CW == 16, "four lanes per 16-column chunk");
-            const float2 cs = chunk_stats16_quad(v[0], v[1], v[2], v[3]);
-            if (in_rows) {
-              if ((lane & 3) == 0) e.part[(long)(col0 >> 4) * e.M + row] = cs;
-              store4<bf16>(e.out16 + (long)row * e.ldo16 + col, v[0], v[1], v[2], v[3]);
-            }
-          }
         }
       }
       if (in_rows) {

@@ -67,8 +67,7 @@ __device__ __forceinline__ void record_timeout(DevError* err, int where, volatil
   }
 }
 
-// FOLD: the folded-LayerNorm instantiation (see epilogue_warp_tile).
-template <int BN, int STAGES, int KIND, typename OutT, typename ResT, bool FOLD>
+template <int BN, int STAGES, int KIND, typename OutT, typename ResT>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                int num_m_tiles, int num_n_tiles, int num_kb, EpiParams ep, DevError* err) {
@@ -206,8 +205,6 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     constexpr int CW = C::CW;
     constexpr int PASSES = EpiLanes<CW>::PASSES;
     float* st = epi_smem + (warp - 2) * 32 * (CW + 4);
-    // folded LayerNorm statistics produced by the residual epilogues
-    constexpr bool stats = FOLD && (KIND == EPI_BIAS_RESID || KIND == EPI_BIAS_RESID_LN);
     int local = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++local) {
       const int acc = local & 1;
@@ -229,7 +226,6 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         ptx::tc_fence_before();
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive(tempty_bar(acc));
-        if constexpr (stats) part_arrive(ep, m_blk * BM + quarter * 32, lane);
         continue;
       }
       // two register buffers: the TMEM load and global prefetch of chunk c + 1 are in
@@ -242,7 +238,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         for (int j = 0; j < CW; j += 4)
           *reinterpret_cast<float4*>(st + lane * (CW + 4) + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
         __syncwarp();
-        epilogue_warp_tile<KIND, OutT, CW, FOLD>(ep, st, row0, gcol + c * CW, lane, pre, bias4);
+        epilogue_warp_tile<KIND, OutT, CW>(ep, st, row0, gcol + c * CW, lane, pre, bias4);
         __syncwarp();
       };
       auto release_if_last = [&](int c) {
@@ -272,7 +268,6 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         }
         process(vb, pb, bb, c + 1);
       }
-      if constexpr (stats) part_arrive(ep, m_blk * BM + quarter * 32, lane);
     }
   }
 
@@ -304,11 +299,11 @@ EncodeTiledFn get_encode_fn() {
   return fn;
 }
 
-template <int BN, int STAGES, int KIND, typename OutT, typename ResT, bool FOLD>
+template <int BN, int STAGES, int KIND, typename OutT, typename ResT>
 cudaError_t launch_impl(const GemmArgs& g, const EpiParams& ep, DevError* err, cudaStream_t st, int num_sms,
                         bool prepare_only) {
   using Cf = TcCfg<BN, STAGES>;
-  auto kern = gemm_tc_kernel<BN, STAGES, KIND, OutT, ResT, FOLD>;
+  auto kern = gemm_tc_kernel<BN, STAGES, KIND, OutT, ResT>;
   if (prepare_only)
     return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cf::SMEM);
   CUtensorMap ta, tb;
@@ -318,9 +313,7 @@ cudaError_t launch_impl(const GemmArgs& g, const EpiParams& ep, DevError* err, c
   const int tiles = mt * nt;
   const int grid = tiles < num_sms ? tiles : num_sms;
   const int kb = (g.K + BK - 1) / BK;
-  EpiParams e = ep;
-  e.part_arrivals = EPI_PARTS * nt;   // every epilogue warp of a lane quarter, for every column tile
-  return launch_kernel(kern, dim3(grid), dim3(NUM_THREADS), Cf::SMEM, st, ta, tb, mt, nt, kb, e, err);
+  return launch_kernel(kern, dim3(grid), dim3(NUM_THREADS), Cf::SMEM, st, ta, tb, mt, nt, kb, ep, err);
 }
 
 }  // namespace
@@ -369,41 +362,35 @@ int make_tmap_plain(CUtensorMap* m, const void* base, int elem, int rows, int co
 // residual stream of the post-norm layers is kept in fp32; operands are bf16).
 static cudaError_t dispatch(const GemmArgs& g, int bn, int kind, bool out_f32, const EpiParams& ep, DevError* err,
                             cudaStream_t st, int num_sms, bool prep) {
-  // the folded-LayerNorm instantiation when this launch consumes or produces row statistics
-  const bool fold = ep.fold_g != nullptr || ep.part != nullptr;
-#define KD_TC_ONE(BN_, ST_, KIND_, OUT_, FOLD_)                                          \
-  if (prep) {                                                                          \
-    cudaError_t e_ = launch_impl<BN_, ST_, KIND_, OUT_, float, FOLD_>(g, ep, err, st, num_sms, true); \
-    if (e_ != cudaSuccess) return e_;                                                  \
-  } else if (bn == BN_ && kind == KIND_ && out_f32 == std::is_same<OUT_, float>::value && fold == FOLD_) \
-    return launch_impl<BN_, ST_, KIND_, OUT_, float, FOLD_>(g, ep, err, st, num_sms, false);
-#define KD_TC(BN_, ST_, KIND_, OUT_) KD_TC_ONE(BN_, ST_, KIND_, OUT_, false)
-#define KD_TCF(BN_, ST_, KIND_, OUT_) KD_TC_ONE(BN_, ST_, KIND_, OUT_, false) KD_TC_ONE(BN_, ST_, KIND_, OUT_, true)
-  KD_TCF(256, 4, EPI_BIAS, bf16)
-  KD_TCF(256, 4, EPI_BIAS_GELU, bf16)
-  KD_TCF(256, 4, EPI_BIAS_RESID, float)
-  KD_TCF(256, 4, EPI_BIAS_RESID_LN, float)
+#define KD_TC(BN_, ST_, KIND_, OUT_)                                                            \
+  if (prep) {                                                                                  \
+    cudaError_t e_ = launch_impl<BN_, ST_, KIND_, OUT_, float>(g, ep, err, st, num_sms, true); \
+    if (e_ != cudaSuccess) return e_;                                                          \
+  } else if (bn == BN_ && kind == KIND_ && out_f32 == std::is_same<OUT_, float>::value)         \
+    return launch_impl<BN_, ST_, KIND_, OUT_, float>(g, ep, err, st, num_sms, false);
+  KD_TC(256, 4, EPI_BIAS, bf16)
+  KD_TC(256, 4, EPI_BIAS_GELU, bf16)
+  KD_TC(256, 4, EPI_BIAS_RESID, float)
+  KD_TC(256, 4, EPI_BIAS_RESID_LN, float)
   KD_TC(256, 4, EPI_INPROJ, bf16)
-  KD_TCF(128, 6, EPI_BIAS, bf16)
+  KD_TC(128, 6, EPI_BIAS, bf16)
   KD_TC(128, 6, EPI_BIAS, float)
-  KD_TCF(128, 6, EPI_BIAS_GELU, bf16)
+  KD_TC(128, 6, EPI_BIAS_GELU, bf16)
   KD_TC(128, 6, EPI_BIAS_SILU, bf16)
-  KD_TCF(128, 6, EPI_BIAS_RESID, float)
-  KD_TCF(128, 6, EPI_BIAS_RESID_LN, float)
+  KD_TC(128, 6, EPI_BIAS_RESID, float)
+  KD_TC(128, 6, EPI_BIAS_RESID_LN, float)
   KD_TC(128, 6, EPI_INPROJ, bf16)
-  KD_TCF(128, 6, EPI_OUTPROJ, float)
-  KD_TCF(64, 8, EPI_BIAS, bf16)
-  KD_TCF(64, 8, EPI_BIAS_GELU, bf16)
-  KD_TCF(64, 8, EPI_BIAS_RESID, float)
-  KD_TCF(64, 8, EPI_BIAS_RESID_LN, float)
-  KD_TCF(32, 8, EPI_BIAS, bf16)
-  KD_TCF(32, 8, EPI_BIAS_GELU, bf16)
-  KD_TCF(32, 8, EPI_BIAS_RESID, float)
-  KD_TCF(32, 8, EPI_BIAS_RESID_LN, float)
-  KD_TCF(16, 8, EPI_OUTPROJ, float)
-#undef KD_TCF
+  KD_TC(128, 6, EPI_OUTPROJ, float)
+  KD_TC(64, 8, EPI_BIAS, bf16)
+  KD_TC(64, 8, EPI_BIAS_GELU, bf16)
+  KD_TC(64, 8, EPI_BIAS_RESID, float)
+  KD_TC(64, 8, EPI_BIAS_RESID_LN, float)
+  KD_TC(32, 8, EPI_BIAS, bf16)
+  KD_TC(32, 8, EPI_BIAS_GELU, bf16)
+  KD_TC(32, 8, EPI_BIAS_RESID, float)
+  KD_TC(32, 8, EPI_BIAS_RESID_LN, float)
+  KD_TC(16, 8, EPI_OUTPROJ, float)
 #undef KD_TC
-#undef KD_TC_ONE
   return prep ? cudaSuccess : cudaErrorInvalidValue;
 }
 

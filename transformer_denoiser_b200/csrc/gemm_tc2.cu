@@ -72,9 +72,7 @@ __device__ __forceinline__ void record_timeout(DevError* err, int where, volatil
   }
 }
 
-// FOLD: the folded-LayerNorm instantiation (the bias / GELU kinds consume the row
-// statistics, the residual kinds produce them); the default ones carry none of that code.
-template <int BN, int STAGES, int KIND, typename OutT, bool FOLD>
+template <int BN, int STAGES, int KIND, typename OutT>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const __grid_constant__ CUtensorMap tmO, const __grid_constant__ CUtensorMap tmR,
@@ -231,10 +229,6 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
     int cc = 0;   // chunks processed by this warp so far: staging tile cc & 1
     int local = 0;
     bool failed = false;
-    // folded LayerNorm: the bias / GELU epilogues consume it, the residual ones produce it
-    constexpr bool FOLDABLE = KIND == EPI_BIAS || KIND == EPI_BIAS_GELU;
-    constexpr bool fold = FOLD && FOLDABLE;
-    constexpr bool stats = FOLD && C::RES;
     for (int tile = pair; tile < num_tiles && !failed; tile += npairs, ++local) {
       const int acc = local & 1;
       const uint32_t acc_phase = (local >> 1) & 1;
@@ -250,8 +244,7 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
       const int cc0 = cc;
       auto stage_tile = [&](int a) { return stg_base + (a % C::NBUF) * C::STG_BYTES; };
       // per-column operands of chunk k: bias, and for EPI_BIAS_RESID_LN the LayerNorm gamma and
-      // (bias + beta), so that x = acc + (bias + beta) + (z * rstd - mean * rstd) * gamma; with
-      // a folded LayerNorm (fold) the row sums of the folded weights
+      // (bias + beta), so that x = acc + (bias + beta) + (z * rstd - mean * rstd) * gamma
       auto load_bias = [&](int k, float4 (&b4)[CW / 4], float4 (&g4)[CW / 4]) {
 #pragma unroll
         for (int j = 0; j < CW / 4; ++j) {
@@ -261,15 +254,11 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
             b4[j].x += be.x; b4[j].y += be.y; b4[j].z += be.z; b4[j].w += be.w;
             g4[j] = ld4(ep.ln_g + gcol + k * CW + 4 * j);
           }
-          if constexpr (FOLDABLE) {
-            if constexpr (fold) g4[j] = ld4(ep.fold_g + gcol + k * CW + 4 * j);
-          }
         }
       };
-      // this lane's row statistics for EPI_BIAS_RESID_LN and a folded LayerNorm:
-      // z * rs_a + rs_b = (z - mean) / std
+      // this lane's row statistics for EPI_BIAS_RESID_LN: z * rs_a + rs_b = (z - mean) / std
       float rs_a = 1.f, rs_b = 0.f;
-      if constexpr (KIND == EPI_BIAS_RESID_LN || fold) {
+      if constexpr (KIND == EPI_BIAS_RESID_LN) {
         const int row = row0 + lane;
         if (nch > 0 && row < ep.M) {
           const float2 st2 = *reinterpret_cast<const float2*>(ep.ln_stats + 2 * (long)row);
@@ -305,7 +294,6 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
       };
       if (nch == 0) {
         release();
-        if constexpr (stats) part_arrive(ep, row0, lane);
         continue;
       }
       // finish chunk k (the warp's chunk number cc == cc0 + k) from accumulator values v, bias b4
@@ -316,23 +304,12 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
         uint8_t* srow = st + lane * C::ROW_BYTES;
         const int swz = C::ROW_BYTES == 64 ? (lane >> 1) & 3 : (lane >> 2) & 1;
         float x[CW];
-        if constexpr (fold) {
-          // folded LayerNorm: acc / std - (mean / std) g + (W beta + b)
 #pragma unroll
-          for (int j = 0; j < CW / 4; ++j) {
-            x[4 * j] = fmaf(v[4 * j], rs_a, fmaf(rs_b, g4[j].x, b4[j].x));
-            x[4 * j + 1] = fmaf(v[4 * j + 1], rs_a, fmaf(rs_b, g4[j].y, b4[j].y));
-            x[4 * j + 2] = fmaf(v[4 * j + 2], rs_a, fmaf(rs_b, g4[j].z, b4[j].z));
-            x[4 * j + 3] = fmaf(v[4 * j + 3], rs_a, fmaf(rs_b, g4[j].w, b4[j].w));
-          }
-        } else {
-#pragma unroll
-          for (int j = 0; j < CW / 4; ++j) {
-            x[4 * j] = v[4 * j] + b4[j].x;
-            x[4 * j + 1] = v[4 * j + 1] + b4[j].y;
-            x[4 * j + 2] = v[4 * j + 2] + b4[j].z;
-            x[4 * j + 3] = v[4 * j + 3] + b4[j].w;
-          }
+        for (int j = 0; j < CW / 4; ++j) {
+          x[4 * j] = v[4 * j] + b4[j].x;
+          x[4 * j + 1] = v[4 * j + 1] + b4[j].y;
+          x[4 * j + 2] = v[4 * j + 2] + b4[j].z;
+          x[4 * j + 3] = v[4 * j + 3] + b4[j].w;
         }
         if constexpr (KIND == EPI_BIAS_GELU) {
 #pragma unroll
@@ -353,19 +330,6 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
               r.z = fmaf(r.z, rs_a, rs_b) * g4[u].z; r.w = fmaf(r.w, rs_a, rs_b) * g4[u].w;
             }
             x[4 * u] += r.x; x[4 * u + 1] += r.y; x[4 * u + 2] += r.z; x[4 * u + 3] += r.w;
-          }
-          if constexpr (stats) {
-            // the new sum's bf16 copy (the next GEMM's operand) and its chunk statistics
-            const int row = row0 + lane;
-            if (row < ep.M) {
-              const int col = gcol + k * CW;
-              ep.part[(long)(col >> 4) * ep.M + row] = chunk_stats16(x);
-              uint4* o16 = reinterpret_cast<uint4*>(ep.out16 + (long)row * ep.ldo16 + col);
-              o16[0] = make_uint4(bf16x2_bits(x[0], x[1]), bf16x2_bits(x[2], x[3]), bf16x2_bits(x[4], x[5]),
-                                  bf16x2_bits(x[6], x[7]));
-              o16[1] = make_uint4(bf16x2_bits(x[8], x[9]), bf16x2_bits(x[10], x[11]), bf16x2_bits(x[12], x[13]),
-                                  bf16x2_bits(x[14], x[15]));
-            }
           }
         } else {
           if (lane == 0) ptx::bulk_wait_read<1>();   // store of chunk cc - 2 has read this tile
@@ -413,9 +377,6 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
         if (!process(vb, bb, gb, c + 1)) { failed = true; break; }
       }
       if (failed && !*abort) record_timeout(err, WHERE_GEMM_EPILOGUE, abort);
-      if constexpr (stats) {
-        if (!failed) part_arrive(ep, row0, lane);
-      }
     }
     if (lane == 0) ptx::bulk_wait_all();
     __syncwarp();
@@ -433,12 +394,12 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
 
 // ------------------------------------------------------------------ host side
 
-template <int BN, int STAGES, int KIND, typename OutT, bool FOLD>
+template <int BN, int STAGES, int KIND, typename OutT>
 struct Tc2Launcher {
   static int max_clusters;
   static cudaError_t prepare() {
     using Cf = Tc2Cfg<BN, STAGES, KIND>;
-    auto kern = gemm_tc2_kernel<BN, STAGES, KIND, OutT, FOLD>;
+    auto kern = gemm_tc2_kernel<BN, STAGES, KIND, OutT>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cf::SMEM);
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 0);
@@ -494,14 +455,12 @@ struct Tc2Launcher {
     cfg.stream = st;
     cfg.attrs = attr;
     cfg.numAttrs = pdl_enabled() ? 2 : 1;
-    EpiParams e = ep;
-    e.part_arrivals = 2 * nt;   // both epilogue warps of a lane quarter, for every column tile
-    return cudaLaunchKernelEx(&cfg, gemm_tc2_kernel<BN, STAGES, KIND, OutT, FOLD>, ta, tb, to, tr, mt, nt,
-                              (g.K + BK - 1) / BK, e, err);
+    return cudaLaunchKernelEx(&cfg, gemm_tc2_kernel<BN, STAGES, KIND, OutT>, ta, tb, to, tr, mt, nt,
+                              (g.K + BK - 1) / BK, ep, err);
   }
 };
-template <int BN, int STAGES, int KIND, typename OutT, bool FOLD>
-int Tc2Launcher<BN, STAGES, KIND, OutT, FOLD>::max_clusters = 0;
+template <int BN, int STAGES, int KIND, typename OutT>
+int Tc2Launcher<BN, STAGES, KIND, OutT>::max_clusters = 0;
 
 // (tile N, pipeline stages) per instantiation: stages fill the shared memory left
 // by the epilogue staging tiles
@@ -518,8 +477,7 @@ int Tc2Launcher<BN, STAGES, KIND, OutT, FOLD>::max_clusters = 0;
 cudaError_t gemm_tc2_prepare() {
 #define KD_PREP(BN_, ST_, KIND_, OUT_)                                        \
   {                                                                          \
-    cudaError_t e_ = Tc2Launcher<BN_, ST_, KIND_, OUT_, false>::prepare();   \
-    if (e_ == cudaSuccess) e_ = Tc2Launcher<BN_, ST_, KIND_, OUT_, true>::prepare(); \
+    cudaError_t e_ = Tc2Launcher<BN_, ST_, KIND_, OUT_>::prepare();          \
     if (e_ != cudaSuccess) return e_;                                        \
   }
   KD_TC2_LIST(KD_PREP)
@@ -541,8 +499,8 @@ int gemm_tc2_pick_bn(int M, int N, int kind) {
   const bool res = kind == EPI_BIAS_RESID || kind == EPI_BIAS_RESID_LN;
   const int* cands = res ? resid : all;
   const int ncand = res ? 2 : 4;
-  const int pairs = Tc2Launcher<256, 6, EPI_BIAS, bf16, false>::max_clusters > 0
-                        ? Tc2Launcher<256, 6, EPI_BIAS, bf16, false>::max_clusters : 74;
+  const int pairs = Tc2Launcher<256, 6, EPI_BIAS, bf16>::max_clusters > 0
+                        ? Tc2Launcher<256, 6, EPI_BIAS, bf16>::max_clusters : 74;
   const long mt = (M + 2 * BMC - 1) / (2 * BMC);
   int best = cands[0];
   long best_cost = -1;
@@ -563,12 +521,9 @@ cudaError_t gemm_tc2(const GemmArgs& g, int bn, int kind, bool out_f32, const Ep
                      cudaStream_t st) {
   if (g.M <= 0 || g.N <= 0) return cudaSuccess;
   if (g.K <= 0 || g.N % 16) return cudaErrorInvalidValue;
-  // the folded-LayerNorm instantiation when this launch consumes or produces row statistics
-  const bool fold = ep.fold_g != nullptr || ep.part != nullptr;
-#define KD_RUN(BN_, ST_, KIND_, OUT_)                                                   \
-  if (bn == BN_ && kind == KIND_ && out_f32 == std::is_same<OUT_, float>::value)        \
-    return fold ? Tc2Launcher<BN_, ST_, KIND_, OUT_, true>::launch(g, ep, err, st)      \
-                : Tc2Launcher<BN_, ST_, KIND_, OUT_, false>::launch(g, ep, err, st);
+#define KD_RUN(BN_, ST_, KIND_, OUT_)                                            \
+  if (bn == BN_ && kind == KIND_ && out_f32 == std::is_same<OUT_, float>::value) \
+    return Tc2Launcher<BN_, ST_, KIND_, OUT_>::launch(g, ep, err, st);
   KD_TC2_LIST(KD_RUN)
 #undef KD_RUN
   return cudaErrorInvalidValue;

@@ -17,8 +17,7 @@ struct GemmArgs {
 };
 
 // tcgen05 bf16 GEMM.  bn in {16, 32, 64, 128, 256}; returns cudaErrorInvalidValue for an
-// unsupported (bn, kind, output type) combination.  A launch whose EpiParams carry
-// folded-LayerNorm row statistics (fold_g or part set) runs the folded instantiation.
+// unsupported (bn, kind, output type) combination.
 cudaError_t gemm_tc(const GemmArgs& g, int bn, int kind, bool out_f32, const EpiParams& ep, DevError* err,
                     cudaStream_t st, int num_sms);
 bool gemm_tc_available();
@@ -31,20 +30,9 @@ int make_tmap_bf16(CUtensorMap* m, const void* base, int rows, int cols, int ld,
 int make_tmap_plain(CUtensorMap* m, const void* base, int elem, int rows, int cols, long ld, int box_cols,
                     int box_rows, int swizzle);
 
-// Stream-K tcgen05 GEMM on CTA pairs (256 x 256 tiles, equal k-block shares per pair).
-// Kinds: EPI_BIAS / EPI_BIAS_GELU with bf16 output, EPI_BIAS_RESID with fp32 output
-// (residual read from global memory; may alias the output).  N % 16 == 0.  partial:
-// gemm_sk_workspace_floats() floats; flags: 2 * GEMM_SK_MAX_PAIRS ints, zero before the
-// first launch (each launch leaves them zero).  Launches on one workspace must not overlap.
-constexpr int GEMM_SK_MAX_PAIRS = 80;
-cudaError_t gemm_sk_prepare();
-size_t gemm_sk_workspace_floats();
-cudaError_t gemm_sk(const GemmArgs& g, int kind, bool out_f32, const EpiParams& ep, float* partial, int* flags,
-                    DevError* err, cudaStream_t st);
-
 // tcgen05 GEMM on CTA pairs (256-row tiles).  bn in {144, 160, 208, 256} for EPI_BIAS /
 // EPI_BIAS_GELU with bf16 output, {144, 160} for EPI_BIAS_RESID / EPI_BIAS_RESID_LN with
-// fp32 output; folded-LayerNorm launches as for gemm_tc.
+// fp32 output.
 cudaError_t gemm_tc2(const GemmArgs& g, int bn, int kind, bool out_f32, const EpiParams& ep, DevError* err,
                      cudaStream_t st);
 cudaError_t gemm_tc2_prepare();
@@ -53,23 +41,19 @@ int gemm_tc2_pick_bn(int M, int N, int kind);
 // Set the dynamic shared-memory limits of every kernel instantiation (call once
 // per device before any launch or graph capture).
 cudaError_t gemm_tc_prepare();
-cudaError_t attention_prepare();
-size_t attention_bf16_smem(int S);
 
 // fp32 SIMT GEMM with the same epilogues (fp32 everywhere).  K % 16 == 0.
 cudaError_t gemm_f32(const GemmArgs& g, int kind, const EpiParams& ep, cudaStream_t st);
 
 // Masked multi-head self-attention over the fused QKV matrix (columns Q | K | V,
-// head h at h*DH).  Padded layout (tok0 null): sequence s owns rows s*S .. s*S + S - 1
-// and keys at token index >= 1 + lengths[s % len_mod] are excluded.  Packed layout:
-// sequence s owns rows tok0[s] .. tok0[s + 1] - 1 (its valid tokens only; S is then
-// the largest sequence).  out has the rows of qkv, D columns.
-cudaError_t attention_bf16(const bf16* qkv, bf16* out, const int* lengths, int len_mod, int nseq, int S,
-                           cudaStream_t st, const int* tok0 = nullptr);
+// head h at h*DH), fp32 path.  Padded layout (tok0 null): sequence s owns rows
+// s*S .. s*S + S - 1 and keys at token index >= 1 + lengths[s % len_mod] are excluded.
+// Packed layout: sequence s owns rows tok0[s] .. tok0[s + 1] - 1 (its valid tokens
+// only; S is then the largest sequence).  out has the rows of qkv, D columns.
 cudaError_t attention_f32(const float* qkv, float* out, const int* lengths, int len_mod, int nseq, int S,
                           cudaStream_t st, const int* tok0 = nullptr);
 
-// The same attention on the tcgen05 tensor cores (bf16): one CTA per (head, sequence,
+// The same attention on the tcgen05 tensor cores (bf16 path): one CTA per (head, sequence,
 // 128-query tile), exact softmax over all keys of the sequence at once.  qkv has M
 // rows (16-byte aligned, row stride 3*D); S <= MAX_FRAMES + 1.
 cudaError_t attention_tc(const bf16* qkv, bf16* out, int M, const int* lengths, int len_mod, int nseq, int S,
@@ -82,10 +66,9 @@ size_t attention_tc_smem(int S);
 cudaError_t build_token_map(const int* lengths, int len_mod, int nseq, int* tok0, int* row_seq, cudaStream_t st);
 
 // Row LayerNorm over D features: y fp32 [M, D] -> out (bf16 or fp32) [M, D], and
-// optionally an fp32 copy into out32 (which may be y itself) and the row statistics
-// (mean, 1/std) into stats [M][2].
+// optionally the row statistics (mean, 1/std) into stats [M][2].
 cudaError_t layernorm(const float* y, void* out, bool out_bf16, const float* gamma, const float* beta, int M,
-                      cudaStream_t st, float* out32 = nullptr, float* stats = nullptr);
+                      cudaStream_t st, float* stats = nullptr);
 
 // ---- motion / sampler kernels (element type of the activation matrices: bf16 or fp32)
 

@@ -2,10 +2,9 @@
 // shaders" table: layer normalization; "Model details": post-norm layers).
 // One warp per row: the row (fp32 residual sum) is held in registers, the mean
 // and the biased variance are two warp-shuffle reductions (two passes over the
-// registers), eps = 1e-5; statistics in fp32, output bf16 or fp32, plus an
-// optional fp32 copy that may overwrite the input row in place (the row is read
-// completely into registers before any store) and optional row statistics, from
-// which a later residual epilogue rebuilds the normalised row instead of reading it.
+// registers), eps = 1e-5; statistics in fp32, output bf16 or fp32, and optional
+// row statistics, from which a later residual epilogue rebuilds the normalised row
+// instead of reading it.
 #include <cuda_runtime.h>
 
 #include "common.cuh"
@@ -29,7 +28,7 @@ __device__ __forceinline__ float warp_sum(float v) {
 template <typename OutT>
 __global__ void __launch_bounds__(LN_WARPS * 32, 18) layernorm_kernel(const float* y, OutT* __restrict__ out,
                                                         const float* __restrict__ gamma,
-                                                        const float* __restrict__ beta, int M, float* out32,
+                                                        const float* __restrict__ beta, int M,
                                                         float* __restrict__ stats) {
   ptx::pdl_wait();
   ptx::pdl_trigger();
@@ -65,7 +64,6 @@ __global__ void __launch_bounds__(LN_WARPS * 32, 18) layernorm_kernel(const floa
     const float r1 = (v[4 * i + 1] - mean) * rstd * g.y + b.y;
     const float r2 = (v[4 * i + 2] - mean) * rstd * g.z + b.z;
     const float r3 = (v[4 * i + 3] - mean) * rstd * g.w + b.w;
-    if (out32 != nullptr) *reinterpret_cast<float4*>(out32 + (long)row * D + c) = make_float4(r0, r1, r2, r3);
     if constexpr (sizeof(OutT) == 2) {
       __nv_bfloat162 p0 = __floats2bfloat162_rn(r0, r1), p1 = __floats2bfloat162_rn(r2, r3);
       uint2 u;
@@ -81,14 +79,14 @@ __global__ void __launch_bounds__(LN_WARPS * 32, 18) layernorm_kernel(const floa
 }  // namespace
 
 cudaError_t layernorm(const float* y, void* out, bool out_bf16, const float* gamma, const float* beta, int M,
-                      cudaStream_t st, float* out32, float* stats) {
+                      cudaStream_t st, float* stats) {
   if (M <= 0) return cudaSuccess;
   const int grid = (M + LN_WARPS - 1) / LN_WARPS;
   if (out_bf16)
     return launch_kernel(layernorm_kernel<bf16>, dim3(grid), dim3(LN_WARPS * 32), 0, st, y, static_cast<bf16*>(out), gamma, beta,
-                         M, out32, stats);
+                         M, stats);
   return launch_kernel(layernorm_kernel<float>, dim3(grid), dim3(LN_WARPS * 32), 0, st, y, static_cast<float*>(out), gamma, beta,
-                       M, out32, stats);
+                       M, stats);
 }
 
 }  // namespace kd
