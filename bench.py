@@ -22,6 +22,7 @@ import os
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 
 import numpy as np
@@ -87,11 +88,10 @@ class ClockSampler:
     def __init__(self, device_index: int):
         self.dev = device_index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{device_index}.csv")
+        self.path = os.path.join(tempfile.gettempdir(), f"kimodo_bench_clocks_{os.getpid()}_{device_index}.csv")
 
     def __enter__(self):
         try:
-            os.makedirs(os.path.dirname(self.path), exist_ok=True)
             self.f = open(self.path, "w")
             self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.FIELDS}",
                                           "--format=csv,noheader,nounits", "-lms", "200"],
@@ -168,11 +168,12 @@ def _ncu_traffic():
         return None
 
 
-# Algorithmic work of one denoiser step (both networks; projections per token per
-# network forward, activation bytes per token per layer: QKV 8192, attention 8192,
-# attention output 10240, FFN1 6144, FFN2 12288, two LayerNorms 6144 each).
+# Algorithmic work of one denoiser step (both networks).  FLOPs: the four projections
+# per token per network forward.  Bytes: the bf16 layer weights, read once per network
+# forward, plus the activations: 18,432 bf16 values per token and layer (one read or
+# write of every GEMM operand and output, LayerNorm as its own pass), 36,864 bytes.
 PROJ_FLOP_PER_TOKEN = 268435456
-ACT_BYTES_PER_TOKEN_LAYER = 57344
+ACT_BYTES_PER_TOKEN_LAYER = 36864
 WEIGHT_BYTES_PER_STEP = 2 * 16 * 8388608 * 2
 
 
@@ -188,9 +189,11 @@ def step_roofline(nseq, tokens_per_seq, ms_per_step):
     t_flop = flops / (float(peaks["bf16_tflops"]) * 1e12)
     t_byte = nbytes / (float(peaks["hbm_gbs"]) * 1e9)
     floor = max(t_flop, t_byte)
+    t_weights = WEIGHT_BYTES_PER_STEP / (float(peaks["hbm_gbs"]) * 1e9)
     return {"bound": "tensor" if t_flop >= t_byte else "hbm", "floor_us": round(floor * 1e6, 2),
             "flop": flops, "bytes": nbytes, "achieved_us": round(ms_per_step * 1e3, 2),
             "frac": round(floor / (ms_per_step * 1e-3), 4),
+            "weights_only_frac": round(t_weights / (ms_per_step * 1e-3), 4),
             "peaks": f"{kind} burst bf16 {peaks['bf16_tflops']} TFLOP/s, HBM {peaks['hbm_gbs']} GB/s"}
 
 

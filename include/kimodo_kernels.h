@@ -83,6 +83,22 @@ KIMODO_API int kimodo_attention_f32(const float* qkv, float* out, const int* len
 KIMODO_API int kimodo_layernorm(const float* y, void* out, int out_bf16, const float* gamma,
                                 const float* beta, int M, void* stream);
 
+/*
+ * globalRootToLocalRoot and the body network's input ("Kimodo WebGPU",
+ * "Architecture" figure: root model -> globalRootToLocalRoot -> body model), the
+ * fp32 form of the kernel the two-stage step runs between its two networks.
+ * root: [batch, frames, 5] global root (x, z, sin heading, cos heading, height), the
+ *   root network's output for one guidance branch.  x: [batch, frames, 279] state x_t.
+ * body_in (output): [batch, frames, 279] = [x[..., 5:279] | local root 5], local root =
+ *   (v'x, v'z, sin d, cos d, height): the displacement from the previous frame turned
+ *   into the current heading's frame, the heading change, the height; headings are
+ *   normalised, and the frame before the first sits at the origin with heading 0.
+ *   Frames at index >= lengths[b] get local root 0 (their body columns are copied).
+ * lengths: int32 [batch], 1..frames.  1 <= batch, 1 <= frames <= 300.
+ */
+KIMODO_API int kimodo_global_to_local_root(const float* root, const float* x, const int* lengths, int batch,
+                                           int frames, float* body_in, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -78,7 +78,10 @@ def test_step_roofline_counts():
     assert bench.PROJ_FLOP_PER_TOKEN == 16 * 2 * (3 + 1 + 2 + 2) * 1024 * 1024
     # attention per sequence and layer: QK^T and PV, 2 x 2 x S^2 x 1024 FLOP
     assert r["flop"] == 2 * (tokens * bench.PROJ_FLOP_PER_TOKEN + 16 * 2 * 4 * 181 * 181 * 1024)
-    assert r["bytes"] == 2 * 16 * (8 * 1024 * 1024) * 2 + 2 * 16 * 57344 * tokens
+    # bytes: bf16 layer weights of both networks, and the activation model's 18,432 bf16
+    # values per token and layer, for both networks
+    assert bench.ACT_BYTES_PER_TOKEN_LAYER == 2 * 18432
+    assert r["bytes"] == 2 * 16 * (8 * 1024 * 1024) * 2 + 2 * 16 * 36864 * tokens
     peaks, _ = bench._measured_peaks()
     t_flop = r["flop"] / (float(peaks["bf16_tflops"]) * 1e12)
     t_byte = r["bytes"] / (float(peaks["hbm_gbs"]) * 1e9)

@@ -17,6 +17,7 @@ import synth
 import transformer_denoiser_b200 as kb
 from gpu_fixtures import blob, gpu_bf16, gpu_fp32, max_abs_rel, padded, params, rel_l2, valid  # noqa: F401
 from oracle import kimodo_oracle as ko
+from oracle_jobs import C3, C4, C5, VAR, c5_sequences, workload_inputs
 
 pytestmark = pytest.mark.gpu
 
@@ -110,16 +111,13 @@ def test_bf16_ddim_step_ragged_batch_and_null_broadcast(gpu_bf16, params):
     assert np.all(padded(a, L) == 0)
 
 
-def test_bf16_sample_c3(gpu_bf16, params):
+def test_bf16_sample_c3(gpu_bf16, oracle_refs):
     """50-step generation, B=1, 180 frames, CFG 2.0: trajectory within 5e-2."""
-    B, T, L = 1, 180, [180]
-    noise = synth.noise(B, T)
-    emb = synth.text_embeddings(B)
-    null = np.zeros(4096, np.float32)
-    got = gpu_bf16.ddim_sample(emb, null, noise, np.array(L, np.int32), 50, 2.0)
-    ref = ko.ddim_sample(params, emb[0], null, noise[0], 180, 50, 2.0)
+    emb, null, noise, L = workload_inputs(C3)
+    got = gpu_bf16.ddim_sample(emb, null, noise, L, C3[3], C3[4])
     assert np.all(np.isfinite(got))
-    report("bf16 sample c3 (50 steps, T=180) trajectory rel-L2", rel_l2(got[0], ref), TOL_BF16_TRAJ)
+    report("bf16 sample c3 (50 steps, T=180) trajectory rel-L2", rel_l2(got[0], oracle_refs.result(C3, 0)),
+           TOL_BF16_TRAJ)
 
 
 def test_sample_equals_repeated_steps(gpu_bf16):
@@ -175,47 +173,51 @@ def test_packed_layout_equals_padded_layout(gpu_bf16, gpu_fp32, precision):
     np.testing.assert_array_equal(s1, s2)
 
 
-def test_c4_full_size_sampled(gpu_bf16, params):
+def test_c4_full_size_sampled(gpu_bf16, oracle_refs):
     """100-step generation at B=16, T=150 (the throughput workload, as bench.py
-    runs it): sequence 0 against the oracle over all 100 steps, sequence 15
-    against the same prompt sampled alone, every output finite and padded-free."""
-    B, T = 16, 150
-    L = np.full(B, T, np.int32)
-    noise = synth.noise(B, T)
-    emb = synth.text_embeddings(B)
-    null = np.zeros(4096, np.float32)
-    got = gpu_bf16.ddim_sample(emb, null, noise, L, 100, 2.0)
+    runs it): sequences 0 and 15 against the oracle over all 100 steps, sequence 15
+    also against the same prompt sampled alone; every output finite."""
+    emb, null, noise, L = workload_inputs(C4)
+    got = gpu_bf16.ddim_sample(emb, null, noise, L, C4[3], C4[4])
     assert np.all(np.isfinite(got))
-    alone = gpu_bf16.ddim_sample(emb[15:16], null, noise[15:16], L[15:16], 100, 2.0)
+    alone = gpu_bf16.ddim_sample(emb[15:16], null, noise[15:16], L[15:16], C4[3], C4[4])
     report("c4 seq 15 batched vs alone rel-L2", rel_l2(got[15], alone[0]), 1e-4)
-    ref = ko.ddim_sample(params, emb[0], null, noise[0], T, 100, 2.0)
-    report("bf16 sample c4 seq 0 (100 steps) trajectory rel-L2", rel_l2(got[0], ref), TOL_BF16_TRAJ)
+    for b in (0, 15):
+        report(f"bf16 sample c4 seq {b} (100 steps) trajectory rel-L2", rel_l2(got[b], oracle_refs.result(C4, b)),
+               TOL_BF16_TRAJ)
 
 
-def test_c5_ragged_garbage_sampled(gpu_bf16, params):
+def test_c5_ragged_garbage_sampled(gpu_bf16, oracle_refs):
     """50-step ragged batch, B=64, lengths U{60..300} padded to 300 frames with
-    garbage, CFG 2.5: the shortest sequence against the oracle; garbage, zeros
-    and NaN in the padding give bit-identical results."""
-    B, T = 64, 300
-    L = synth.lengths_uniform(B, 60, 300)
-    noise = synth.noise(B, T)
-    emb = synth.text_embeddings(B)
-    null = np.zeros(4096, np.float32)
-    garbage = synth.fill_padding(noise, L)
-    got = gpu_bf16.ddim_sample(emb, null, garbage, L, 50, 2.5)
+    garbage, CFG 2.5: the shortest, the longest and two seeded random sequences
+    against the oracle; garbage, zeros and NaN in the padding give bit-identical
+    results; the padded token layout agrees with the packed one."""
+    emb, null, garbage, L = workload_inputs(C5)
+    got = gpu_bf16.ddim_sample(emb, null, garbage, L, C5[3], C5[4])
     assert np.all(np.isfinite(got))
     assert np.all(padded(got, L) == 0)
+    noise = synth.noise(C5[1], C5[2])
     zeros = noise.copy()
-    for b in range(B):
+    for b in range(C5[1]):
         zeros[b, L[b]:] = 0
-    np.testing.assert_array_equal(gpu_bf16.ddim_sample(emb, null, zeros, L, 50, 2.5), got)
+    np.testing.assert_array_equal(gpu_bf16.ddim_sample(emb, null, zeros, L, C5[3], C5[4]), got)
     nans = synth.fill_padding(noise, L, nan=True)
-    np.testing.assert_array_equal(gpu_bf16.ddim_sample(emb, null, nans, L, 50, 2.5), got)
+    np.testing.assert_array_equal(gpu_bf16.ddim_sample(emb, null, nans, L, C5[3], C5[4]), got)
     # lengths in device memory: the padded token layout, the same result up to summation order
-    dense = gpu_bf16.ddim_sample(emb, null, garbage, torch.from_numpy(L).cuda(), 50, 2.5)
+    dense = gpu_bf16.ddim_sample(emb, null, garbage, torch.from_numpy(L).cuda(), C5[3], C5[4])
     torch.cuda.synchronize()
     report("bf16 sample c5 padded vs packed layout rel-L2", rel_l2(valid(dense, L), valid(got, L)), 1e-2)
-    b = int(np.argmin(L))
-    ref = ko.ddim_sample(params, emb[b], null, garbage[b], int(L[b]), 50, 2.5)
-    report(f"bf16 sample c5 seq {b} len {L[b]} (50 steps, cfg 2.5) trajectory rel-L2",
-           rel_l2(got[b, :L[b]], ref[:L[b]]), TOL_BF16_TRAJ)
+    for b in c5_sequences():
+        n = int(L[b])
+        report(f"bf16 sample c5 seq {b} len {n} (50 steps, cfg 2.5) trajectory rel-L2",
+               rel_l2(got[b, :n], oracle_refs.result(C5, b)[:n]), TOL_BF16_TRAJ)
+
+
+def test_variations_against_oracle(gpu_bf16, oracle_refs):
+    """Variations of a prompt: 2 prompts x 3 takes with their own noise (text rows shared
+    by the takes), 10 steps; every sequence against the oracle run on its prompt."""
+    prompts, null, noise, L = workload_inputs(VAR)
+    got = gpu_bf16.ddim_sample(prompts, null, noise, L, VAR[3], VAR[4])
+    for b in range(VAR[1]):
+        report(f"bf16 variations seq {b} (prompt {b // 3}) trajectory rel-L2",
+               rel_l2(got[b], oracle_refs.result(VAR, b)), TOL_BF16_TRAJ)

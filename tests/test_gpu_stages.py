@@ -1,0 +1,114 @@
+"""Each stage of one two-stage DDIM step against the oracle, element by element.
+
+The kimodo.cpp parity method ("kimodo.cpp 소개", parity-fixture section) checks every
+boundary of the step separately: root network I/O, global -> local root, body network
+I/O, the guided prediction and DDIM x(t-1).  Here each stage runs through the C ABI on
+the oracle's own input for that stage (so an error in one stage cannot hide in, or be
+blamed on, another), and the 5 root columns are checked apart from the 274 body
+columns, with tolerances of their own: a sign or normalisation error in the root
+transform is a few per cent of the root columns but under a per cent of all 279.
+
+Tolerances: fp32 path max|g - o| / max|o| <= 1e-4 per stage (the global -> local
+transform alone, pure fp32 arithmetic on the same input, 1e-5); bf16 path relative
+L2 <= 2e-2 per stage.  Valid frames only; padded frames must be 0.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import synth
+import transformer_denoiser_b200 as kb
+from gpu_fixtures import blob, gpu_bf16, gpu_fp32, max_abs_rel, padded, params, rel_l2, valid  # noqa: F401
+from oracle import kimodo_oracle as ko
+
+pytestmark = pytest.mark.gpu
+
+AB = ko.alphabar_linear()
+CASES = {  # name: (batch, frames, lengths, seed)
+    "c2": (1, 150, [150], 900),
+    "c2 ragged": (3, 150, [150, 97, 1], 910),
+    "c1": (1, 30, [30], 920),
+    "c1 ragged": (2, 30, [30, 11], 930),
+}
+T_STEP, T_PREV, CFG = 999, 979, 2.0
+
+
+def _inputs(case):
+    B, T, L, seed = CASES[case]
+    x = synth.fill_padding(synth.noise(B, T, seed=seed), L, seed=seed + 1)
+    emb = synth.text_embeddings(B, seed=seed + 2)
+    return x, emb, np.zeros(4096, np.float32), np.array(L, np.int32)
+
+
+def _oracle_stages(params, x, emb, null, L):
+    """two_stage_predict of both guidance branches for every sequence."""
+    return [{"cond": ko.two_stage_predict(params, x[b], emb[b], T_STEP, int(L[b])),
+             "uncond": ko.two_stage_predict(params, x[b], null, T_STEP, int(L[b]))} for b in range(x.shape[0])]
+
+
+def _stack(stages, branch, key, L, T):
+    out = np.zeros((len(stages), T, stages[0][branch][key].shape[1]))
+    for b, s in enumerate(stages):
+        out[b, :L[b]] = s[branch][key][:L[b]]
+    return out
+
+
+def _check(name, got, ref, L, metric, tol):
+    err = metric(valid(got, L), valid(ref, L))
+    print(f"PARITY stage {name}: {err:.3e} (tolerance {tol:.0e})")
+    assert err <= tol, (name, err)
+
+
+@pytest.mark.parametrize("precision,case", [("bf16", "c2"), ("bf16", "c2 ragged"), ("fp32", "c1"),
+                                            ("fp32", "c1 ragged")])
+def test_two_stage_step_stage_by_stage(precision, case, request, params):
+    model = request.getfixturevalue("gpu_" + precision)
+    metric, tol = (rel_l2, 2e-2) if precision == "bf16" else (max_abs_rel, 1e-4)
+    x, emb, null, L = _inputs(case)
+    B, T = x.shape[0], x.shape[1]
+    st = _oracle_stages(params, x, emb, null, L)
+    embs = {"cond": emb, "uncond": np.zeros_like(emb)}
+    for branch in ("cond", "uncond"):
+        # root network I/O
+        root = model.denoiser_forward(kb.NET_ROOT, np.ascontiguousarray(x[..., :5]), embs[branch], T_STEP, L)
+        _check(f"{precision} {case} {branch} root_out", root, _stack(st, branch, "root_out", L, T), L, metric, tol)
+        assert np.all(padded(root, L) == 0)
+        # global -> local root, on the oracle's root output (fp32 kernel, fp32 arithmetic)
+        ref_root = _stack(st, branch, "root_out", L, T).astype(np.float32)
+        body_in = kb.global_to_local_root(torch.from_numpy(ref_root).cuda(), torch.from_numpy(x).cuda(),
+                                          torch.from_numpy(L).cuda()).cpu().numpy()
+        ref_local = _stack(st, branch, "local_root", L, T)
+        _check(f"{precision} {case} {branch} local_root", body_in[..., 274:], ref_local, L, max_abs_rel, 1e-5)
+        np.testing.assert_array_equal(valid(body_in[..., :274], L), valid(x[..., 5:], L))
+        assert np.all(padded(body_in[..., 274:], L) == 0)
+        # the same transform on the GPU's own root output: the chain root -> local root
+        chain = kb.global_to_local_root(torch.from_numpy(root).cuda(), torch.from_numpy(x).cuda(),
+                                        torch.from_numpy(L).cuda()).cpu().numpy()
+        _check(f"{precision} {case} {branch} root -> local_root chain", chain[..., 274:], ref_local, L, metric, tol)
+        # body network I/O, on the oracle's body input
+        ref_body_in = _stack(st, branch, "body_in", L, T).astype(np.float32)
+        body = model.denoiser_forward(kb.NET_BODY, ref_body_in, embs[branch], T_STEP, L)
+        _check(f"{precision} {case} {branch} body_out", body, _stack(st, branch, "body_out", L, T), L, metric, tol)
+        assert np.all(padded(body, L) == 0)
+    # guided prediction (t_prev = -1 returns x0 itself) and x(t-1), root and body columns apart
+    x0_ref = np.zeros((B, T, 279))
+    for b in range(B):
+        x0_ref[b, :L[b]] = ko.cfg_combine(st[b]["cond"]["x0"], st[b]["uncond"]["x0"], CFG)[:L[b]]
+    x0 = model.ddim_step(x, emb, null, L, T_STEP, -1, CFG)
+    assert np.all(padded(x0, L) == 0)
+    _check(f"{precision} {case} guided x0 root columns", x0[..., :5], x0_ref[..., :5], L, metric, tol)
+    _check(f"{precision} {case} guided x0 body columns", x0[..., 5:], x0_ref[..., 5:], L, metric, tol)
+    xp = model.ddim_step(x, emb, null, L, T_STEP, T_PREV, CFG)
+    xp_ref = np.zeros((B, T, 279))
+    for b in range(B):
+        xp_ref[b, :L[b]] = ko.ddim_update(x[b].astype(np.float64), x0_ref[b], AB[T_STEP], AB[T_PREV])[:L[b]]
+    # the prediction-carrying part x_prev - c1 x_t, and x_prev itself
+    c1 = math.sqrt(1 - AB[T_PREV]) / math.sqrt(1 - AB[T_STEP])
+    for cols, what in ((slice(0, 5), "root"), (slice(5, 279), "body")):
+        _check(f"{precision} {case} x(t-1) - c1 x_t {what} columns", (xp - c1 * x)[..., cols],
+               (xp_ref - c1 * x)[..., cols], L, metric, tol)
+        _check(f"{precision} {case} x(t-1) {what} columns", xp[..., cols], xp_ref[..., cols], L, metric,
+               tol if precision == "fp32" else 1e-3)
+    assert np.all(padded(xp, L) == 0)

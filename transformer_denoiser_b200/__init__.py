@@ -46,6 +46,7 @@ SIGNATURES = [
     ("kimodo_attention_bf16", _I, [_P, _P, _P, _I, _I, _P]),
     ("kimodo_attention_f32", _I, [_P, _P, _P, _I, _I, _P]),
     ("kimodo_layernorm", _I, [_P, _P, _I, _P, _P, _I, _P]),
+    ("kimodo_global_to_local_root", _I, [_P, _P, _P, _I, _I, _P, _P]),
 ]
 EPI_BIAS, EPI_BIAS_GELU, EPI_BIAS_SILU, EPI_BIAS_RESID = 0, 1, 2, 3
 
@@ -197,6 +198,17 @@ def layernorm(y, gamma, beta, out_bf16=True):
     out = torch.empty(y.shape, dtype=torch.bfloat16 if out_bf16 else torch.float32, device=y.device)
     _check(lib.kimodo_layernorm(_ptr(y), _ptr(out), int(bool(out_bf16)), _ptr(gamma), _ptr(beta), y.shape[0],
                                 _cur_stream()))
+    return out
+
+
+def global_to_local_root(root, x, lengths):
+    """[x[..., 5:] | globalRootToLocalRoot(root)] (fp32 CUDA tensors root [B, T, 5],
+    x [B, T, 279], int32 lengths [B])."""
+    import torch
+    lib = load_library()
+    B, T = x.shape[0], x.shape[1]
+    out = torch.empty((B, T, MOTION_DIM), dtype=torch.float32, device=x.device)
+    _check(lib.kimodo_global_to_local_root(_ptr(root), _ptr(x), _ptr(lengths), B, T, _ptr(out), _cur_stream()))
     return out
 
 

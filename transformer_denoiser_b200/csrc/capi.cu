@@ -1108,6 +1108,20 @@ int kimodo_layernorm(const float* y, void* out, int out_bf16, const float* gamma
   return KIMODO_OK;
 }
 
+int kimodo_global_to_local_root(const float* root, const float* x, const int* lengths, int batch, int frames,
+                                float* body_in, void* stream) {
+  g_last_error.clear();
+  if (!root || !x || !lengths || !body_in) return set_error(KIMODO_EINVAL, "NULL tensor argument");
+  KD_TRY(check_shape(batch, frames));
+  // The kernel places frame i of sequence s at row s * S + 1 + i of its output matrix
+  // (row s * S is the condition token).  With S = frames and the base one row before
+  // body_in, that row is body_in's row s * frames + i; row 0 itself is never written.
+  float* base = body_in - MOTION_F;
+  KD_CUDA(g2l_body_input(root, x, lengths, batch, batch, frames, frames, base, false, MOTION_F,
+                         static_cast<cudaStream_t>(stream)));
+  return KIMODO_OK;
+}
+
 }  // extern "C"
 
 // ====================================================================== allocation-free forward
