@@ -212,6 +212,15 @@ KIMODO_API int kimodo_ddim_step_ex(kimodo_ctx* ctx, const float* x_t, const floa
  * last check (KIMODO_ETIMEOUT with the kernel named in kimodo_last_error()). */
 KIMODO_API int kimodo_sync_status(kimodo_ctx* ctx, void* stream);
 
+/* Diagnostic of the device error path: enqueue on `stream` one kernel whose bounded
+ * wait, on a barrier that nothing completes, gives up after limit_us microseconds
+ * (1 .. 2000000) and records KIMODO_ETIMEOUT in the context's error word, as the path's
+ * kernels do when one of their waits runs out.  No fault and no unbounded wait occur;
+ * kimodo_sync_status() then reports the timeout ("wait self-test") and clears it, and
+ * the context stays usable.  While the error is recorded, the tensor-core kernels of
+ * calls enqueued after it skip their work. */
+KIMODO_API int kimodo_wait_selftest(kimodo_ctx* ctx, int limit_us, void* stream);
+
 /* Per-kernel-class timing of the next calls (instrumentation, off by default).
  * With enable != 0, every launch is bracketed by CUDA events; kimodo_ddim_sample
  * then captures a fresh, uncached graph whose kernel nodes sit between timing

@@ -179,3 +179,23 @@ def test_text_batch_must_divide_batch(gpu_bf16):
     rc = gpu_bf16._lib.kimodo_ddim_sample_ex(gpu_bf16._ctx, emb.ctypes.data, null.ctypes.data, 1, x.ctypes.data,
                                              L.ctypes.data, B, T, 3, 2.0, ctypes.byref(opts), out.ctypes.data, st)
     assert rc == -1, rc
+
+
+def test_device_timeout_is_reported_and_the_context_recovers(gpu_bf16):
+    """A bounded wait that runs out (kimodo_wait_selftest: a barrier that nothing
+    completes, 2 ms limit) records KIMODO_ETIMEOUT; kimodo_sync_status reports it with
+    the stage's name and clears it; the next call computes what it computed before."""
+    B, T, L = 1, 20, np.array([20], np.int32)
+    x = synth.noise(B, T, seed=491)
+    emb = synth.text_embeddings(B, seed=492)
+    null = np.zeros(4096, np.float32)
+    before = gpu_bf16.ddim_step(x, emb, null, L, 999, 899, 2.0)
+    gpu_bf16.sync_status()
+    gpu_bf16.wait_selftest(2000)
+    with pytest.raises(kb.KimodoError) as e:
+        gpu_bf16.sync_status()
+    assert e.value.status == -5 and "wait self-test" in str(e.value)
+    gpu_bf16.sync_status()                       # cleared
+    after = gpu_bf16.ddim_step(x, emb, null, L, 999, 899, 2.0)
+    gpu_bf16.sync_status()
+    np.testing.assert_array_equal(before, after)

@@ -104,11 +104,15 @@ def test_two_stage_step_stage_by_stage(precision, case, request, params):
     xp_ref = np.zeros((B, T, 279))
     for b in range(B):
         xp_ref[b, :L[b]] = ko.ddim_update(x[b].astype(np.float64), x0_ref[b], AB[T_STEP], AB[T_PREV])[:L[b]]
-    # the prediction-carrying part x_prev - c1 x_t, and x_prev itself
+    # x_prev itself, and on the bf16 path also its prediction-carrying part x_prev - c1 x_t
+    # (on the fp32 path that difference would only magnify the final fp32 rounding of
+    # x_prev, about 1e-7 |x_t|, by |x_t| / |c0 x0|, some hundreds; the guided x0 columns
+    # above already check the prediction at 1e-4)
     c1 = math.sqrt(1 - AB[T_PREV]) / math.sqrt(1 - AB[T_STEP])
     for cols, what in ((slice(0, 5), "root"), (slice(5, 279), "body")):
-        _check(f"{precision} {case} x(t-1) - c1 x_t {what} columns", (xp - c1 * x)[..., cols],
-               (xp_ref - c1 * x)[..., cols], L, metric, tol)
+        if precision == "bf16":
+            _check(f"{precision} {case} x(t-1) - c1 x_t {what} columns", (xp - c1 * x)[..., cols],
+                   (xp_ref - c1 * x)[..., cols], L, metric, tol)
         _check(f"{precision} {case} x(t-1) {what} columns", xp[..., cols], xp_ref[..., cols], L, metric,
                tol if precision == "fp32" else 1e-3)
     assert np.all(padded(xp, L) == 0)

@@ -34,6 +34,7 @@ SIGNATURES = [
     ("kimodo_ddim_step_ex", _I, [_P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _F, _P, _P, _P]),
     ("kimodo_ddim_sample_ex", _I, [_P, _P, _P, _I, _P, _P, _I, _I, _I, _F, _P, _P, _P]),
     ("kimodo_sync_status", _I, [_P, _P]),
+    ("kimodo_wait_selftest", _I, [_P, _I, _P]),
     ("kimodo_profile_enable", _I, [_P, _I]),
     ("kimodo_profile_read", _I, [_P, _I, _P, _P, _P, _P]),
     ("kimodo_last_launch_count", _LL, [_P]),
@@ -301,6 +302,10 @@ class Kimodo:
                                                    _ptr(lengths), B, T, int(steps), float(cfg_scale),
                                                    ctypes.byref(opts), _ptr(out), _stream(stream, noise, out)))
         return out
+
+    def wait_selftest(self, limit_us: int, stream=None):
+        """kimodo_wait_selftest: a kernel whose bounded wait runs out and records a timeout."""
+        _check(self._lib.kimodo_wait_selftest(self._ctx, int(limit_us), stream))
 
     def sync_status(self, stream=None):
         _check(self._lib.kimodo_sync_status(self._ctx, stream))

@@ -16,9 +16,10 @@
 //      and write P in bf16 into the key buffer (dead once S is formed) in the
 //      K-major 128-byte-swizzle layout.  They zero the value rows past the valid
 //      keys inside the MMA's K range, so 0 * garbage cannot occur either.
-//   4. The same thread issues O = P V as two N = 64 halves (K = keys) with each value
-//      half read in place as an MN-major operand, into the TMEM columns S occupied
-//      (up to 256 keys: a 256-column allocation); the softmax warps scale O by 1 / sum
+//   4. The same thread issues O = P V as one N = 128 MMA per 16-key step (K = keys),
+//      the two 64-dimension value halves read in place as one MN-major operand whose
+//      halves lie one leading-byte offset apart, into the TMEM columns S occupied (up
+//      to 256 keys: a 256-column allocation); the softmax warps scale O by 1 / sum
 //      and store the valid query rows in bf16.
 // Rows of the key and value tiles past the sequence belong to other tokens or lie
 // outside the matrix (zero fill) and are masked as above.  Every wait is bounded.

@@ -27,6 +27,7 @@
 #include "common.cuh"
 #include "epilogue.cuh"
 #include "kernels.h"
+#include "ptx.cuh"
 
 using namespace kd;
 
@@ -560,6 +561,32 @@ int stage_lengths(kimodo_ctx* c, const int* lengths, int batch, int frames, cuda
   return KIMODO_OK;
 }
 
+const char* where_name(int where) {
+  switch (where) {
+    case WHERE_GEMM_PRODUCER: return "GEMM TMA producer";
+    case WHERE_GEMM_MMA: return "GEMM MMA issuer";
+    case WHERE_GEMM_EPILOGUE: return "GEMM epilogue";
+    case WHERE_GEMM_DRAIN: return "GEMM MMA drain";
+    case WHERE_ATTENTION: return "attention";
+    case WHERE_WAIT_SELFTEST: return "wait self-test";
+    default: return "unknown stage";
+  }
+}
+
+// One CTA, one thread: a bounded wait on an mbarrier that nothing arrives on, with the
+// same helper and the same error record as the GEMM and attention kernels.
+__global__ void wait_selftest_kernel(DevError* err, unsigned long long limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  const uint32_t b = ptx::smem_u32(&bar);
+  ptx::mbar_init(b, 1);
+  ptx::fence_mbar_init();
+  volatile int abort = 0;
+  if (!ptx::mbar_wait_bounded(b, 0, &abort, limit_ns) && atomicCAS(&err->code, 0, KIMODO_ETIMEOUT) == 0) {
+    err->where = WHERE_WAIT_SELFTEST;
+    err->block = blockIdx.x;
+  }
+}
+
 int finish_outputs(kimodo_ctx* c, const void* out, cudaStream_t st) {
   if (!is_device_memory(out)) {
     KD_CUDA(cudaStreamSynchronize(st));
@@ -567,7 +594,7 @@ int finish_outputs(kimodo_ctx* c, const void* out, cudaStream_t st) {
     KD_CUDA(cudaMemcpy(&h, c->derr, sizeof(h), cudaMemcpyDeviceToHost));
     if (h.code != 0) {
       cudaMemset(c->derr, 0, sizeof(DevError));
-      return set_error(h.code, "device wait timed out in kernel stage %d (block %d)", h.where, h.block);
+      return set_error(h.code, "device wait timed out in %s (block %d)", where_name(h.where), h.block);
     }
   }
   return KIMODO_OK;
@@ -925,8 +952,17 @@ int kimodo_sync_status(kimodo_ctx* c, void* stream) {
   KD_CUDA(cudaMemcpy(&h, c->derr, sizeof(h), cudaMemcpyDeviceToHost));
   if (h.code != 0) {
     KD_CUDA(cudaMemset(c->derr, 0, sizeof(DevError)));
-    return set_error(h.code, "device wait timed out in kernel stage %d (block %d)", h.where, h.block);
+    return set_error(h.code, "device wait timed out in %s (block %d)", where_name(h.where), h.block);
   }
+  return KIMODO_OK;
+}
+
+int kimodo_wait_selftest(kimodo_ctx* c, int limit_us, void* stream) {
+  g_last_error.clear();
+  KD_TRY(check_ctx(c));
+  if (limit_us < 1 || limit_us > 2000000) return set_error(KIMODO_EINVAL, "limit_us must be in [1, 2000000]");
+  wait_selftest_kernel<<<1, 1, 0, static_cast<cudaStream_t>(stream)>>>(c->derr, 1000ull * (unsigned)limit_us);
+  KD_CUDA(cudaGetLastError());
   return KIMODO_OK;
 }
 

@@ -42,6 +42,7 @@ enum DevErrWhere : int {
   WHERE_GEMM_EPILOGUE = 3,
   WHERE_GEMM_DRAIN = 4,
   WHERE_ATTENTION = 5,
+  WHERE_WAIT_SELFTEST = 6,
 };
 
 }  // namespace kd
