@@ -31,6 +31,8 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 WORKLOAD = dict(batch=16, frames=150, steps=100, cfg_scale=2.0)
+# the one-prompt latency workload, for profiling runs only (--workload c3)
+WORKLOAD_C3 = dict(batch=1, frames=180, steps=50, cfg_scale=2.0)
 METRIC = "clips/min (150-frame, 100-step DDIM, B=16) + denoiser % of roofline"
 UNIT = "clips/min"
 L2_FLUSH_BYTES = 256 << 20
@@ -39,8 +41,9 @@ GEMM_FLOP_PER_TOKEN = 268_435_456      # 2 * 16 * (3d^2 + d^2 + 2 d F), per netw
 
 def workload_config(n_gpus):
     w = WORKLOAD
-    return {"workload": f"100-step DDIM two-stage generation, B={w['batch']} prompts x {w['frames']} frames, "
-                        f"CFG {w['cfg_scale']}, cond+uncond batched (32 x 151 tokens per forward)",
+    return {"workload": f"{w['steps']}-step DDIM two-stage generation, B={w['batch']} prompts x {w['frames']} "
+                        f"frames, CFG {w['cfg_scale']}, cond+uncond batched ({2 * w['batch']} x {w['frames'] + 1} "
+                        f"tokens per forward)",
             "batch_per_gpu": w["batch"], "frames": w["frames"], "ddim_steps": w["steps"],
             "cfg_scale": w["cfg_scale"], "global_batch": w["batch"] * n_gpus,
             "parallelism": f"replicas x{n_gpus} (independent prompts per GPU)",
@@ -404,9 +407,9 @@ def run_ours(args, rank, world, local_rank):
     }
     if secondary is not None:
         line["secondary"] = secondary
-    if args.ddim_steps:
-        line["note"] = (f"profiling case: {args.ddim_steps} DDIM steps per generation instead of "
-                        f"{w['steps']}; not a benchmark number")
+    if args.ddim_steps or args.workload != "c4":
+        line["note"] = (f"profiling case: workload {args.workload}, {ddim_steps} DDIM steps per generation; "
+                        f"not a benchmark number")
     if world == 1 and not args.no_cpu_baseline:
         clips, per_step, desc, threads = oracle_sample()
         line["cpu_baseline"] = {"value": round(clips, 6), "unit": UNIT, "cores": threads, "kind": "oracle",
@@ -445,7 +448,12 @@ def main(argv=None):
                     help="skip the c3 latency and c5 ragged-batch measurements")
     ap.add_argument("--ddim-steps", type=int, default=0,
                     help="profiling only: DDIM steps per generation (default: the workload's 100)")
+    ap.add_argument("--workload", choices=["c4", "c3"], default="c4",
+                    help="profiling only: c3 runs the one-prompt 180-frame workload in the timed loop")
     args = ap.parse_args(argv)
+    if args.workload == "c3":
+        WORKLOAD.update(WORKLOAD_C3)
+        args.no_secondary = True
     rank = int(os.environ.get("RANK", 0))
     world = int(os.environ.get("WORLD_SIZE", 1))
     local_rank = int(os.environ.get("LOCAL_RANK", 0))

@@ -81,6 +81,11 @@ def test_kernel_entry_argument_checks(lib):
     assert b"not built" in lib.kimodo_last_error()
     assert lib.kimodo_gemm_bf16(p, 64, p, 64, p, None, 0, p, 64, 1, 64, 64, 0, 1, 64, None) == -1  # fp32 bias
     assert b"not built" in lib.kimodo_last_error()
+    # pair GEMM: N a multiple of 16; tile_n 144, 160, 208, 256 or 0
+    assert lib.kimodo_gemm_bf16_pair(p, 64, p, 64, p, None, 0, p, 64, 1, 40, 64, 0, 0, 0, None) == -1
+    assert b"N % 16" in lib.kimodo_last_error()
+    assert lib.kimodo_gemm_bf16_pair(p, 64, p, 64, p, None, 0, p, 64, 1, 64, 64, 0, 0, 48, None) == -1
+    assert b"tile_n must be" in lib.kimodo_last_error()
     assert lib.kimodo_attention_bf16(p, p, p, 1, 302, None) == -1
     assert lib.kimodo_layernorm(p, p, 1, p, p, 0, None) == -1
 

@@ -59,6 +59,14 @@ int set_error(int code, const char* fmt, ...) {
     if (s_ != KIMODO_OK) return s_; \
   } while (0)
 
+#ifndef KD_SAMPLE_GROUPS
+#define KD_SAMPLE_GROUPS 2
+#endif
+constexpr int SAMPLE_GROUPS = KD_SAMPLE_GROUPS;
+// a call is split into prompt groups only when each group keeps at least this many token
+// rows per network forward (below it the kernels are latency-bound and splitting adds launches)
+constexpr int GROUP_MIN_ROWS = 1024;
+
 enum LaunchClass { CLS_GEMM_TC = 0, CLS_ATTN = 1, CLS_LN = 2, CLS_MOTION = 3, CLS_GEMM_F32 = 4, CLS_SETUP = 5,
                    NUM_CLS = 8 };
 
@@ -125,6 +133,13 @@ struct kimodo_ctx {
   long long launches = 0;
   long long last_launches = 0;
   Tokens tk;                    // token layout of the call being enqueued
+  // Prompt groups of the sampler: the prompts of a large call are split into
+  // SAMPLE_GROUPS halves whose whole sampling loops run as independent branches of the
+  // graph (own workspace, own stream), so that one group's kernels fill the SMs the
+  // other's leave idle (tails of the GEMMs, attention, LayerNorm).
+  Workspace gws[SAMPLE_GROUPS];
+  cudaStream_t gst[SAMPLE_GROUPS] = {};
+  cudaEvent_t gev[SAMPLE_GROUPS + 1] = {};
   bool bf16() const { return precision == KIMODO_BF16; }
   size_t elem() const { return bf16() ? 2 : 4; }
 };
@@ -286,18 +301,20 @@ void free_graphs(kimodo_ctx* c) {
   c->graphs.clear();
 }
 
-int ensure_workspace(kimodo_ctx* c, int nseq, int frames, int steps) {
+// Grows workspace w to hold nseq sequences of `frames` frames and `steps` timestep rows;
+// *grown tells whether it was (re)allocated, which invalidates graphs captured on it.
+int alloc_workspace(kimodo_ctx* c, Workspace& w, int nseq, int frames, int steps, bool* grown) {
   const int S = frames + 1;
   const int rows = nseq * S;
-  Workspace& w = c->ws;
+  *grown = false;
   if (w.arena && rows <= w.cap_rows && nseq <= w.cap_seq && frames <= w.cap_frames && steps <= w.cap_steps)
     return KIMODO_OK;
+  *grown = true;
   const int R = rows > w.cap_rows ? rows : w.cap_rows;
   const int NS = nseq > w.cap_seq ? nseq : w.cap_seq;
   const int TF = frames > w.cap_frames ? frames : w.cap_frames;
   const int ST = steps > w.cap_steps ? steps : w.cap_steps;
   const int R2 = NS * (TF + 1) > R ? NS * (TF + 1) : R;
-  free_graphs(c);
   if (w.arena) cudaFree(w.arena);
   w = Workspace();
   const size_t e = c->elem();
@@ -333,6 +350,13 @@ int ensure_workspace(kimodo_ctx* c, int nseq, int frames, int steps) {
   }
   w.cap_rows = R2; w.cap_seq = NS; w.cap_frames = TF; w.cap_steps = ST;
   return KIMODO_OK;
+}
+
+int ensure_workspace(kimodo_ctx* c, int nseq, int frames, int steps) {
+  bool grown = false;
+  const int r = alloc_workspace(c, c->ws, nseq, frames, steps, &grown);
+  if (grown) free_graphs(c);
+  return r;
 }
 
 // ------------------------------------------------------------------ forward pieces
@@ -713,6 +737,12 @@ void kimodo_free(kimodo_ctx* c) {
   free_graphs(c);
   for (auto e : c->ev_pool) cudaEventDestroy(e);
   if (c->ws.arena) cudaFree(c->ws.arena);
+  for (int g = 0; g < SAMPLE_GROUPS; ++g) {
+    if (c->gws[g].arena) cudaFree(c->gws[g].arena);
+    if (c->gst[g]) cudaStreamDestroy(c->gst[g]);
+  }
+  for (int i = 0; i <= SAMPLE_GROUPS; ++i)
+    if (c->gev[i]) cudaEventDestroy(c->gev[i]);
   if (c->zbuf) cudaFree(c->zbuf);
   if (c->warena) cudaFree(c->warena);
   if (c->pe) cudaFree(c->pe);
@@ -840,8 +870,11 @@ int kimodo_ddim_step_ex(kimodo_ctx* c, const float* x_t, const float* text_emb, 
   return finish_outputs(c, x_prev, st);
 }
 
-static int enqueue_sample(kimodo_ctx* c, int batch, int frames, int steps, float cfg, int null_batch,
-                          const Sampler& smp, cudaStream_t st) {
+// The sampling loop of `batch` prompts on the current workspace: set-up, then `steps`
+// two-stage steps.  Step draws z (eta > 0) are read at prompt offset b0 of a call of
+// batch_all prompts ([steps, batch_all, frames, 279]).
+static int enqueue_loop(kimodo_ctx* c, int batch, int frames, int steps, float cfg, int null_batch,
+                        const Sampler& smp, int b0, int batch_all, cudaStream_t st) {
   Workspace& w = c->ws;
   KD_TRY(enqueue_token_map(c, batch, 2 * batch, st));
   KD_TRY(launch(c, CLS_SETUP, 0, (double)2 * batch * DTXT * 6, st, "pack_embeddings", [&] {
@@ -851,13 +884,72 @@ static int enqueue_sample(kimodo_ctx* c, int batch, int frames, int steps, float
   KD_TRY(condition_setup(c, 0, 2 * batch, steps, st));
   KD_TRY(condition_setup(c, 1, 2 * batch, steps, st));
   KD_TRY(pack_root_input(c, batch, 2 * batch, frames, st));
-  const size_t zstep = (size_t)batch * frames * MOTION_F;
+  const size_t zstep = (size_t)batch_all * frames * MOTION_F;
   for (int k = 0; k < steps; ++k) {
-    const float* z = smp.z ? smp.z + k * zstep : nullptr;
+    const float* z = smp.z ? smp.z + k * zstep + (size_t)b0 * frames * MOTION_F : nullptr;
     KD_TRY(two_stage_step(c, batch, frames, trailing_t(k, steps), trailing_t(k + 1, steps), cfg, k, k + 1 < steps,
                           smp, z, st));
   }
   return KIMODO_OK;
+}
+
+// Prompt groups for a call: SAMPLE_GROUPS when the prompts split evenly (takes of one
+// prompt stay together) and every group keeps GROUP_MIN_ROWS token rows, else 1.
+static int sample_groups(const kimodo_ctx* c, int batch, const Sampler& smp) {
+  if (SAMPLE_GROUPS < 2 || c->profiling || batch % SAMPLE_GROUPS) return 1;
+  const int bg = batch / SAMPLE_GROUPS;
+  if (bg % smp.takes) return 1;
+  return 2 * bg * (c->tk.M / (2 * batch)) >= GROUP_MIN_ROWS ? SAMPLE_GROUPS : 1;
+}
+
+static int ensure_group_resources(kimodo_ctx* c, int groups, int batch, int frames, int steps) {
+  for (int g = 0; g < groups; ++g) {
+    bool grown = false;
+    KD_TRY(alloc_workspace(c, c->gws[g], 2 * (batch / groups), frames, steps, &grown));
+    if (grown) free_graphs(c);
+    if (!c->gst[g] && cudaStreamCreateWithFlags(&c->gst[g], cudaStreamNonBlocking) != cudaSuccess)
+      return set_error(KIMODO_ECUDA, "stream creation failed");
+  }
+  for (int i = 0; i <= groups; ++i)
+    if (!c->gev[i] && cudaEventCreateWithFlags(&c->gev[i], cudaEventDisableTiming) != cudaSuccess)
+      return set_error(KIMODO_ECUDA, "event creation failed");
+  return KIMODO_OK;
+}
+
+// The whole sampling call.  With prompt groups, each group's loop is enqueued on its own
+// stream (forked from st and joined back, so a capture on st records them as parallel
+// graph branches) on its own workspace; the state x, lengths and embedding staging are
+// the call's, viewed at the group's prompt offset.
+static int enqueue_sample(kimodo_ctx* c, int batch, int frames, int steps, float cfg, int null_batch,
+                          const Sampler& smp, const int* lengths, cudaStream_t st) {
+  const int groups = sample_groups(c, batch, smp);
+  if (groups == 1) return enqueue_loop(c, batch, frames, steps, cfg, null_batch, smp, 0, batch, st);
+  const Workspace main_ws = c->ws;
+  const Tokens main_tk = c->tk;
+  const int bg = batch / groups;
+  KD_CUDA(cudaEventRecord(c->gev[0], st));
+  int r = KIMODO_OK;
+  for (int g = 0; g < groups && r == KIMODO_OK; ++g) {
+    const int b0 = g * bg;
+    Workspace w = c->gws[g];
+    w.x = main_ws.x + (size_t)b0 * frames * MOTION_F;
+    w.lengths = main_ws.lengths + b0;
+    w.st_text = main_ws.st_text + (size_t)(b0 / smp.takes) * DTXT;
+    w.st_null = main_ws.st_null + (null_batch == 1 ? 0 : (size_t)b0 * DTXT);
+    c->ws = w;
+    c->tk = plan_tokens(lengths + b0, bg, 2 * bg, frames);
+    if (cudaStreamWaitEvent(c->gst[g], c->gev[0], 0) != cudaSuccess) {
+      r = set_error(KIMODO_ECUDA, "stream fork failed");
+      break;
+    }
+    r = enqueue_loop(c, bg, frames, steps, cfg, null_batch == 1 ? 1 : bg, smp, b0, batch, c->gst[g]);
+    if (r == KIMODO_OK && (cudaEventRecord(c->gev[1 + g], c->gst[g]) != cudaSuccess ||
+                           cudaStreamWaitEvent(st, c->gev[1 + g], 0) != cudaSuccess))
+      r = set_error(KIMODO_ECUDA, "stream join failed");
+  }
+  c->ws = main_ws;
+  c->tk = main_tk;
+  return r;
 }
 
 int kimodo_ddim_sample(kimodo_ctx* c, const float* text_emb, const float* null_emb, int null_batch,
@@ -885,6 +977,9 @@ int kimodo_ddim_sample_ex(kimodo_ctx* c, const float* text_emb, const float* nul
   Workspace& w = c->ws;
   KD_TRY(stage_lengths(c, lengths, batch, frames, st));
   c->tk = plan_tokens(lengths, batch, 2 * batch, frames);
+  // the prompt groups' workspaces and streams exist before any capture begins
+  const int groups = sample_groups(c, batch, smp);
+  if (groups > 1) KD_TRY(ensure_group_resources(c, groups, batch, frames, steps));
   KD_CUDA(cudaMemcpyAsync(w.x, noise, (size_t)batch * frames * MOTION_F * 4, cudaMemcpyDefault, st));
   KD_CUDA(cudaMemcpyAsync(w.st_text, text_emb, (size_t)(batch / smp.takes) * DTXT * 4, cudaMemcpyDefault, st));
   KD_CUDA(cudaMemcpyAsync(w.st_null, null_emb, (size_t)null_batch * DTXT * 4, cudaMemcpyDefault, st));
@@ -895,7 +990,7 @@ int kimodo_ddim_sample_ex(kimodo_ctx* c, const float* text_emb, const float* nul
     // The graph is not cached: its event nodes belong to this profile.
     KD_CUDA(cudaStreamBeginCapture(c->cap_stream, cudaStreamCaptureModeThreadLocal));
     c->prof_flags = cudaEventRecordExternal;
-    int s = enqueue_sample(c, batch, frames, steps, cfg_scale, null_batch, smp, c->cap_stream);
+    int s = enqueue_sample(c, batch, frames, steps, cfg_scale, null_batch, smp, lengths, c->cap_stream);
     c->prof_flags = cudaEventRecordDefault;
     cudaGraph_t g = nullptr;
     cudaError_t e = cudaStreamEndCapture(c->cap_stream, &g);
@@ -923,7 +1018,7 @@ int kimodo_ddim_sample_ex(kimodo_ctx* c, const float* text_emb, const float* nul
     if (it == c->graphs.end()) {
       KD_CUDA(cudaStreamBeginCapture(c->cap_stream, cudaStreamCaptureModeThreadLocal));
       const long long lc = c->launches;
-      int s = enqueue_sample(c, batch, frames, steps, cfg_scale, null_batch, smp, c->cap_stream);
+      int s = enqueue_sample(c, batch, frames, steps, cfg_scale, null_batch, smp, lengths, c->cap_stream);
       cudaGraph_t g = nullptr;
       cudaError_t e = cudaStreamEndCapture(c->cap_stream, &g);
       if (s != KIMODO_OK) {
