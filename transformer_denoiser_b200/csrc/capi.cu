@@ -212,6 +212,12 @@ int gemm(kimodo_ctx* c, const void* A, int lda, const void* W, int ldw, int M, i
       return launch(c, cls_override >= 0 ? cls_override : CLS_GEMM_TC, flops, bytes, st, "gemm_tc2",
                     [&] { return gemm_tc2(g, bn, kind, out_f32, ep, c->derr, st); });
     }
+    // a few hundred tokens: the layer projections split K over a cluster (the MMA chain
+    // of a full-K tile, not the bytes, would set the time)
+    if (M < 1024 && gemm_splitk_supports(kind, out_f32) && gemm_splitk_factor(N, K) >= 2) {
+      return launch(c, cls_override >= 0 ? cls_override : CLS_GEMM_TC, flops, bytes, st, "gemm_splitk",
+                    [&] { return gemm_splitk(g, kind, out_f32, ep, c->derr, st); });
+    }
     const int bn = pick_bn(c, M, N, kind, out_f32);
     return launch(c, cls_override >= 0 ? cls_override : CLS_GEMM_TC, flops, bytes, st, "gemm_tc",
                   [&] { return gemm_tc(g, bn, kind, out_f32, ep, c->derr, st, c->num_sms); });
@@ -493,6 +499,69 @@ struct Sampler {
   int takes = 1;              // sequences per text-embedding row (variations of one prompt)
 };
 
+// Guidance branches of a small step: when the cond and uncond sequences of a step hold
+// fewer than BRANCH_MAX_ROWS token rows in all (one or a few prompts), the two branches'
+// root network, global-to-local transform and body network run as two parallel chains
+// (own activation workspace, own stream, forked from and joined back to the step's
+// stream), since every kernel at that size leaves most SMs idle; CFG and DDIM follow the
+// join.  Padded token layout only.
+constexpr int BRANCH_MAX_ROWS = 1024;
+
+bool use_branches(const kimodo_ctx* c, int B, int T) {
+  return SAMPLE_GROUPS >= 2 && !c->profiling && !c->tk.packed && 2 * B * (T + 1) < BRANCH_MAX_ROWS;
+}
+
+int ensure_branch_resources(kimodo_ctx* c, int B, int frames) {
+  for (int g = 0; g < 2; ++g) {
+    bool grown = false;
+    KD_TRY(alloc_workspace(c, c->gws[g], B, frames, 1, &grown));
+    if (grown) free_graphs(c);
+    if (!c->gst[g] && cudaStreamCreateWithFlags(&c->gst[g], cudaStreamNonBlocking) != cudaSuccess)
+      return set_error(KIMODO_ECUDA, "stream creation failed");
+  }
+  for (int i = 0; i < 3; ++i)
+    if (!c->gev[i] && cudaEventCreateWithFlags(&c->gev[i], cudaEventDisableTiming) != cudaSuccess)
+      return set_error(KIMODO_ECUDA, "event creation failed");
+  return KIMODO_OK;
+}
+
+// The networks of both guidance branches of one step, branch g (0 cond, 1 uncond) on
+// stream gst[g] with workspace gws[g]; the inputs, predictions and the state stay in the
+// step's workspace (branch g's sequences are its rows g B .. g B + B - 1).
+int branch_nets(kimodo_ctx* c, int B, int T, int k_row, cudaStream_t st) {
+  const Workspace main_ws = c->ws;
+  const int S = T + 1;
+  const size_t e = c->elem();
+  const double eb = (double)e;
+  KD_CUDA(cudaEventRecord(c->gev[0], st));
+  int r = KIMODO_OK;
+  for (int g = 0; g < 2 && r == KIMODO_OK; ++g) {
+    cudaStream_t bs = c->gst[g];
+    Workspace wb = c->gws[g];
+    wb.lengths = main_ws.lengths;
+    c->ws = wb;
+    const size_t s0 = (size_t)g * B;
+    const void* A_root = static_cast<const char*>(main_ws.A_root) + s0 * S * ROOT_IN_LD * e;
+    void* A_body = static_cast<char*>(main_ws.A_body) + s0 * S * BODY_IN_LD * e;
+    float* rh = main_ws.root_hat + s0 * T * ROOT_F;
+    float* bh = main_ws.body_hat + s0 * T * BODY_F;
+    if (cudaStreamWaitEvent(bs, c->gev[0], 0) != cudaSuccess) r = set_error(KIMODO_ECUDA, "stream fork failed");
+    if (r == KIMODO_OK)
+      r = run_net(c, 0, B, T, B, A_root, main_ws.tmlp[0] + (long)k_row * D, main_ws.txt[0] + s0 * D, rh, bs);
+    if (r == KIMODO_OK)
+      r = launch(c, CLS_MOTION, 0, (double)B * T * (ROOT_F * 4 + MOTION_F * (4 + eb)), bs, "g2l_body_input", [&] {
+        return g2l_body_input(rh, main_ws.x, main_ws.lengths, B, B, T, S, A_body, c->bf16(), BODY_IN_LD, bs);
+      });
+    if (r == KIMODO_OK)
+      r = run_net(c, 1, B, T, B, A_body, main_ws.tmlp[1] + (long)k_row * D, main_ws.txt[1] + s0 * D, bh, bs);
+    if (r == KIMODO_OK && (cudaEventRecord(c->gev[1 + g], bs) != cudaSuccess ||
+                           cudaStreamWaitEvent(st, c->gev[1 + g], 0) != cudaSuccess))
+      r = set_error(KIMODO_ECUDA, "stream join failed");
+  }
+  c->ws = main_ws;
+  return r;
+}
+
 // One two-stage step for B prompts (cond rows 0..B-1, uncond rows B..2B-1).
 // Reads ws.x, writes ws.x.  tvec_root / tvec_body are the timestep-MLP rows.
 int two_stage_step(kimodo_ctx* c, int B, int T, int t, int t_prev, float w_cfg, int k_row, bool pack_next,
@@ -500,12 +569,17 @@ int two_stage_step(kimodo_ctx* c, int B, int T, int t, int t_prev, float w_cfg, 
   Workspace& w = c->ws;
   const int nseq = 2 * B, S = T + 1;
   const double eb = (double)c->elem();
-  KD_TRY(run_net(c, 0, nseq, T, B, w.A_root, w.tmlp[0] + (long)k_row * D, w.txt[0], w.root_hat, st));
-  KD_TRY(launch(c, CLS_MOTION, 0, (double)nseq * T * (ROOT_F * 4 + MOTION_F * (4 + eb)), st, "g2l_body_input", [&] {
-    return g2l_body_input(w.root_hat, w.x, w.lengths, B, nseq, T, S, w.A_body, c->bf16(), BODY_IN_LD, st,
-                          c->tk.packed ? w.tok0 : nullptr);
-  }));
-  KD_TRY(run_net(c, 1, nseq, T, B, w.A_body, w.tmlp[1] + (long)k_row * D, w.txt[1], w.body_hat, st));
+  if (use_branches(c, B, T)) {
+    KD_TRY(branch_nets(c, B, T, k_row, st));
+  } else {
+    KD_TRY(run_net(c, 0, nseq, T, B, w.A_root, w.tmlp[0] + (long)k_row * D, w.txt[0], w.root_hat, st));
+    KD_TRY(launch(c, CLS_MOTION, 0, (double)nseq * T * (ROOT_F * 4 + MOTION_F * (4 + eb)), st, "g2l_body_input",
+                  [&] {
+                    return g2l_body_input(w.root_hat, w.x, w.lengths, B, nseq, T, S, w.A_body, c->bf16(),
+                                          BODY_IN_LD, st, c->tk.packed ? w.tok0 : nullptr);
+                  }));
+    KD_TRY(run_net(c, 1, nseq, T, B, w.A_body, w.tmlp[1] + (long)k_row * D, w.txt[1], w.body_hat, st));
+  }
   float c0, c1, c2;
   ddim_coeffs(c, smp.schedule, t, t_prev, smp.eta, &c0, &c1, &c2);
   const float* z = c2 != 0.f ? z_step : nullptr;
@@ -656,7 +730,8 @@ int kimodo_load_weights(kimodo_ctx** out_ctx, const float* host_blob, size_t n_f
   if (precision == KIMODO_BF16 && !gemm_tc_available())
     return set_error(KIMODO_EUNSUPPORTED, "cuTensorMapEncodeTiled is unavailable in this driver");
 
-  if (gemm_tc_prepare() != cudaSuccess || gemm_tc2_prepare() != cudaSuccess || attention_tc_prepare() != cudaSuccess) {
+  if (gemm_tc_prepare() != cudaSuccess || gemm_tc2_prepare() != cudaSuccess || gemm_splitk_prepare() != cudaSuccess ||
+      attention_tc_prepare() != cudaSuccess) {
     cudaGetLastError();
     return set_error(KIMODO_EUNSUPPORTED, "kernel attributes could not be set on device %d", device);
   }
@@ -853,6 +928,7 @@ int kimodo_ddim_step_ex(kimodo_ctx* c, const float* x_t, const float* text_emb, 
   Workspace& w = c->ws;
   KD_TRY(stage_lengths(c, lengths, batch, frames, st));
   c->tk = plan_tokens(lengths, batch, 2 * batch, frames);
+  if (use_branches(c, batch, frames)) KD_TRY(ensure_branch_resources(c, batch, frames));
   KD_TRY(enqueue_token_map(c, batch, 2 * batch, st));
   KD_CUDA(cudaMemcpyAsync(w.x, x_t, (size_t)batch * frames * MOTION_F * 4, cudaMemcpyDefault, st));
   KD_CUDA(cudaMemcpyAsync(w.st_text, text_emb, (size_t)(batch / smp.takes) * DTXT * 4, cudaMemcpyDefault, st));
@@ -980,6 +1056,7 @@ int kimodo_ddim_sample_ex(kimodo_ctx* c, const float* text_emb, const float* nul
   // the prompt groups' workspaces and streams exist before any capture begins
   const int groups = sample_groups(c, batch, smp);
   if (groups > 1) KD_TRY(ensure_group_resources(c, groups, batch, frames, steps));
+  if (use_branches(c, batch, frames)) KD_TRY(ensure_branch_resources(c, batch, frames));
   KD_CUDA(cudaMemcpyAsync(w.x, noise, (size_t)batch * frames * MOTION_F * 4, cudaMemcpyDefault, st));
   KD_CUDA(cudaMemcpyAsync(w.st_text, text_emb, (size_t)(batch / smp.takes) * DTXT * 4, cudaMemcpyDefault, st));
   KD_CUDA(cudaMemcpyAsync(w.st_null, null_emb, (size_t)null_batch * DTXT * 4, cudaMemcpyDefault, st));
@@ -1120,6 +1197,7 @@ int prepared_device() {
   if (!done[dev]) {
     KD_CUDA(gemm_tc_prepare());
     KD_CUDA(gemm_tc2_prepare());
+    KD_CUDA(gemm_splitk_prepare());
     KD_CUDA(attention_tc_prepare());
     done[dev] = true;
   }
@@ -1195,6 +1273,29 @@ int kimodo_gemm_bf16_pair(const void* A, int lda, const void* W, int ldw, const 
   ep.bias = bias; ep.out = out; ep.ldo = ldo; ep.resid = resid; ep.ldr = ldr; ep.N = N; ep.M = M;
   const int bn = tile_n ? tile_n : gemm_tc2_pick_bn(M, N, epilogue);
   KD_CUDA(gemm_tc2(g, bn, epilogue, out_f32 != 0, ep, kernel_error_word(), static_cast<cudaStream_t>(stream)));
+  return KIMODO_OK;
+}
+
+int kimodo_gemm_bf16_splitk(const void* A, int lda, const void* W, int ldw, const float* bias, const void* resid,
+                            int ldr, void* out, int ldo, int M, int N, int K, int epilogue, int out_f32,
+                            void* stream) {
+  g_last_error.clear();
+  KD_TRY(check_gemm_args(A, lda, W, ldw, bias, resid, out, ldo, M, N, K, epilogue));
+  if (lda % 8 || ldw % 8 || (reinterpret_cast<uintptr_t>(A) & 15) || (reinterpret_cast<uintptr_t>(W) & 15))
+    return set_error(KIMODO_EINVAL, "bf16 operands need 16-byte aligned rows (lda, ldw multiples of 8)");
+  if (ldo % 4 || (reinterpret_cast<uintptr_t>(out) & 15) || (epilogue == 3 && (ldr % 4 ||
+      (reinterpret_cast<uintptr_t>(resid) & 15))) || (reinterpret_cast<uintptr_t>(bias) & 15))
+    return set_error(KIMODO_EINVAL, "out, resid and bias need 16-byte alignment and ldo, ldr multiples of 4");
+  if (!gemm_splitk_supports(epilogue, out_f32 != 0))
+    return set_error(KIMODO_EINVAL, "split-K epilogues: bias or GELU with bf16 output, residual with fp32 output");
+  if (gemm_splitk_factor(N, K) < 2)
+    return set_error(KIMODO_EINVAL, "split-K GEMM needs N % 256 == 0 and K / 256 in 2..8");
+  KD_TRY(prepared_device());
+  GemmArgs g;
+  g.A = A; g.B = W; g.M = M; g.N = N; g.K = K; g.lda = lda; g.ldb = ldw;
+  EpiParams ep;
+  ep.bias = bias; ep.out = out; ep.ldo = ldo; ep.resid = resid; ep.ldr = ldr; ep.N = N; ep.M = M;
+  KD_CUDA(gemm_splitk(g, epilogue, out_f32 != 0, ep, kernel_error_word(), static_cast<cudaStream_t>(stream)));
   return KIMODO_OK;
 }
 
