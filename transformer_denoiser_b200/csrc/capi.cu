@@ -64,8 +64,9 @@ int set_error(int code, const char* fmt, ...) {
 #endif
 constexpr int SAMPLE_GROUPS = KD_SAMPLE_GROUPS;
 // a call is split into prompt groups only when each group keeps at least this many token
-// rows per network forward (below it the kernels are latency-bound and splitting adds launches)
-constexpr int GROUP_MIN_ROWS = 1024;
+// rows per network forward: measured, 64 ragged prompts (about 11,600 rows per group) run 8 %
+// faster in two groups, 16 prompts of 150 frames (2,416 rows per group) 11 % slower
+constexpr int GROUP_MIN_ROWS = 8192;
 
 enum LaunchClass { CLS_GEMM_TC = 0, CLS_ATTN = 1, CLS_LN = 2, CLS_MOTION = 3, CLS_GEMM_F32 = 4, CLS_SETUP = 5,
                    NUM_CLS = 8 };
