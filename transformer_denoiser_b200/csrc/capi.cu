@@ -90,6 +90,9 @@ struct Workspace {
   int* lengths = nullptr; float* st_text = nullptr; float* st_null = nullptr;
   int* tok0 = nullptr; int* row_seq = nullptr;   // packed token layout (valid tokens only)
   float* stats[2] = {};                           // LayerNorm row statistics (mean, 1/std) [M][2]
+  int* flow = nullptr;                            // row-block dataflow counters [FLOW_EVENTS][flow_stride]
+  int flow_stride = 0;
+  int flow_epoch = 0;                             // host: layer epochs enqueued since the counters were zeroed
 };
 
 // Token rows of a call: the padded layout (every sequence frames + 1 rows) or, when the
@@ -213,12 +216,6 @@ int gemm(kimodo_ctx* c, const void* A, int lda, const void* W, int ldw, int M, i
       return launch(c, cls_override >= 0 ? cls_override : CLS_GEMM_TC, flops, bytes, st, "gemm_tc2",
                     [&] { return gemm_tc2(g, bn, kind, out_f32, ep, c->derr, st); });
     }
-    // a few hundred tokens: the layer projections split K over a cluster (the MMA chain
-    // of a full-K tile, not the bytes, would set the time)
-    if (M < 1024 && gemm_splitk_supports(kind, out_f32) && gemm_splitk_factor(N, K) >= 2) {
-      return launch(c, cls_override >= 0 ? cls_override : CLS_GEMM_TC, flops, bytes, st, "gemm_splitk",
-                    [&] { return gemm_splitk(g, kind, out_f32, ep, c->derr, st); });
-    }
     const int bn = pick_bn(c, M, N, kind, out_f32);
     return launch(c, cls_override >= 0 ? cls_override : CLS_GEMM_TC, flops, bytes, st, "gemm_tc",
                   [&] { return gemm_tc(g, bn, kind, out_f32, ep, c->derr, st, c->num_sms); });
@@ -339,7 +336,8 @@ int alloc_workspace(kimodo_ctx* c, Workspace& w, int nseq, int frames, int steps
       {(void**)&w.lengths, (size_t)NS * 4},                {(void**)&w.st_text, (size_t)NS * DTXT * 4},
       {(void**)&w.st_null, (size_t)NS * DTXT * 4},        {(void**)&w.tok0, (size_t)(NS + 1) * 4},
       {(void**)&w.row_seq, (size_t)R2 * 4},               {(void**)&w.stats[0], (size_t)R2 * 8},
-      {(void**)&w.stats[1], (size_t)R2 * 8}};
+      {(void**)&w.stats[1], (size_t)R2 * 8},
+      {(void**)&w.flow, (size_t)FLOW_EVENTS * ((R2 + FLOW_BLOCK - 1) / FLOW_BLOCK) * 4}};
   for (auto& p : plan) off += align256(p.second);
   void* arena = nullptr;
   cudaError_t err = cudaMalloc(&arena, off);
@@ -356,6 +354,15 @@ int alloc_workspace(kimodo_ctx* c, Workspace& w, int nseq, int frames, int steps
     off += align256(p.second);
   }
   w.cap_rows = R2; w.cap_seq = NS; w.cap_frames = TF; w.cap_steps = ST;
+  w.flow_stride = (R2 + FLOW_BLOCK - 1) / FLOW_BLOCK;
+  return KIMODO_OK;
+}
+
+// Zero the dataflow counters of the current workspace at the start of a call.
+int flow_reset(kimodo_ctx* c, cudaStream_t st) {
+  Workspace& w = c->ws;
+  w.flow_epoch = 0;
+  if (w.flow) KD_CUDA(cudaMemsetAsync(w.flow, 0, (size_t)FLOW_EVENTS * w.flow_stride * 4, st));
   return KIMODO_OK;
 }
 
@@ -425,6 +432,19 @@ int run_net(kimodo_ctx* c, int net, int nseq, int T, int len_mod, const void* A_
   const bool bf = c->bf16();
   const void* resid = bf ? static_cast<const void*>(w.y) : w.h;
   const double eb = (double)c->elem();
+  // Row-block dataflow inside the layers when every projection runs on the CTA-pair GEMM:
+  // each kernel waits for the 256-row blocks it reads instead of its whole predecessor.
+  // Per-block counts per epoch: a pair GEMM adds 16 (its epilogue warps) per tile column,
+  // attention the block's rows per head, LayerNorm the block's rows.
+  const bool flow_on = bf && M >= 1024 && w.flow != nullptr && w.flow_stride * FLOW_BLOCK >= M;
+  auto flow_of = [&](int wait_ev, int epochs, int unit, int rows, int sig_ev) {
+    Flow f;
+    if (!flow_on) return f;
+    f.ctr = w.flow; f.stride = w.flow_stride; f.M = M; f.err = c->derr;
+    f.wait_ev = wait_ev; f.wait_epochs = epochs; f.wait_unit = unit; f.wait_rows = rows; f.sig_ev = sig_ev;
+    return f;
+  };
+  auto pair_cols = [&](int N, int kind) { return 16 * ((N + gemm_tc2_pick_bn(M, N, kind) - 1) / gemm_tc2_pick_bn(M, N, kind)); };
   auto resid_epi = [&](EpiParams& e, int which, const float* g, const float* b) {
     if (!bf || g == nullptr) return EPI_BIAS_RESID;
     e.ln_stats = w.stats[which];
@@ -433,15 +453,20 @@ int run_net(kimodo_ctx* c, int net, int nseq, int T, int len_mod, const void* A_
     return EPI_BIAS_RESID_LN;
   };
   for (int l = 0; l < L; ++l) {
+    const int ep_ = w.flow_epoch;
+    const int u_qkv = pair_cols(3 * D, EPI_BIAS), u_f1 = pair_cols(F, EPI_BIAS_GELU);
+    const int u_o = pair_cols(D, l > 0 ? EPI_BIAS_RESID_LN : EPI_BIAS_RESID), u_f2 = pair_cols(D, EPI_BIAS_RESID_LN);
     EpiParams e;
     e.bias = n.qkv_b[l]; e.out = w.qkv; e.ldo = 3 * D; e.N = 3 * D; e.M = M;
+    // layer 0 reads the input projection (whole-grid wait); later layers the previous LayerNorm 2
+    e.flow = flow_of(l > 0 ? FLOW_LN2 : -1, ep_, 1, 1, FLOW_QKV);
     KD_TRY(gemm(c, w.h, D, n.qkv_W[l], D, M, 3 * D, D, EPI_BIAS, act_f32, e, st));
     const double aflops = packed ? 4.0 * (double)M * S * DH * H : 4.0 * (double)nseq * S * S * DH * H;
     const double abytes = (double)M * 3 * D * eb + (double)M * D * eb;
     if (bf) {
       KD_TRY(launch(c, CLS_ATTN, aflops, abytes, st, "attention_tc", [&] {
         return attention_tc(static_cast<const bf16*>(w.qkv), static_cast<bf16*>(w.attn), M, w.lengths, len_mod,
-                            nseq, S, c->derr, st, tok0);
+                            nseq, S, c->derr, st, tok0, flow_of(FLOW_QKV, ep_ + 1, u_qkv, 0, FLOW_ATTN));
       }));
     } else {
       KD_TRY(launch(c, CLS_ATTN, aflops, abytes, st, "attention_f32", [&] {
@@ -454,22 +479,28 @@ int run_net(kimodo_ctx* c, int net, int nseq, int T, int len_mod, const void* A_
     eo.N = D; eo.M = M;
     // layer 0 adds the un-normalised input projection; later layers the previous LayerNorm 2
     const int ko = resid_epi(eo, 1, l > 0 ? n.ln2_g[l - 1] : nullptr, l > 0 ? n.ln2_b[l - 1] : nullptr);
+    eo.flow = flow_of(FLOW_ATTN, ep_ + 1, H, 1, FLOW_O);
     KD_TRY(gemm(c, w.attn, D, n.o_W[l], D, M, D, D, ko, true, eo, st));
     const double lnb = bf ? (double)M * D * (4.0 + eb) + (double)M * 8 : (double)M * D * 8.0;
     KD_TRY(launch(c, CLS_LN, 0, lnb, st, "layernorm", [&] {
-      return layernorm(w.y, w.h, bf, n.ln1_g[l], n.ln1_b[l], M, st, bf ? w.stats[0] : nullptr);
+      return layernorm(w.y, w.h, bf, n.ln1_g[l], n.ln1_b[l], M, st, bf ? w.stats[0] : nullptr,
+                       flow_of(FLOW_O, ep_ + 1, u_o, 0, FLOW_LN1));
     }));
     EpiParams e1;
     e1.bias = n.ff1_b[l]; e1.out = w.u; e1.ldo = F; e1.N = F; e1.M = M;
+    e1.flow = flow_of(FLOW_LN1, ep_ + 1, 1, 1, FLOW_FFN1);
     KD_TRY(gemm(c, w.h, D, n.ff1_W[l], D, M, F, D, EPI_BIAS_GELU, act_f32, e1, st));
     EpiParams e2;
     e2.bias = n.ff2_b[l]; e2.out = w.y; e2.ldo = D; e2.resid = resid; e2.ldr = D;
     e2.N = D; e2.M = M;
     const int kf = resid_epi(e2, 0, n.ln1_g[l], n.ln1_b[l]);
+    e2.flow = flow_of(FLOW_FFN1, ep_ + 1, u_f1, 0, FLOW_FFN2);
     KD_TRY(gemm(c, w.u, F, n.ff2_W[l], F, M, D, F, kf, true, e2, st));
     KD_TRY(launch(c, CLS_LN, 0, lnb, st, "layernorm", [&] {
-      return layernorm(w.y, w.h, bf, n.ln2_g[l], n.ln2_b[l], M, st, bf ? w.stats[1] : nullptr);
+      return layernorm(w.y, w.h, bf, n.ln2_g[l], n.ln2_b[l], M, st, bf ? w.stats[1] : nullptr,
+                       flow_of(FLOW_FFN2, ep_ + 1, u_f2, 0, FLOW_LN2));
     }));
+    w.flow_epoch = ep_ + 1;
   }
   EpiParams eo;
   eo.bias = n.out_b; eo.out = hat; eo.ldo = n.dout; eo.lengths = w.lengths; eo.len_mod = len_mod; eo.S = S;
@@ -500,69 +531,6 @@ struct Sampler {
   int takes = 1;              // sequences per text-embedding row (variations of one prompt)
 };
 
-// Guidance branches of a small step: when the cond and uncond sequences of a step hold
-// fewer than BRANCH_MAX_ROWS token rows in all (one or a few prompts), the two branches'
-// root network, global-to-local transform and body network run as two parallel chains
-// (own activation workspace, own stream, forked from and joined back to the step's
-// stream), since every kernel at that size leaves most SMs idle; CFG and DDIM follow the
-// join.  Padded token layout only.
-constexpr int BRANCH_MAX_ROWS = 1024;
-
-bool use_branches(const kimodo_ctx* c, int B, int T) {
-  return SAMPLE_GROUPS >= 2 && !c->profiling && !c->tk.packed && 2 * B * (T + 1) < BRANCH_MAX_ROWS;
-}
-
-int ensure_branch_resources(kimodo_ctx* c, int B, int frames) {
-  for (int g = 0; g < 2; ++g) {
-    bool grown = false;
-    KD_TRY(alloc_workspace(c, c->gws[g], B, frames, 1, &grown));
-    if (grown) free_graphs(c);
-    if (!c->gst[g] && cudaStreamCreateWithFlags(&c->gst[g], cudaStreamNonBlocking) != cudaSuccess)
-      return set_error(KIMODO_ECUDA, "stream creation failed");
-  }
-  for (int i = 0; i < 3; ++i)
-    if (!c->gev[i] && cudaEventCreateWithFlags(&c->gev[i], cudaEventDisableTiming) != cudaSuccess)
-      return set_error(KIMODO_ECUDA, "event creation failed");
-  return KIMODO_OK;
-}
-
-// The networks of both guidance branches of one step, branch g (0 cond, 1 uncond) on
-// stream gst[g] with workspace gws[g]; the inputs, predictions and the state stay in the
-// step's workspace (branch g's sequences are its rows g B .. g B + B - 1).
-int branch_nets(kimodo_ctx* c, int B, int T, int k_row, cudaStream_t st) {
-  const Workspace main_ws = c->ws;
-  const int S = T + 1;
-  const size_t e = c->elem();
-  const double eb = (double)e;
-  KD_CUDA(cudaEventRecord(c->gev[0], st));
-  int r = KIMODO_OK;
-  for (int g = 0; g < 2 && r == KIMODO_OK; ++g) {
-    cudaStream_t bs = c->gst[g];
-    Workspace wb = c->gws[g];
-    wb.lengths = main_ws.lengths;
-    c->ws = wb;
-    const size_t s0 = (size_t)g * B;
-    const void* A_root = static_cast<const char*>(main_ws.A_root) + s0 * S * ROOT_IN_LD * e;
-    void* A_body = static_cast<char*>(main_ws.A_body) + s0 * S * BODY_IN_LD * e;
-    float* rh = main_ws.root_hat + s0 * T * ROOT_F;
-    float* bh = main_ws.body_hat + s0 * T * BODY_F;
-    if (cudaStreamWaitEvent(bs, c->gev[0], 0) != cudaSuccess) r = set_error(KIMODO_ECUDA, "stream fork failed");
-    if (r == KIMODO_OK)
-      r = run_net(c, 0, B, T, B, A_root, main_ws.tmlp[0] + (long)k_row * D, main_ws.txt[0] + s0 * D, rh, bs);
-    if (r == KIMODO_OK)
-      r = launch(c, CLS_MOTION, 0, (double)B * T * (ROOT_F * 4 + MOTION_F * (4 + eb)), bs, "g2l_body_input", [&] {
-        return g2l_body_input(rh, main_ws.x, main_ws.lengths, B, B, T, S, A_body, c->bf16(), BODY_IN_LD, bs);
-      });
-    if (r == KIMODO_OK)
-      r = run_net(c, 1, B, T, B, A_body, main_ws.tmlp[1] + (long)k_row * D, main_ws.txt[1] + s0 * D, bh, bs);
-    if (r == KIMODO_OK && (cudaEventRecord(c->gev[1 + g], bs) != cudaSuccess ||
-                           cudaStreamWaitEvent(st, c->gev[1 + g], 0) != cudaSuccess))
-      r = set_error(KIMODO_ECUDA, "stream join failed");
-  }
-  c->ws = main_ws;
-  return r;
-}
-
 // One two-stage step for B prompts (cond rows 0..B-1, uncond rows B..2B-1).
 // Reads ws.x, writes ws.x.  tvec_root / tvec_body are the timestep-MLP rows.
 int two_stage_step(kimodo_ctx* c, int B, int T, int t, int t_prev, float w_cfg, int k_row, bool pack_next,
@@ -570,17 +538,12 @@ int two_stage_step(kimodo_ctx* c, int B, int T, int t, int t_prev, float w_cfg, 
   Workspace& w = c->ws;
   const int nseq = 2 * B, S = T + 1;
   const double eb = (double)c->elem();
-  if (use_branches(c, B, T)) {
-    KD_TRY(branch_nets(c, B, T, k_row, st));
-  } else {
-    KD_TRY(run_net(c, 0, nseq, T, B, w.A_root, w.tmlp[0] + (long)k_row * D, w.txt[0], w.root_hat, st));
-    KD_TRY(launch(c, CLS_MOTION, 0, (double)nseq * T * (ROOT_F * 4 + MOTION_F * (4 + eb)), st, "g2l_body_input",
-                  [&] {
-                    return g2l_body_input(w.root_hat, w.x, w.lengths, B, nseq, T, S, w.A_body, c->bf16(),
-                                          BODY_IN_LD, st, c->tk.packed ? w.tok0 : nullptr);
-                  }));
-    KD_TRY(run_net(c, 1, nseq, T, B, w.A_body, w.tmlp[1] + (long)k_row * D, w.txt[1], w.body_hat, st));
-  }
+  KD_TRY(run_net(c, 0, nseq, T, B, w.A_root, w.tmlp[0] + (long)k_row * D, w.txt[0], w.root_hat, st));
+  KD_TRY(launch(c, CLS_MOTION, 0, (double)nseq * T * (ROOT_F * 4 + MOTION_F * (4 + eb)), st, "g2l_body_input", [&] {
+    return g2l_body_input(w.root_hat, w.x, w.lengths, B, nseq, T, S, w.A_body, c->bf16(), BODY_IN_LD, st,
+                          c->tk.packed ? w.tok0 : nullptr);
+  }));
+  KD_TRY(run_net(c, 1, nseq, T, B, w.A_body, w.tmlp[1] + (long)k_row * D, w.txt[1], w.body_hat, st));
   float c0, c1, c2;
   ddim_coeffs(c, smp.schedule, t, t_prev, smp.eta, &c0, &c1, &c2);
   const float* z = c2 != 0.f ? z_step : nullptr;
@@ -731,8 +694,7 @@ int kimodo_load_weights(kimodo_ctx** out_ctx, const float* host_blob, size_t n_f
   if (precision == KIMODO_BF16 && !gemm_tc_available())
     return set_error(KIMODO_EUNSUPPORTED, "cuTensorMapEncodeTiled is unavailable in this driver");
 
-  if (gemm_tc_prepare() != cudaSuccess || gemm_tc2_prepare() != cudaSuccess || gemm_splitk_prepare() != cudaSuccess ||
-      attention_tc_prepare() != cudaSuccess) {
+  if (gemm_tc_prepare() != cudaSuccess || gemm_tc2_prepare() != cudaSuccess || attention_tc_prepare() != cudaSuccess) {
     cudaGetLastError();
     return set_error(KIMODO_EUNSUPPORTED, "kernel attributes could not be set on device %d", device);
   }
@@ -842,6 +804,7 @@ int kimodo_denoiser_forward(kimodo_ctx* c, int net, const float* x, const float*
   NetW& n = c->net[net];
   KD_TRY(stage_lengths(c, lengths, batch, frames, st));
   c->tk = plan_tokens(lengths, batch, batch, frames);
+  KD_TRY(flow_reset(c, st));
   KD_TRY(enqueue_token_map(c, batch, batch, st));
   KD_CUDA(cudaMemcpyAsync(w.x, x, (size_t)batch * frames * n.din * 4, cudaMemcpyDefault, st));
   KD_CUDA(cudaMemcpyAsync(w.st_text, emb, (size_t)batch * DTXT * 4, cudaMemcpyDefault, st));
@@ -929,7 +892,7 @@ int kimodo_ddim_step_ex(kimodo_ctx* c, const float* x_t, const float* text_emb, 
   Workspace& w = c->ws;
   KD_TRY(stage_lengths(c, lengths, batch, frames, st));
   c->tk = plan_tokens(lengths, batch, 2 * batch, frames);
-  if (use_branches(c, batch, frames)) KD_TRY(ensure_branch_resources(c, batch, frames));
+  KD_TRY(flow_reset(c, st));
   KD_TRY(enqueue_token_map(c, batch, 2 * batch, st));
   KD_CUDA(cudaMemcpyAsync(w.x, x_t, (size_t)batch * frames * MOTION_F * 4, cudaMemcpyDefault, st));
   KD_CUDA(cudaMemcpyAsync(w.st_text, text_emb, (size_t)(batch / smp.takes) * DTXT * 4, cudaMemcpyDefault, st));
@@ -953,6 +916,7 @@ int kimodo_ddim_step_ex(kimodo_ctx* c, const float* x_t, const float* text_emb, 
 static int enqueue_loop(kimodo_ctx* c, int batch, int frames, int steps, float cfg, int null_batch,
                         const Sampler& smp, int b0, int batch_all, cudaStream_t st) {
   Workspace& w = c->ws;
+  KD_TRY(flow_reset(c, st));
   KD_TRY(enqueue_token_map(c, batch, 2 * batch, st));
   KD_TRY(launch(c, CLS_SETUP, 0, (double)2 * batch * DTXT * 6, st, "pack_embeddings", [&] {
     return pack_embeddings(w.st_text, batch, w.st_null, null_batch, batch, w.emb, c->bf16(), st, smp.takes);
@@ -1057,7 +1021,6 @@ int kimodo_ddim_sample_ex(kimodo_ctx* c, const float* text_emb, const float* nul
   // the prompt groups' workspaces and streams exist before any capture begins
   const int groups = sample_groups(c, batch, smp);
   if (groups > 1) KD_TRY(ensure_group_resources(c, groups, batch, frames, steps));
-  if (use_branches(c, batch, frames)) KD_TRY(ensure_branch_resources(c, batch, frames));
   KD_CUDA(cudaMemcpyAsync(w.x, noise, (size_t)batch * frames * MOTION_F * 4, cudaMemcpyDefault, st));
   KD_CUDA(cudaMemcpyAsync(w.st_text, text_emb, (size_t)(batch / smp.takes) * DTXT * 4, cudaMemcpyDefault, st));
   KD_CUDA(cudaMemcpyAsync(w.st_null, null_emb, (size_t)null_batch * DTXT * 4, cudaMemcpyDefault, st));
@@ -1198,7 +1161,6 @@ int prepared_device() {
   if (!done[dev]) {
     KD_CUDA(gemm_tc_prepare());
     KD_CUDA(gemm_tc2_prepare());
-    KD_CUDA(gemm_splitk_prepare());
     KD_CUDA(attention_tc_prepare());
     done[dev] = true;
   }
@@ -1274,29 +1236,6 @@ int kimodo_gemm_bf16_pair(const void* A, int lda, const void* W, int ldw, const 
   ep.bias = bias; ep.out = out; ep.ldo = ldo; ep.resid = resid; ep.ldr = ldr; ep.N = N; ep.M = M;
   const int bn = tile_n ? tile_n : gemm_tc2_pick_bn(M, N, epilogue);
   KD_CUDA(gemm_tc2(g, bn, epilogue, out_f32 != 0, ep, kernel_error_word(), static_cast<cudaStream_t>(stream)));
-  return KIMODO_OK;
-}
-
-int kimodo_gemm_bf16_splitk(const void* A, int lda, const void* W, int ldw, const float* bias, const void* resid,
-                            int ldr, void* out, int ldo, int M, int N, int K, int epilogue, int out_f32,
-                            void* stream) {
-  g_last_error.clear();
-  KD_TRY(check_gemm_args(A, lda, W, ldw, bias, resid, out, ldo, M, N, K, epilogue));
-  if (lda % 8 || ldw % 8 || (reinterpret_cast<uintptr_t>(A) & 15) || (reinterpret_cast<uintptr_t>(W) & 15))
-    return set_error(KIMODO_EINVAL, "bf16 operands need 16-byte aligned rows (lda, ldw multiples of 8)");
-  if (ldo % 4 || (reinterpret_cast<uintptr_t>(out) & 15) || (epilogue == 3 && (ldr % 4 ||
-      (reinterpret_cast<uintptr_t>(resid) & 15))) || (reinterpret_cast<uintptr_t>(bias) & 15))
-    return set_error(KIMODO_EINVAL, "out, resid and bias need 16-byte alignment and ldo, ldr multiples of 4");
-  if (!gemm_splitk_supports(epilogue, out_f32 != 0))
-    return set_error(KIMODO_EINVAL, "split-K epilogues: bias or GELU with bf16 output, residual with fp32 output");
-  if (gemm_splitk_factor(N, K) < 2)
-    return set_error(KIMODO_EINVAL, "split-K GEMM needs N % 256 == 0 and K / 256 in 2..8");
-  KD_TRY(prepared_device());
-  GemmArgs g;
-  g.A = A; g.B = W; g.M = M; g.N = N; g.K = K; g.lda = lda; g.ldb = ldw;
-  EpiParams ep;
-  ep.bias = bias; ep.out = out; ep.ldo = ldo; ep.resid = resid; ep.ldr = ldr; ep.N = N; ep.M = M;
-  KD_CUDA(gemm_splitk(g, epilogue, out_f32 != 0, ep, kernel_error_word(), static_cast<cudaStream_t>(stream)));
   return KIMODO_OK;
 }
 

@@ -38,16 +38,6 @@ cudaError_t gemm_tc2(const GemmArgs& g, int bn, int kind, bool out_f32, const Ep
 cudaError_t gemm_tc2_prepare();
 bool gemm_tc2_supports(int kind, bool out_f32);
 int gemm_tc2_pick_bn(int M, int N, int kind);
-// tcgen05 GEMM for a few hundred tokens: 128 x 256 output tiles, K split over a cluster of
-// S = gemm_splitk_factor(N, K) CTAs (four 64-deep k-blocks each), the fp32 partials summed
-// in cluster-rank order through distributed shared memory, then the usual epilogue.
-// EPI_BIAS / EPI_BIAS_GELU with bf16 output, EPI_BIAS_RESID / EPI_BIAS_RESID_LN with fp32
-// output; N % 256 == 0.
-int gemm_splitk_factor(int N, int K);   // 0 when the shape does not split (S outside 2..8)
-bool gemm_splitk_supports(int kind, bool out_f32);
-cudaError_t gemm_splitk(const GemmArgs& g, int kind, bool out_f32, const EpiParams& ep, DevError* err,
-                        cudaStream_t st);
-cudaError_t gemm_splitk_prepare();
 // Set the dynamic shared-memory limits of every kernel instantiation (call once
 // per device before any launch or graph capture).
 cudaError_t gemm_tc_prepare();
@@ -67,7 +57,7 @@ cudaError_t attention_f32(const float* qkv, float* out, const int* lengths, int 
 // 128-query tile), exact softmax over all keys of the sequence at once.  qkv has M
 // rows (16-byte aligned, row stride 3*D); S <= MAX_FRAMES + 1.
 cudaError_t attention_tc(const bf16* qkv, bf16* out, int M, const int* lengths, int len_mod, int nseq, int S,
-                         DevError* err, cudaStream_t st, const int* tok0 = nullptr);
+                         DevError* err, cudaStream_t st, const int* tok0 = nullptr, const Flow& flow = Flow());
 cudaError_t attention_tc_prepare();
 size_t attention_tc_smem(int S);
 
@@ -78,7 +68,7 @@ cudaError_t build_token_map(const int* lengths, int len_mod, int nseq, int* tok0
 // Row LayerNorm over D features: y fp32 [M, D] -> out (bf16 or fp32) [M, D], and
 // optionally the row statistics (mean, 1/std) into stats [M][2].
 cudaError_t layernorm(const float* y, void* out, bool out_bf16, const float* gamma, const float* beta, int M,
-                      cudaStream_t st, float* stats = nullptr);
+                      cudaStream_t st, float* stats = nullptr, const Flow& flow = Flow());
 
 // ---- motion / sampler kernels (element type of the activation matrices: bf16 or fp32)
 
