@@ -224,25 +224,3 @@ def test_variations_against_oracle(gpu_bf16, oracle_refs):
         report(f"bf16 variations seq {b} (prompt {b // 3}) trajectory rel-L2",
                rel_l2(got[b], oracle_refs.result(VAR, b)), TOL_BF16_TRAJ)
 
-
-def test_row_block_dataflow_matches_serialised_kernels(gpu_bf16):
-    """At 16 prompts the layer kernels wait for the row blocks they read, not for the whole
-    previous kernel, so consecutive kernels overlap.  The same generation with every kernel
-    serialised (profiling mode puts timing events between the kernels) must give the same
-    bits, and two overlapped runs must agree: a missing or misplaced wait would show as a
-    difference."""
-    B, T = 16, 150
-    L = np.full(B, T, np.int32)
-    noise = synth.noise(B, T, seed=81)
-    emb = synth.text_embeddings(B, seed=82)
-    null = np.zeros(4096, np.float32)
-    a = gpu_bf16.ddim_sample(emb, null, noise, L, 6, 2.0)
-    b = gpu_bf16.ddim_sample(emb, null, noise, L, 6, 2.0)
-    gpu_bf16.profile_enable(True)
-    try:
-        s = gpu_bf16.ddim_sample(emb, null, noise, L, 6, 2.0)
-    finally:
-        gpu_bf16.profile_enable(False)
-    gpu_bf16.sync_status()
-    np.testing.assert_array_equal(a, b)
-    np.testing.assert_array_equal(a, s)

@@ -29,7 +29,6 @@
 #include "common.cuh"
 #include "epilogue.cuh"
 #include "kernels.h"
-#include "flow.cuh"
 #include "launch.cuh"
 #include "ptx.cuh"
 
@@ -86,7 +85,7 @@ __device__ __forceinline__ uint64_t smem_desc_sw128_mn(uint32_t saddr, uint32_t 
 __global__ void __launch_bounds__(NUM_THREADS, 2)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmKV,
                const __grid_constant__ CUtensorMap tmO, bf16* __restrict__ out, const int* __restrict__ lengths, int len_mod, int S_pad, int ka,
-               uint32_t tmem_cols, uint32_t o_col, const int* __restrict__ tok0, Flow flow, DevError* err) {
+               uint32_t tmem_cols, uint32_t o_col, const int* __restrict__ tok0, DevError* err) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t kp = kp_of(ka);
@@ -111,8 +110,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int h = blockIdx.x, seq = blockIdx.y, qt = blockIdx.z;
-  // with a row-block dataflow the CTA waits below for the QKV rows of its sequence only
-  if (flow.ctr == nullptr || flow.wait_ev < 0) ptx::pdl_wait();
+  ptx::pdl_wait();
   ptx::pdl_trigger();
   const long row0 = tok0 ? tok0[seq] : (long)seq * S_pad;
   const int S = tok0 ? tok0[seq + 1] - tok0[seq] : S_pad;
@@ -131,9 +129,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     ptx::mbar_init(bar_o, 1);
     ptx::fence_mbar_init();
     *abort = (err != nullptr && *reinterpret_cast<volatile int*>(&err->code) != 0) ? 1 : 0;
-    // the QKV rows of this sequence are complete
-    for (int b = (int)(row0 / FLOW_BLOCK); !*abort && b <= (int)((row0 + S - 1) / FLOW_BLOCK); ++b)
-      if (!flow_wait(flow, b, abort, WAIT_LIMIT_NS)) record_timeout(err, abort);
     if (!*abort) {
       // the query tile, the keys and the upper value half, issued before the TMEM allocation
       // and the CTA barrier so that their latency overlaps the set-up
@@ -327,22 +322,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     }
     if (!ok && !*abort) record_timeout(err, abort);
   }
-  if (flow.ctr != nullptr) __threadfence();   // this thread's output rows, before the count below
   ptx::tc_fence_before();
   __syncthreads();
   if (warp == 1) {
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem_base, tmem_cols);
-  }
-  if (threadIdx.x == 0 && !skip && !*abort) {
-    // count this head's output rows per row block for the attention-output projection
-    const long r0 = row0 + qt * QT;
-    const long r1 = row0 + (S - qt * QT < QT ? S : qt * QT + QT);
-    for (long b = r0 / FLOW_BLOCK; b * FLOW_BLOCK < r1; ++b) {
-      const long lo = b * FLOW_BLOCK > r0 ? b * FLOW_BLOCK : r0;
-      const long hi = (b + 1) * FLOW_BLOCK < r1 ? (b + 1) * FLOW_BLOCK : r1;
-      flow_signal(flow, (int)b, (int)(hi - lo));
-    }
   }
 }
 
@@ -359,7 +343,7 @@ cudaError_t attention_tc_prepare() {
 }
 
 cudaError_t attention_tc(const bf16* qkv, bf16* out, int M, const int* lengths, int len_mod, int nseq, int S,
-                         DevError* err, cudaStream_t st, const int* tok0, const Flow& flow) {
+                         DevError* err, cudaStream_t st, const int* tok0) {
   if (nseq <= 0 || S <= 0 || M <= 0) return cudaSuccess;
   if (S > MAX_FRAMES + 1) return cudaErrorInvalidValue;
   CUtensorMap tq, tkv, to;
@@ -374,7 +358,7 @@ cudaError_t attention_tc(const bf16* qkv, bf16* out, int M, const int* lengths, 
   const uint32_t o_col = n_cols_max <= 256 ? 0u : 320u;
   dim3 grid(H, nseq, (S + QT - 1) / QT);
   return launch_kernel(attn_tc_kernel, grid, dim3(NUM_THREADS), smem_bytes(ka), st, tq, tkv, to, out, lengths, len_mod,
-                       S, ka, tmem_cols, o_col, tok0, flow, err);
+                       S, ka, tmem_cols, o_col, tok0, err);
 }
 
 }  // namespace kd

@@ -90,9 +90,6 @@ struct Workspace {
   int* lengths = nullptr; float* st_text = nullptr; float* st_null = nullptr;
   int* tok0 = nullptr; int* row_seq = nullptr;   // packed token layout (valid tokens only)
   float* stats[2] = {};                           // LayerNorm row statistics (mean, 1/std) [M][2]
-  int* flow = nullptr;                            // row-block dataflow counters [FLOW_EVENTS][flow_stride]
-  int flow_stride = 0;
-  int flow_epoch = 0;                             // host: layer epochs enqueued since the counters were zeroed
 };
 
 // Token rows of a call: the padded layout (every sequence frames + 1 rows) or, when the
@@ -336,8 +333,7 @@ int alloc_workspace(kimodo_ctx* c, Workspace& w, int nseq, int frames, int steps
       {(void**)&w.lengths, (size_t)NS * 4},                {(void**)&w.st_text, (size_t)NS * DTXT * 4},
       {(void**)&w.st_null, (size_t)NS * DTXT * 4},        {(void**)&w.tok0, (size_t)(NS + 1) * 4},
       {(void**)&w.row_seq, (size_t)R2 * 4},               {(void**)&w.stats[0], (size_t)R2 * 8},
-      {(void**)&w.stats[1], (size_t)R2 * 8},
-      {(void**)&w.flow, (size_t)FLOW_EVENTS * ((R2 + FLOW_BLOCK - 1) / FLOW_BLOCK) * 4}};
+      {(void**)&w.stats[1], (size_t)R2 * 8}};
   for (auto& p : plan) off += align256(p.second);
   void* arena = nullptr;
   cudaError_t err = cudaMalloc(&arena, off);
@@ -354,15 +350,6 @@ int alloc_workspace(kimodo_ctx* c, Workspace& w, int nseq, int frames, int steps
     off += align256(p.second);
   }
   w.cap_rows = R2; w.cap_seq = NS; w.cap_frames = TF; w.cap_steps = ST;
-  w.flow_stride = (R2 + FLOW_BLOCK - 1) / FLOW_BLOCK;
-  return KIMODO_OK;
-}
-
-// Zero the dataflow counters of the current workspace at the start of a call.
-int flow_reset(kimodo_ctx* c, cudaStream_t st) {
-  Workspace& w = c->ws;
-  w.flow_epoch = 0;
-  if (w.flow) KD_CUDA(cudaMemsetAsync(w.flow, 0, (size_t)FLOW_EVENTS * w.flow_stride * 4, st));
   return KIMODO_OK;
 }
 
@@ -432,19 +419,6 @@ int run_net(kimodo_ctx* c, int net, int nseq, int T, int len_mod, const void* A_
   const bool bf = c->bf16();
   const void* resid = bf ? static_cast<const void*>(w.y) : w.h;
   const double eb = (double)c->elem();
-  // Row-block dataflow inside the layers when every projection runs on the CTA-pair GEMM:
-  // each kernel waits for the 256-row blocks it reads instead of its whole predecessor.
-  // Per-block counts per epoch: a pair GEMM adds 16 (its epilogue warps) per tile column,
-  // attention the block's rows per head, LayerNorm the block's rows.
-  const bool flow_on = bf && M >= 1024 && w.flow != nullptr && w.flow_stride * FLOW_BLOCK >= M;
-  auto flow_of = [&](int wait_ev, int epochs, int unit, int rows, int sig_ev) {
-    Flow f;
-    if (!flow_on) return f;
-    f.ctr = w.flow; f.stride = w.flow_stride; f.M = M; f.err = c->derr;
-    f.wait_ev = wait_ev; f.wait_epochs = epochs; f.wait_unit = unit; f.wait_rows = rows; f.sig_ev = sig_ev;
-    return f;
-  };
-  auto pair_cols = [&](int N, int kind) { return 16 * ((N + gemm_tc2_pick_bn(M, N, kind) - 1) / gemm_tc2_pick_bn(M, N, kind)); };
   auto resid_epi = [&](EpiParams& e, int which, const float* g, const float* b) {
     if (!bf || g == nullptr) return EPI_BIAS_RESID;
     e.ln_stats = w.stats[which];
@@ -453,20 +427,15 @@ int run_net(kimodo_ctx* c, int net, int nseq, int T, int len_mod, const void* A_
     return EPI_BIAS_RESID_LN;
   };
   for (int l = 0; l < L; ++l) {
-    const int ep_ = w.flow_epoch;
-    const int u_qkv = pair_cols(3 * D, EPI_BIAS), u_f1 = pair_cols(F, EPI_BIAS_GELU);
-    const int u_o = pair_cols(D, l > 0 ? EPI_BIAS_RESID_LN : EPI_BIAS_RESID), u_f2 = pair_cols(D, EPI_BIAS_RESID_LN);
     EpiParams e;
     e.bias = n.qkv_b[l]; e.out = w.qkv; e.ldo = 3 * D; e.N = 3 * D; e.M = M;
-    // layer 0 reads the input projection (whole-grid wait); later layers the previous LayerNorm 2
-    e.flow = flow_of(l > 0 ? FLOW_LN2 : -1, ep_, 1, 1, FLOW_QKV);
     KD_TRY(gemm(c, w.h, D, n.qkv_W[l], D, M, 3 * D, D, EPI_BIAS, act_f32, e, st));
     const double aflops = packed ? 4.0 * (double)M * S * DH * H : 4.0 * (double)nseq * S * S * DH * H;
     const double abytes = (double)M * 3 * D * eb + (double)M * D * eb;
     if (bf) {
       KD_TRY(launch(c, CLS_ATTN, aflops, abytes, st, "attention_tc", [&] {
         return attention_tc(static_cast<const bf16*>(w.qkv), static_cast<bf16*>(w.attn), M, w.lengths, len_mod,
-                            nseq, S, c->derr, st, tok0, flow_of(FLOW_QKV, ep_ + 1, u_qkv, 0, FLOW_ATTN));
+                            nseq, S, c->derr, st, tok0);
       }));
     } else {
       KD_TRY(launch(c, CLS_ATTN, aflops, abytes, st, "attention_f32", [&] {
@@ -479,28 +448,22 @@ int run_net(kimodo_ctx* c, int net, int nseq, int T, int len_mod, const void* A_
     eo.N = D; eo.M = M;
     // layer 0 adds the un-normalised input projection; later layers the previous LayerNorm 2
     const int ko = resid_epi(eo, 1, l > 0 ? n.ln2_g[l - 1] : nullptr, l > 0 ? n.ln2_b[l - 1] : nullptr);
-    eo.flow = flow_of(FLOW_ATTN, ep_ + 1, H, 1, FLOW_O);
     KD_TRY(gemm(c, w.attn, D, n.o_W[l], D, M, D, D, ko, true, eo, st));
     const double lnb = bf ? (double)M * D * (4.0 + eb) + (double)M * 8 : (double)M * D * 8.0;
     KD_TRY(launch(c, CLS_LN, 0, lnb, st, "layernorm", [&] {
-      return layernorm(w.y, w.h, bf, n.ln1_g[l], n.ln1_b[l], M, st, bf ? w.stats[0] : nullptr,
-                       flow_of(FLOW_O, ep_ + 1, u_o, 0, FLOW_LN1));
+      return layernorm(w.y, w.h, bf, n.ln1_g[l], n.ln1_b[l], M, st, bf ? w.stats[0] : nullptr);
     }));
     EpiParams e1;
     e1.bias = n.ff1_b[l]; e1.out = w.u; e1.ldo = F; e1.N = F; e1.M = M;
-    e1.flow = flow_of(FLOW_LN1, ep_ + 1, 1, 1, FLOW_FFN1);
     KD_TRY(gemm(c, w.h, D, n.ff1_W[l], D, M, F, D, EPI_BIAS_GELU, act_f32, e1, st));
     EpiParams e2;
     e2.bias = n.ff2_b[l]; e2.out = w.y; e2.ldo = D; e2.resid = resid; e2.ldr = D;
     e2.N = D; e2.M = M;
     const int kf = resid_epi(e2, 0, n.ln1_g[l], n.ln1_b[l]);
-    e2.flow = flow_of(FLOW_FFN1, ep_ + 1, u_f1, 0, FLOW_FFN2);
     KD_TRY(gemm(c, w.u, F, n.ff2_W[l], F, M, D, F, kf, true, e2, st));
     KD_TRY(launch(c, CLS_LN, 0, lnb, st, "layernorm", [&] {
-      return layernorm(w.y, w.h, bf, n.ln2_g[l], n.ln2_b[l], M, st, bf ? w.stats[1] : nullptr,
-                       flow_of(FLOW_FFN2, ep_ + 1, u_f2, 0, FLOW_LN2));
+      return layernorm(w.y, w.h, bf, n.ln2_g[l], n.ln2_b[l], M, st, bf ? w.stats[1] : nullptr);
     }));
-    w.flow_epoch = ep_ + 1;
   }
   EpiParams eo;
   eo.bias = n.out_b; eo.out = hat; eo.ldo = n.dout; eo.lengths = w.lengths; eo.len_mod = len_mod; eo.S = S;
@@ -804,7 +767,6 @@ int kimodo_denoiser_forward(kimodo_ctx* c, int net, const float* x, const float*
   NetW& n = c->net[net];
   KD_TRY(stage_lengths(c, lengths, batch, frames, st));
   c->tk = plan_tokens(lengths, batch, batch, frames);
-  KD_TRY(flow_reset(c, st));
   KD_TRY(enqueue_token_map(c, batch, batch, st));
   KD_CUDA(cudaMemcpyAsync(w.x, x, (size_t)batch * frames * n.din * 4, cudaMemcpyDefault, st));
   KD_CUDA(cudaMemcpyAsync(w.st_text, emb, (size_t)batch * DTXT * 4, cudaMemcpyDefault, st));
@@ -892,7 +854,6 @@ int kimodo_ddim_step_ex(kimodo_ctx* c, const float* x_t, const float* text_emb, 
   Workspace& w = c->ws;
   KD_TRY(stage_lengths(c, lengths, batch, frames, st));
   c->tk = plan_tokens(lengths, batch, 2 * batch, frames);
-  KD_TRY(flow_reset(c, st));
   KD_TRY(enqueue_token_map(c, batch, 2 * batch, st));
   KD_CUDA(cudaMemcpyAsync(w.x, x_t, (size_t)batch * frames * MOTION_F * 4, cudaMemcpyDefault, st));
   KD_CUDA(cudaMemcpyAsync(w.st_text, text_emb, (size_t)(batch / smp.takes) * DTXT * 4, cudaMemcpyDefault, st));
@@ -916,7 +877,6 @@ int kimodo_ddim_step_ex(kimodo_ctx* c, const float* x_t, const float* text_emb, 
 static int enqueue_loop(kimodo_ctx* c, int batch, int frames, int steps, float cfg, int null_batch,
                         const Sampler& smp, int b0, int batch_all, cudaStream_t st) {
   Workspace& w = c->ws;
-  KD_TRY(flow_reset(c, st));
   KD_TRY(enqueue_token_map(c, batch, 2 * batch, st));
   KD_TRY(launch(c, CLS_SETUP, 0, (double)2 * batch * DTXT * 6, st, "pack_embeddings", [&] {
     return pack_embeddings(w.st_text, batch, w.st_null, null_batch, batch, w.emb, c->bf16(), st, smp.takes);

@@ -9,7 +9,6 @@
 #include <type_traits>
 
 #include "common.cuh"
-#include "flow.cuh"
 
 namespace kd {
 
@@ -49,7 +48,6 @@ struct EpiParams {
   int T = 1;                     // frames per sequence (EPI_OUTPROJ)
   int N = 0;                     // valid output columns
   int M = 0;                     // valid rows
-  Flow flow;                     // row-block dataflow (CTA-pair GEMM only)
 };
 
 // erf by Abramowitz & Stegun, Handbook of Mathematical Functions, formula 7.1.26:

@@ -123,11 +123,9 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
     ptx::tmem_alloc_pair(ptx::smem_u32(tmem_slot), C::TMEM_COLS);
     ptx::tmem_relinquish_pair();
   }
-  // prologue done: let the next kernel launch, then wait for the previous one (with a
-  // row-block dataflow, the producer and the epilogue wait per tile instead)
+  // prologue done: let the next kernel launch, then wait for the previous one
   ptx::pdl_trigger();
-  const bool flow_in = ep.flow.ctr != nullptr && ep.flow.wait_ev >= 0;
-  if (!flow_in) ptx::pdl_wait();
+  ptx::pdl_wait();
   // A launch after a recorded timeout does no work; both CTAs of a pair read the
   // same word (written by an earlier kernel, visible after the wait), so they agree.
   if (threadIdx.x == 0) *abort = (err != nullptr && *reinterpret_cast<volatile int*>(&err->code) != 0) ? 1 : 0;
@@ -149,11 +147,6 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
         const int m_blk = tile % num_m_tiles, n_blk = tile / num_m_tiles;
         const int arow = m_blk * 2 * BMC + (int)rank * BMC;
         const int brow = n_blk * BN + (int)rank * (BN / 2);
-        // the rows of A this tile reads are complete
-        if (!flow_wait(ep.flow, m_blk, abort, WAIT_LIMIT_NS)) {
-          ok = false;
-          break;
-        }
         for (int kb = 0; kb < num_kb; ++kb) {
           if (!ptx::mbar_wait_bounded(empty_bar(stage), phase ^ 1u, abort, WAIT_LIMIT_NS)) {
             ok = false;
@@ -263,27 +256,12 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
           }
         }
       };
-      if constexpr (C::RES) {
-        // the residual rows and their LayerNorm statistics are complete (the same wait as
-        // the producer's for this row block)
-        if (flow_in) {
-          int fw = 1;
-          if (lane == 0) fw = flow_wait(ep.flow, m_blk, abort, WAIT_LIMIT_NS) ? 1 : 0;
-          fw = __shfl_sync(0xffffffffu, fw, 0);
-          __threadfence();
-          if (!fw) {
-            if (!*abort) record_timeout(err, WHERE_GEMM_EPILOGUE, abort);
-            failed = true;
-            break;
-          }
-        }
-      }
       // this lane's row statistics for EPI_BIAS_RESID_LN: z * rs_a + rs_b = (z - mean) / std
       float rs_a = 1.f, rs_b = 0.f;
       if constexpr (KIND == EPI_BIAS_RESID_LN) {
         const int row = row0 + lane;
         if (nch > 0 && row < ep.M) {
-          const float2 st2 = __ldcg(reinterpret_cast<const float2*>(ep.ln_stats + 2 * (long)row));
+          const float2 st2 = *reinterpret_cast<const float2*>(ep.ln_stats + 2 * (long)row);
           rs_a = st2.y;
           rs_b = -st2.x * st2.y;
         }
@@ -314,16 +292,8 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive_remote(acc ? leader_tempty1 : leader_tempty0);
       };
-      // this warp's part of the tile is stored: count it for the row block's consumers
-      auto signal = [&]() {
-        if (lane == 0 && ep.flow.ctr != nullptr && ep.flow.sig_ev >= 0) {
-          ptx::bulk_wait_all();
-          flow_signal(ep.flow, m_blk, 1);
-        }
-      };
       if (nch == 0) {
         release();
-        signal();
         continue;
       }
       // finish chunk k (the warp's chunk number cc == cc0 + k) from accumulator values v, bias b4
@@ -407,7 +377,6 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
         if (!process(vb, bb, gb, c + 1)) { failed = true; break; }
       }
       if (failed && !*abort) record_timeout(err, WHERE_GEMM_EPILOGUE, abort);
-      if (!failed) signal();
     }
     if (lane == 0) ptx::bulk_wait_all();
     __syncwarp();

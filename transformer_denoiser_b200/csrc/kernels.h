@@ -57,7 +57,7 @@ cudaError_t attention_f32(const float* qkv, float* out, const int* lengths, int 
 // 128-query tile), exact softmax over all keys of the sequence at once.  qkv has M
 // rows (16-byte aligned, row stride 3*D); S <= MAX_FRAMES + 1.
 cudaError_t attention_tc(const bf16* qkv, bf16* out, int M, const int* lengths, int len_mod, int nseq, int S,
-                         DevError* err, cudaStream_t st, const int* tok0 = nullptr, const Flow& flow = Flow());
+                         DevError* err, cudaStream_t st, const int* tok0 = nullptr);
 cudaError_t attention_tc_prepare();
 size_t attention_tc_smem(int S);
 
@@ -68,7 +68,7 @@ cudaError_t build_token_map(const int* lengths, int len_mod, int nseq, int* tok0
 // Row LayerNorm over D features: y fp32 [M, D] -> out (bf16 or fp32) [M, D], and
 // optionally the row statistics (mean, 1/std) into stats [M][2].
 cudaError_t layernorm(const float* y, void* out, bool out_bf16, const float* gamma, const float* beta, int M,
-                      cudaStream_t st, float* stats = nullptr, const Flow& flow = Flow());
+                      cudaStream_t st, float* stats = nullptr);
 
 // ---- motion / sampler kernels (element type of the activation matrices: bf16 or fp32)
 

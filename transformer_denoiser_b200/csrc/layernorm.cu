@@ -9,7 +9,6 @@
 
 #include "common.cuh"
 #include "kernels.h"
-#include "flow.cuh"
 #include "launch.cuh"
 #include "ptx.cuh"
 
@@ -30,27 +29,17 @@ template <typename OutT>
 __global__ void __launch_bounds__(LN_WARPS * 32, 18) layernorm_kernel(const float* y, OutT* __restrict__ out,
                                                         const float* __restrict__ gamma,
                                                         const float* __restrict__ beta, int M,
-                                                        float* __restrict__ stats, Flow flow) {
-  // with a row-block dataflow each warp waits for its own row's block only
-  if (flow.ctr == nullptr || flow.wait_ev < 0) ptx::pdl_wait();
+                                                        float* __restrict__ stats) {
+  ptx::pdl_wait();
   ptx::pdl_trigger();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int row = blockIdx.x * LN_WARPS + warp;
   if (row >= M) return;
-  if (flow.ctr != nullptr && flow.wait_ev >= 0) {
-    // a give-up (2 s)
-    // leaves the row unwritten and uncounted, so the next kernel's bounded wait reports it
-    int ok = 1;
-    if (lane == 0) ok = flow_wait(flow, row / FLOW_BLOCK, nullptr, 2000000000ull) ? 1 : 0;
-    ok = __shfl_sync(0xffffffffu, ok, 0);
-    if (!ok) return;
-    __threadfence();
-  }
   const float* yr = y + (long)row * D;
   float v[32];
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    const float4 t = __ldcg(reinterpret_cast<const float4*>(yr + i * 128 + lane * 4));   // L2: written by another SM
+    const float4 t = *reinterpret_cast<const float4*>(yr + i * 128 + lane * 4);
     v[4 * i] = t.x; v[4 * i + 1] = t.y; v[4 * i + 2] = t.z; v[4 * i + 3] = t.w;
   }
   float s = 0.f;
@@ -85,24 +74,19 @@ __global__ void __launch_bounds__(LN_WARPS * 32, 18) layernorm_kernel(const floa
       *reinterpret_cast<float4*>(orow + c) = make_float4(r0, r1, r2, r3);
     }
   }
-  if (flow.ctr != nullptr && flow.sig_ev >= 0) {
-    __threadfence();
-    __syncwarp();
-    if (lane == 0) flow_signal(flow, row / FLOW_BLOCK, 1);
-  }
 }
 
 }  // namespace
 
 cudaError_t layernorm(const float* y, void* out, bool out_bf16, const float* gamma, const float* beta, int M,
-                      cudaStream_t st, float* stats, const Flow& flow) {
+                      cudaStream_t st, float* stats) {
   if (M <= 0) return cudaSuccess;
   const int grid = (M + LN_WARPS - 1) / LN_WARPS;
   if (out_bf16)
     return launch_kernel(layernorm_kernel<bf16>, dim3(grid), dim3(LN_WARPS * 32), 0, st, y, static_cast<bf16*>(out), gamma, beta,
-                         M, stats, flow);
+                         M, stats);
   return launch_kernel(layernorm_kernel<float>, dim3(grid), dim3(LN_WARPS * 32), 0, st, y, static_cast<float*>(out), gamma, beta,
-                       M, stats, flow);
+                       M, stats);
 }
 
 }  // namespace kd
