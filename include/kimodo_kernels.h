@@ -55,19 +55,6 @@ KIMODO_API int kimodo_gemm_bf16_pair(const void* A, int lda, const void* W, int 
                                      const void* resid, int ldr, void* out, int ldo, int M, int N, int K,
                                      int epilogue, int out_f32, int tile_n, void* stream);
 
-/*
- * The same product for a few hundred tokens, the kernel the denoiser uses below 1024
- * token rows for its layer projections: 128 x 256 output tiles, each shared by a cluster
- * of S = K / 256 CTAs (2..8) that take four 64-deep k-blocks apiece; the fp32 partial
- * sums are added in cluster-rank order through distributed shared memory, so every
- * output element sums the same k ranges in the same order at every M.  Arguments as
- * kimodo_gemm_bf16; epilogues KIMODO_EPI_BIAS and KIMODO_EPI_BIAS_GELU with bf16 output,
- * KIMODO_EPI_BIAS_RESID with fp32 output; N % 256 == 0, K a multiple of 512 up to 2048.
- */
-KIMODO_API int kimodo_gemm_bf16_splitk(const void* A, int lda, const void* W, int ldw, const float* bias,
-                                       const void* resid, int ldr, void* out, int ldo, int M, int N, int K,
-                                       int epilogue, int out_f32, void* stream);
-
 /* fp32 SIMT GEMM with the same epilogues; all operands fp32; K % 16 == 0,
  * lda, ldw multiples of 4. */
 KIMODO_API int kimodo_gemm_f32(const float* A, int lda, const float* W, int ldw, const float* bias,

@@ -110,53 +110,6 @@ def test_gemm_tcgen05_pair_vs_oracle(M, N, K, epi, out_f32, tile):
         np.testing.assert_allclose(got, ref, rtol=2 ** -8, atol=1e-5 * scale)
 
 
-SPLITK_CASES = [
-    # M, N, K, epilogue, out_f32 (cluster split-K kernel for a few hundred tokens)
-    (362, 3072, 1024, kb.EPI_BIAS, False),         # QKV of one prompt with CFG at 180 frames
-    (362, 1024, 1024, kb.EPI_BIAS_RESID, True),
-    (362, 2048, 1024, kb.EPI_BIAS_GELU, False),
-    (362, 1024, 2048, kb.EPI_BIAS_RESID, True),    # eight CTAs per cluster
-    (1, 1024, 1024, kb.EPI_BIAS, False),           # one row
-    (181, 2048, 2048, kb.EPI_BIAS_GELU, False),
-    (1000, 1024, 1024, kb.EPI_BIAS_RESID, True),   # eight row blocks, several waves
-    (77, 3072, 512, kb.EPI_BIAS, False),           # two CTAs per cluster
-]
-
-
-@pytest.mark.parametrize("M,N,K,epi,out_f32", SPLITK_CASES)
-def test_gemm_tcgen05_splitk_vs_oracle(M, N, K, epi, out_f32):
-    require_cuda()
-    seed = M * 13 + N * 5 + K
-    A = _bf16(synth.random_vectors((M, K), seed))
-    W = _bf16(synth.random_vectors((N, K), seed + 1, 0.05))
-    bias = torch.from_numpy(synth.random_vectors((N,), seed + 2, 0.1))
-    resid = torch.from_numpy(synth.random_vectors((M, N), seed + 3)) if epi == kb.EPI_BIAS_RESID else None
-    out = kb.gemm_bf16(A.cuda(), W.cuda(), bias.cuda(), epi, out_f32, None if resid is None else resid.cuda(),
-                       splitk=True)
-    torch.cuda.synchronize()
-    ref = _epi_ref(epi, ko.linear(_f64(A), _f64(W), bias.double().numpy()),
-                   None if resid is None else resid.double().numpy())
-    got = out.float().cpu().double().numpy()
-    scale = np.abs(ref).max()
-    if out_f32:
-        np.testing.assert_allclose(got, ref, rtol=0, atol=2e-5 * scale)
-    else:
-        np.testing.assert_allclose(got, ref, rtol=2 ** -8, atol=1e-5 * scale)
-
-
-def test_gemm_splitk_rows_independent_of_m():
-    """The split is fixed by (N, K): a row's result is the same bits at any row count."""
-    require_cuda()
-    N, K = 1024, 2048
-    A = _bf16(synth.random_vectors((700, K), 61)).cuda()
-    W = _bf16(synth.random_vectors((N, K), 62, 0.05)).cuda()
-    bias = torch.from_numpy(synth.random_vectors((N,), 63, 0.1)).cuda()
-    full = kb.gemm_bf16(A, W, bias, kb.EPI_BIAS, False, splitk=True)
-    part = kb.gemm_bf16(A[:131].contiguous(), W, bias, kb.EPI_BIAS, False, splitk=True)
-    torch.cuda.synchronize()
-    assert torch.equal(full[:131], part)
-
-
 def test_gemm_residual_in_place():
     """The residual epilogue may read and write the same fp32 buffer."""
     require_cuda()

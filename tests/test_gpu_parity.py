@@ -176,15 +176,14 @@ def test_packed_layout_equals_padded_layout(gpu_bf16, gpu_fp32, precision):
 def test_c4_full_size_sampled(gpu_bf16, oracle_refs):
     """100-step generation at B=16, T=150 (the throughput workload, as bench.py
     runs it): sequences 0 and 15 against the oracle over all 100 steps, sequence 15
-    also against the same prompt sampled alone; every output finite.  Alone, the
-    prompt's projections run on the split-K kernel (fewer than 1024 token rows), whose
-    sums take another order than the full-K CTA-pair tiles of the batch: the two agree
-    within the bf16 trajectory tolerance, not bit for bit."""
+    also against the same prompt sampled alone (every projection tile sums its full K
+    extent in the same order at any batch size, so the two agree bit for bit); every
+    output finite."""
     emb, null, noise, L = workload_inputs(C4)
     got = gpu_bf16.ddim_sample(emb, null, noise, L, C4[3], C4[4])
     assert np.all(np.isfinite(got))
     alone = gpu_bf16.ddim_sample(emb[15:16], null, noise[15:16], L[15:16], C4[3], C4[4])
-    report("c4 seq 15 batched vs alone rel-L2", rel_l2(got[15], alone[0]), TOL_BF16_TRAJ)
+    report("c4 seq 15 batched vs alone rel-L2", rel_l2(got[15], alone[0]), 1e-4)
     for b in (0, 15):
         report(f"bf16 sample c4 seq {b} (100 steps) trajectory rel-L2", rel_l2(got[b], oracle_refs.result(C4, b)),
                TOL_BF16_TRAJ)

@@ -43,7 +43,6 @@ SIGNATURES = [
     # include/kimodo_kernels.h
     ("kimodo_gemm_bf16", _I, [_P, _I, _P, _I, _P, _P, _I, _P, _I, _I, _I, _I, _I, _I, _I, _P]),
     ("kimodo_gemm_bf16_pair", _I, [_P, _I, _P, _I, _P, _P, _I, _P, _I, _I, _I, _I, _I, _I, _I, _P]),
-    ("kimodo_gemm_bf16_splitk", _I, [_P, _I, _P, _I, _P, _P, _I, _P, _I, _I, _I, _I, _I, _I, _P]),
     ("kimodo_gemm_f32", _I, [_P, _I, _P, _I, _P, _P, _I, _P, _I, _I, _I, _I, _I, _P]),
     ("kimodo_attention_bf16", _I, [_P, _P, _P, _I, _I, _P]),
     ("kimodo_attention_f32", _I, [_P, _P, _P, _I, _I, _P]),
@@ -154,10 +153,9 @@ def _cur_stream():
 
 # ------------------------------------------------------------ kernel-level calls (torch CUDA tensors)
 
-def gemm_bf16(A, W, bias, epilogue=EPI_BIAS, out_f32=False, resid=None, out=None, K=None, tile_n=0, pair=False,
-              splitk=False):
+def gemm_bf16(A, W, bias, epilogue=EPI_BIAS, out_f32=False, resid=None, out=None, K=None, tile_n=0, pair=False):
     """out = epilogue(A[:, :K] W[:, :K]^T + bias) on the tcgen05 GEMM (A, W bf16 CUDA tensors);
-    pair=True runs the CTA-pair kernel (256-row tiles), splitk=True the cluster split-K one."""
+    pair=True runs the CTA-pair kernel (256-row tiles)."""
     import torch
     lib = load_library()
     M, N = A.shape[0], W.shape[0]
@@ -167,11 +165,8 @@ def gemm_bf16(A, W, bias, epilogue=EPI_BIAS, out_f32=False, resid=None, out=None
     args = [_ptr_rows(A), A.stride(0), _ptr_rows(W), W.stride(0), _ptr(bias), _ptr_rows(resid),
             0 if resid is None else resid.stride(0), _ptr_rows(out), out.stride(0), M, N, K,
             int(epilogue), int(bool(out_f32))]
-    if splitk:
-        _check(lib.kimodo_gemm_bf16_splitk(*args, _cur_stream()))
-    else:
-        fn = lib.kimodo_gemm_bf16_pair if pair else lib.kimodo_gemm_bf16
-        _check(fn(*args, int(tile_n), _cur_stream()))
+    fn = lib.kimodo_gemm_bf16_pair if pair else lib.kimodo_gemm_bf16
+    _check(fn(*args, int(tile_n), _cur_stream()))
     return out
 
 

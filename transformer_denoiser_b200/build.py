@@ -18,7 +18,7 @@ BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(HERE, "libkimodo.so")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
-SOURCES = ["gemm_tc.cu", "gemm_tc2.cu", "gemm_splitk.cu", "gemm_f32.cu", "attention.cu", "attention_tc.cu", "layernorm.cu", "motion.cu", "capi.cu"]
+SOURCES = ["gemm_tc.cu", "gemm_tc2.cu", "gemm_f32.cu", "attention.cu", "attention_tc.cu", "layernorm.cu", "motion.cu", "capi.cu"]
 
 
 def nvcc() -> str:

@@ -1,7 +1,8 @@
 // Masked multi-head self-attention on the tcgen05 tensor cores ("Kimodo WebGPU",
 // "WGSL compute shaders" table: multi-head self-attention with optional key masking).
 //
-// One CTA per (head, sequence, 128-query tile), two CTAs per SM up to 256 keys.
+// One CTA per (head, sequence, query tile), two CTAs per SM up to 256 keys; the S query
+// rows of a sequence are split into ceil(S / 128) tiles of equal size (151: 76 + 75).
 // Every key of a sequence fits in one pass (at most 301 tokens), so the softmax is
 // exact, not online:
 //   1. TMA stages the query tile (128 x 128), the keys and the upper half of the
@@ -114,7 +115,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   ptx::pdl_trigger();
   const long row0 = tok0 ? tok0[seq] : (long)seq * S_pad;
   const int S = tok0 ? tok0[seq + 1] - tok0[seq] : S_pad;
-  if (qt * QT >= S) return;   // uniform over the CTA: nothing allocated yet
+  // the sequence's query rows in ceil(S / 128) tiles of equal size (151 tokens: 76 + 75
+  // rows, so that neither CTA of a (head, sequence) is left with a short tail)
+  const int n_qt = (S + QT - 1) / QT;
+  const int qrows = (S + n_qt - 1) / n_qt;
+  const int q0 = qt * qrows;                 // first query row of this tile
+  if (qt >= n_qt) return;   // uniform over the CTA: nothing allocated yet
   int n_valid = 1 + lengths[seq % len_mod];
   n_valid = n_valid < 1 ? 1 : (n_valid > S ? S : n_valid);
   const int n_cols = (n_valid + 15) & ~15;                 // MMA N for S = Q K^T, K range of O = P V
@@ -134,7 +140,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       // and the CTA barrier so that their latency overlaps the set-up
       ptx::tma_prefetch_desc(&tmQ);
       ptx::tma_prefetch_desc(&tmKV);
-      const int qrow = (int)row0 + qt * QT;
+      const int qrow = (int)row0 + q0;
       ptx::mbar_arrive_expect_tx(bar_qk, Q_BYTES + (uint32_t)n_boxes * 2 * KB_ROWS * 128);
       for (int hf = 0; hf < 2; ++hf) ptx::tma_load_2d(sQ + hf * (QT * 128), &tmQ, bar_qk, h * DH + hf * 64, qrow);
       for (int b = 0; b < n_boxes; ++b)
@@ -218,7 +224,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     const float sc = 0.08838834764831845f * 1.4426950408889634f;   // log2(e) / sqrt(128)
     // query rows of this tile that exist: whole warps past them skip the softmax and the
     // epilogue (TMEM loads are warp-collective), single lanes skip their arithmetic
-    const int rows_valid = S - qt * QT < QT ? S - qt * QT : QT;
+    const int rows_valid = S - q0 < qrows ? S - q0 : qrows;
     const bool warp_rows = q * 32 < rows_valid;
     const bool row_ok = r < rows_valid;
     bool ok = true;
@@ -291,7 +297,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       const float inv = 1.f / l;
       const bool full = q * 32 + 32 <= rows_valid;
       uint8_t* stg = smem + (size_t)ew * 4096 + (size_t)lane * 128;
-      bf16* orow = out + (row0 + qt * QT + r) * D + h * DH + kh * 64;
+      bf16* orow = out + (row0 + q0 + r) * D + h * DH + kh * 64;
       for (int c0 = 0; c0 < 64; c0 += 16) {
         float v[16];
         ptx::tmem_ld(tmem_base + lane_addr + o_col + kh * 64 + c0, v);
@@ -313,7 +319,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         ptx::fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
-          ptx::tma_store_2d(&tmO, sQ + (uint32_t)ew * 4096, h * DH + kh * 64, (int)row0 + qt * QT + q * 32);
+          ptx::tma_store_2d(&tmO, sQ + (uint32_t)ew * 4096, h * DH + kh * 64, (int)row0 + q0 + q * 32);
           ptx::bulk_commit();
           ptx::bulk_wait_all();
         }

@@ -213,12 +213,6 @@ int gemm(kimodo_ctx* c, const void* A, int lda, const void* W, int ldw, int M, i
       return launch(c, cls_override >= 0 ? cls_override : CLS_GEMM_TC, flops, bytes, st, "gemm_tc2",
                     [&] { return gemm_tc2(g, bn, kind, out_f32, ep, c->derr, st); });
     }
-    // a few hundred tokens: the layer projections split K over a cluster (the chain of
-    // MMA instructions of a full-K tile, not the bytes, would set the time)
-    if (M < 1024 && gemm_splitk_supports(kind, out_f32) && gemm_splitk_factor(N, K) >= 2) {
-      return launch(c, cls_override >= 0 ? cls_override : CLS_GEMM_TC, flops, bytes, st, "gemm_splitk",
-                    [&] { return gemm_splitk(g, kind, out_f32, ep, c->derr, st); });
-    }
     const int bn = pick_bn(c, M, N, kind, out_f32);
     return launch(c, cls_override >= 0 ? cls_override : CLS_GEMM_TC, flops, bytes, st, "gemm_tc",
                   [&] { return gemm_tc(g, bn, kind, out_f32, ep, c->derr, st, c->num_sms); });
@@ -663,8 +657,7 @@ int kimodo_load_weights(kimodo_ctx** out_ctx, const float* host_blob, size_t n_f
   if (precision == KIMODO_BF16 && !gemm_tc_available())
     return set_error(KIMODO_EUNSUPPORTED, "cuTensorMapEncodeTiled is unavailable in this driver");
 
-  if (gemm_tc_prepare() != cudaSuccess || gemm_tc2_prepare() != cudaSuccess || gemm_splitk_prepare() != cudaSuccess ||
-      attention_tc_prepare() != cudaSuccess) {
+  if (gemm_tc_prepare() != cudaSuccess || gemm_tc2_prepare() != cudaSuccess || attention_tc_prepare() != cudaSuccess) {
     cudaGetLastError();
     return set_error(KIMODO_EUNSUPPORTED, "kernel attributes could not be set on device %d", device);
   }
@@ -1128,7 +1121,6 @@ int prepared_device() {
   if (!done[dev]) {
     KD_CUDA(gemm_tc_prepare());
     KD_CUDA(gemm_tc2_prepare());
-    KD_CUDA(gemm_splitk_prepare());
     KD_CUDA(attention_tc_prepare());
     done[dev] = true;
   }
@@ -1204,29 +1196,6 @@ int kimodo_gemm_bf16_pair(const void* A, int lda, const void* W, int ldw, const 
   ep.bias = bias; ep.out = out; ep.ldo = ldo; ep.resid = resid; ep.ldr = ldr; ep.N = N; ep.M = M;
   const int bn = tile_n ? tile_n : gemm_tc2_pick_bn(M, N, epilogue);
   KD_CUDA(gemm_tc2(g, bn, epilogue, out_f32 != 0, ep, kernel_error_word(), static_cast<cudaStream_t>(stream)));
-  return KIMODO_OK;
-}
-
-int kimodo_gemm_bf16_splitk(const void* A, int lda, const void* W, int ldw, const float* bias, const void* resid,
-                            int ldr, void* out, int ldo, int M, int N, int K, int epilogue, int out_f32,
-                            void* stream) {
-  g_last_error.clear();
-  KD_TRY(check_gemm_args(A, lda, W, ldw, bias, resid, out, ldo, M, N, K, epilogue));
-  if (lda % 8 || ldw % 8 || (reinterpret_cast<uintptr_t>(A) & 15) || (reinterpret_cast<uintptr_t>(W) & 15))
-    return set_error(KIMODO_EINVAL, "bf16 operands need 16-byte aligned rows (lda, ldw multiples of 8)");
-  if (ldo % 4 || (reinterpret_cast<uintptr_t>(out) & 15) || (epilogue == 3 && (ldr % 4 ||
-      (reinterpret_cast<uintptr_t>(resid) & 15))) || (reinterpret_cast<uintptr_t>(bias) & 15))
-    return set_error(KIMODO_EINVAL, "out, resid and bias need 16-byte alignment and ldo, ldr multiples of 4");
-  if (!gemm_splitk_supports(epilogue, out_f32 != 0))
-    return set_error(KIMODO_EINVAL, "split-K epilogues: bias or GELU with bf16 output, residual with fp32 output");
-  if (gemm_splitk_factor(N, K) < 2)
-    return set_error(KIMODO_EINVAL, "split-K GEMM needs N % 256 == 0 and K / 256 in 2..8");
-  KD_TRY(prepared_device());
-  GemmArgs g;
-  g.A = A; g.B = W; g.M = M; g.N = N; g.K = K; g.lda = lda; g.ldb = ldw;
-  EpiParams ep;
-  ep.bias = bias; ep.out = out; ep.ldo = ldo; ep.resid = resid; ep.ldr = ldr; ep.N = N; ep.M = M;
-  KD_CUDA(gemm_splitk(g, epilogue, out_f32 != 0, ep, kernel_error_word(), static_cast<cudaStream_t>(stream)));
   return KIMODO_OK;
 }
 

@@ -118,6 +118,12 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
     ptx::tma_prefetch_desc(&tmB);
     ptx::tma_prefetch_desc(&tmO);
     if (C::RES) ptx::tma_prefetch_desc(&tmR);
+    // The weights do not depend on the previous kernel: while it still runs, the CTAs
+    // together pull this launch's whole weight matrix into L2 (one box of 64 columns x
+    // BN / 2 rows per CTA and step), so the first tiles of every round find it there.
+    const int nbr = (ep.N + BN / 2 - 1) / (BN / 2);   // row boxes covering N
+    for (int i = blockIdx.x; i < nbr * num_kb; i += gridDim.x)
+      ptx::tma_prefetch_l2_2d(&tmB, (i % num_kb) * BK, (i / num_kb) * (BN / 2));
   }
   if (warp == 1) {
     ptx::tmem_alloc_pair(ptx::smem_u32(tmem_slot), C::TMEM_COLS);

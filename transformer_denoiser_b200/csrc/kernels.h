@@ -38,16 +38,6 @@ cudaError_t gemm_tc2(const GemmArgs& g, int bn, int kind, bool out_f32, const Ep
 cudaError_t gemm_tc2_prepare();
 bool gemm_tc2_supports(int kind, bool out_f32);
 int gemm_tc2_pick_bn(int M, int N, int kind);
-// tcgen05 GEMM for a few hundred tokens: 128 x 256 output tiles, K split over a cluster of
-// S = gemm_splitk_factor(N, K) CTAs (four 64-deep k-blocks each); each CTA pushes its fp32
-// partial to the owners of the column slices, which sum the S partials in cluster-rank
-// order and run the usual epilogue.  EPI_BIAS / EPI_BIAS_GELU with bf16 output,
-// EPI_BIAS_RESID / EPI_BIAS_RESID_LN with fp32 output; N % 256 == 0.
-int gemm_splitk_factor(int N, int K);   // 0 when the shape does not split (S outside 2..8)
-bool gemm_splitk_supports(int kind, bool out_f32);
-cudaError_t gemm_splitk(const GemmArgs& g, int kind, bool out_f32, const EpiParams& ep, DevError* err,
-                        cudaStream_t st);
-cudaError_t gemm_splitk_prepare();
 // Set the dynamic shared-memory limits of every kernel instantiation (call once
 // per device before any launch or graph capture).
 cudaError_t gemm_tc_prepare();
