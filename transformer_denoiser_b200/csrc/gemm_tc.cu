@@ -45,8 +45,14 @@ constexpr uint32_t tmem_cols_for(uint32_t n) {
 
 template <int BN, int STAGES>
 struct TcCfg {
-  static constexpr uint32_t A_BYTES = BM * BK * 2;
-  static constexpr uint32_t B_BYTES = BN * BK * 2;
+  // K columns per pipeline stage: KA swizzle atoms of 64 (one TMA box each).  Below N = 256
+  // two atoms per stage halve the stage hand-offs (wait, fence, commit: about 200 ns on
+  // the issuing thread, more than the MMA time of a 64-column step at N <= 128).
+  static constexpr int KA = BN <= 128 ? 2 : 1;
+  static constexpr uint32_t ATOM_A = BM * 128;          // one 64-column atom (128-byte rows)
+  static constexpr uint32_t ATOM_B = BN * 128;
+  static constexpr uint32_t A_BYTES = KA * ATOM_A;
+  static constexpr uint32_t B_BYTES = KA * ATOM_B;
   static constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr uint32_t TMEM_COLS = tmem_cols_for(2 * BN);
   static constexpr uint32_t NUM_BARS = 2 * STAGES + 5;
@@ -137,8 +143,13 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             break;
           }
           ptx::mbar_arrive_expect_tx(full_bar(stage), C::STAGE_BYTES);
-          ptx::tma_load_2d(sA + stage * C::A_BYTES, &tmA, full_bar(stage), kb * BK, m_blk * BM);
-          ptx::tma_load_2d(sB + stage * C::B_BYTES, &tmB, full_bar(stage), kb * BK, n_blk * BN);
+#pragma unroll
+          for (int at = 0; at < C::KA; ++at) {
+            ptx::tma_load_2d(sA + stage * C::A_BYTES + at * C::ATOM_A, &tmA, full_bar(stage), (kb * C::KA + at) * BK,
+                             m_blk * BM);
+            ptx::tma_load_2d(sB + stage * C::B_BYTES + at * C::ATOM_B, &tmB, full_bar(stage), (kb * C::KA + at) * BK,
+                             n_blk * BN);
+          }
           ++issued;
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
@@ -181,9 +192,9 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
           const uint32_t a0 = sA + stage * C::A_BYTES;
           const uint32_t b0 = sB + stage * C::B_BYTES;
 #pragma unroll
-          for (int k = 0; k < BK / 16; ++k) {
-            ptx::tc_mma_bf16(d_tmem, ptx::smem_desc_sw128(a0 + k * 32), ptx::smem_desc_sw128(b0 + k * 32),
-                             C::IDESC, (kb | k) != 0);
+          for (int k = 0; k < C::KA * BK / 16; ++k) {
+            ptx::tc_mma_bf16(d_tmem, ptx::smem_desc_sw128(a0 + (k >> 2) * C::ATOM_A + (k & 3) * 32),
+                             ptx::smem_desc_sw128(b0 + (k >> 2) * C::ATOM_B + (k & 3) * 32), C::IDESC, (kb | k) != 0);
           }
           ptx::tc_commit(empty_bar(stage));
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
@@ -312,7 +323,7 @@ cudaError_t launch_impl(const GemmArgs& g, const EpiParams& ep, DevError* err, c
   const int mt = (g.M + BM - 1) / BM, nt = (g.N + BN - 1) / BN;
   const int tiles = mt * nt;
   const int grid = tiles < num_sms ? tiles : num_sms;
-  const int kb = (g.K + BK - 1) / BK;
+  const int kb = (g.K + Cf::KA * BK - 1) / (Cf::KA * BK);
   return launch_kernel(kern, dim3(grid), dim3(NUM_THREADS), Cf::SMEM, st, ta, tb, mt, nt, kb, ep, err);
 }
 
@@ -373,23 +384,23 @@ static cudaError_t dispatch(const GemmArgs& g, int bn, int kind, bool out_f32, c
   KD_TC(256, 4, EPI_BIAS_RESID, float)
   KD_TC(256, 4, EPI_BIAS_RESID_LN, float)
   KD_TC(256, 4, EPI_INPROJ, bf16)
-  KD_TC(128, 6, EPI_BIAS, bf16)
-  KD_TC(128, 6, EPI_BIAS, float)
-  KD_TC(128, 6, EPI_BIAS_GELU, bf16)
-  KD_TC(128, 6, EPI_BIAS_SILU, bf16)
-  KD_TC(128, 6, EPI_BIAS_RESID, float)
-  KD_TC(128, 6, EPI_BIAS_RESID_LN, float)
-  KD_TC(128, 6, EPI_INPROJ, bf16)
-  KD_TC(128, 6, EPI_OUTPROJ, float)
-  KD_TC(64, 8, EPI_BIAS, bf16)
-  KD_TC(64, 8, EPI_BIAS_GELU, bf16)
-  KD_TC(64, 8, EPI_BIAS_RESID, float)
-  KD_TC(64, 8, EPI_BIAS_RESID_LN, float)
-  KD_TC(32, 8, EPI_BIAS, bf16)
-  KD_TC(32, 8, EPI_BIAS_GELU, bf16)
-  KD_TC(32, 8, EPI_BIAS_RESID, float)
-  KD_TC(32, 8, EPI_BIAS_RESID_LN, float)
-  KD_TC(16, 8, EPI_OUTPROJ, float)
+  KD_TC(128, 3, EPI_BIAS, bf16)
+  KD_TC(128, 3, EPI_BIAS, float)
+  KD_TC(128, 3, EPI_BIAS_GELU, bf16)
+  KD_TC(128, 3, EPI_BIAS_SILU, bf16)
+  KD_TC(128, 3, EPI_BIAS_RESID, float)
+  KD_TC(128, 3, EPI_BIAS_RESID_LN, float)
+  KD_TC(128, 3, EPI_INPROJ, bf16)
+  KD_TC(128, 3, EPI_OUTPROJ, float)
+  KD_TC(64, 4, EPI_BIAS, bf16)
+  KD_TC(64, 4, EPI_BIAS_GELU, bf16)
+  KD_TC(64, 4, EPI_BIAS_RESID, float)
+  KD_TC(64, 4, EPI_BIAS_RESID_LN, float)
+  KD_TC(32, 5, EPI_BIAS, bf16)
+  KD_TC(32, 5, EPI_BIAS_GELU, bf16)
+  KD_TC(32, 5, EPI_BIAS_RESID, float)
+  KD_TC(32, 5, EPI_BIAS_RESID_LN, float)
+  KD_TC(16, 5, EPI_OUTPROJ, float)
 #undef KD_TC
   return prep ? cudaSuccess : cudaErrorInvalidValue;
 }

@@ -41,8 +41,16 @@ constexpr uint32_t tmem_cols_for(uint32_t n) {
 
 template <int BN, int STAGES, int KIND>
 struct Tc2Cfg {
-  static constexpr uint32_t A_BYTES = BMC * BK * 2;
-  static constexpr uint32_t B_BYTES = (BN / 2) * BK * 2;
+  static constexpr bool RES = KIND == EPI_BIAS_RESID || KIND == EPI_BIAS_RESID_LN;
+  // K columns per pipeline stage: KA swizzle atoms of 64 (one TMA box each).  Two atoms
+  // halve the stage hand-offs per MMA (wait, fence, commit: measured about 200 ns on the
+  // issuing thread, more than the MMA time of a 64-column step below N = 256) and are
+  // faster once three stages fit; beside the residual tiles only two would (slower).
+  static constexpr int KA = RES ? 1 : 2;
+  static constexpr uint32_t ATOM_A = BMC * 128;          // one 64-column atom of A (128-byte rows)
+  static constexpr uint32_t ATOM_B = (BN / 2) * 128;
+  static constexpr uint32_t A_BYTES = KA * ATOM_A;
+  static constexpr uint32_t B_BYTES = KA * ATOM_B;
   static constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr uint32_t TMEM_COLS = tmem_cols_for(2 * BN);
   static constexpr int CW = 16;                         // columns per epilogue chunk
@@ -50,7 +58,6 @@ struct Tc2Cfg {
   static constexpr int PART_CH = (NCH + 1) / 2;
   static constexpr uint32_t STG_BYTES = 32 * CW * 4;     // one 32-row staging tile (fp32 size)
   // bytes of one staging row of the stored type (fp32 64, bf16 32): also the TMA swizzle span
-  static constexpr bool RES = KIND == EPI_BIAS_RESID || KIND == EPI_BIAS_RESID_LN;
   static constexpr int ROW_BYTES = CW * (RES ? 4 : 2);
   // staging tiles per epilogue warp: two alternating ones, or, with a residual, one per
   // chunk of the warp's tile share so the whole residual share is loaded ahead of the MMA
@@ -122,8 +129,9 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
     // together pull this launch's whole weight matrix into L2 (one box of 64 columns x
     // BN / 2 rows per CTA and step), so the first tiles of every round find it there.
     const int nbr = (ep.N + BN / 2 - 1) / (BN / 2);   // row boxes covering N
-    for (int i = blockIdx.x; i < nbr * num_kb; i += gridDim.x)
-      ptx::tma_prefetch_l2_2d(&tmB, (i % num_kb) * BK, (i / num_kb) * (BN / 2));
+    const int nkc = num_kb * C::KA;                      // column boxes covering K
+    for (int i = blockIdx.x; i < nbr * nkc; i += gridDim.x)
+      ptx::tma_prefetch_l2_2d(&tmB, (i % nkc) * BK, (i / nkc) * (BN / 2));
   }
   if (warp == 1) {
     ptx::tmem_alloc_pair(ptx::smem_u32(tmem_slot), C::TMEM_COLS);
@@ -160,8 +168,11 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
           }
           if (rank == 0) ptx::mbar_arrive_expect_tx(full_bar(stage), 2 * C::STAGE_BYTES);
           const uint32_t lbar = ptx::mapa_shared(full_bar(stage), 0);
-          ptx::tma_load_2d_pair(sA + stage * C::A_BYTES, &tmA, lbar, kb * BK, arow);
-          ptx::tma_load_2d_pair(sB + stage * C::B_BYTES, &tmB, lbar, kb * BK, brow);
+#pragma unroll
+          for (int at = 0; at < C::KA; ++at) {
+            ptx::tma_load_2d_pair(sA + stage * C::A_BYTES + at * C::ATOM_A, &tmA, lbar, (kb * C::KA + at) * BK, arow);
+            ptx::tma_load_2d_pair(sB + stage * C::B_BYTES + at * C::ATOM_B, &tmB, lbar, (kb * C::KA + at) * BK, brow);
+          }
           ++issued;
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
@@ -205,9 +216,10 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
           const uint32_t a0 = sA + stage * C::A_BYTES;
           const uint32_t b0 = sB + stage * C::B_BYTES;
 #pragma unroll
-          for (int k = 0; k < BK / 16; ++k)
-            ptx::tc_mma_bf16_pair(d_tmem, ptx::smem_desc_sw128(a0 + k * 32), ptx::smem_desc_sw128(b0 + k * 32),
-                                  C::IDESC, (kb | k) != 0);
+          for (int k = 0; k < C::KA * BK / 16; ++k)
+            ptx::tc_mma_bf16_pair(d_tmem, ptx::smem_desc_sw128(a0 + (k >> 2) * C::ATOM_A + (k & 3) * 32),
+                                  ptx::smem_desc_sw128(b0 + (k >> 2) * C::ATOM_B + (k & 3) * 32), C::IDESC,
+                                  (kb | k) != 0);
           ptx::tc_commit_pair(empty_bar(stage), 0x3);
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
@@ -462,21 +474,37 @@ struct Tc2Launcher {
     cfg.attrs = attr;
     cfg.numAttrs = pdl_enabled() ? 2 : 1;
     return cudaLaunchKernelEx(&cfg, gemm_tc2_kernel<BN, STAGES, KIND, OutT>, ta, tb, to, tr, mt, nt,
-                              (g.K + BK - 1) / BK, ep, err);
+                              (g.K + Cf::KA * BK - 1) / (Cf::KA * BK), ep, err);
   }
 };
 template <int BN, int STAGES, int KIND, typename OutT>
 int Tc2Launcher<BN, STAGES, KIND, OutT>::max_clusters = 0;
 
-// (tile N, pipeline stages) per instantiation: stages fill the shared memory left
-// by the epilogue staging tiles
-#define KD_TC2_LIST(X)                                  \
-  X(256, 6, EPI_BIAS, bf16) X(208, 6, EPI_BIAS, bf16)   \
-  X(160, 7, EPI_BIAS, bf16) X(144, 7, EPI_BIAS, bf16)   \
-  X(256, 6, EPI_BIAS_GELU, bf16) X(208, 6, EPI_BIAS_GELU, bf16) \
-  X(160, 7, EPI_BIAS_GELU, bf16) X(144, 7, EPI_BIAS_GELU, bf16) \
-  X(160, 5, EPI_BIAS_RESID, float) X(144, 5, EPI_BIAS_RESID, float)   \
-  X(160, 5, EPI_BIAS_RESID_LN, float) X(144, 5, EPI_BIAS_RESID_LN, float)
+// Pipeline stages of a (tile N, epilogue) instantiation: as many as fit in the shared
+// memory left by the epilogue staging tiles, at most 8.
+template <int BN, int KIND>
+constexpr int tc2_stages() {
+  using C1 = Tc2Cfg<BN, 1, KIND>;
+  const long fixed = 1024 + (long)C1::EPI_BYTES + (5 + C1::NBUF * EPI_WARPS) * 8 + 16;
+  const long st = (232448 - fixed) / ((long)C1::STAGE_BYTES + 16);
+  return st > 8 ? 8 : (int)st;
+}
+#define KD_TC2_ST(BN_, KIND_) tc2_stages<BN_, KIND_>()
+
+// (tile N, epilogue, output type) per instantiation
+#define KD_TC2_LIST(X)                                                                     \
+  X(256, KD_TC2_ST(256, EPI_BIAS), EPI_BIAS, bf16)                                         \
+  X(208, KD_TC2_ST(208, EPI_BIAS), EPI_BIAS, bf16)                                         \
+  X(160, KD_TC2_ST(160, EPI_BIAS), EPI_BIAS, bf16)                                         \
+  X(144, KD_TC2_ST(144, EPI_BIAS), EPI_BIAS, bf16)                                         \
+  X(256, KD_TC2_ST(256, EPI_BIAS_GELU), EPI_BIAS_GELU, bf16)                               \
+  X(208, KD_TC2_ST(208, EPI_BIAS_GELU), EPI_BIAS_GELU, bf16)                               \
+  X(160, KD_TC2_ST(160, EPI_BIAS_GELU), EPI_BIAS_GELU, bf16)                               \
+  X(144, KD_TC2_ST(144, EPI_BIAS_GELU), EPI_BIAS_GELU, bf16)                               \
+  X(160, KD_TC2_ST(160, EPI_BIAS_RESID), EPI_BIAS_RESID, float)                            \
+  X(144, KD_TC2_ST(144, EPI_BIAS_RESID), EPI_BIAS_RESID, float)                            \
+  X(160, KD_TC2_ST(160, EPI_BIAS_RESID_LN), EPI_BIAS_RESID_LN, float)                      \
+  X(144, KD_TC2_ST(144, EPI_BIAS_RESID_LN), EPI_BIAS_RESID_LN, float)
 
 }  // namespace
 
@@ -505,8 +533,8 @@ int gemm_tc2_pick_bn(int M, int N, int kind) {
   const bool res = kind == EPI_BIAS_RESID || kind == EPI_BIAS_RESID_LN;
   const int* cands = res ? resid : all;
   const int ncand = res ? 2 : 4;
-  const int pairs = Tc2Launcher<256, 6, EPI_BIAS, bf16>::max_clusters > 0
-                        ? Tc2Launcher<256, 6, EPI_BIAS, bf16>::max_clusters : 74;
+  using L256 = Tc2Launcher<256, KD_TC2_ST(256, EPI_BIAS), EPI_BIAS, bf16>;
+  const int pairs = L256::max_clusters > 0 ? L256::max_clusters : 74;
   const long mt = (M + 2 * BMC - 1) / (2 * BMC);
   int best = cands[0];
   long best_cost = -1;
