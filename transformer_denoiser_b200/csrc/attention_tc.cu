@@ -37,7 +37,7 @@ namespace kd {
 namespace {
 
 constexpr int QT = 128;                    // query rows per CTA
-constexpr int KB_ROWS = 32;                // key rows per TMA box
+constexpr int KB_ROWS = 32;                // key rows are staged in multiples of 32
 constexpr int SM_WARPS = 8;                // softmax / epilogue warps
 constexpr int NUM_THREADS = 64 + 32 * SM_WARPS;
 constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;
@@ -86,7 +86,7 @@ __device__ __forceinline__ uint64_t smem_desc_sw128_mn(uint32_t saddr, uint32_t 
 __global__ void __launch_bounds__(NUM_THREADS, 2)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmKV,
                const __grid_constant__ CUtensorMap tmO, bf16* __restrict__ out, const int* __restrict__ lengths, int len_mod, int S_pad, int ka,
-               uint32_t tmem_cols, uint32_t o_col, const int* __restrict__ tok0, DevError* err) {
+               uint32_t tmem_cols, uint32_t o_col, const int* __restrict__ tok0, int kbox, DevError* err) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t kp = kp_of(ka);
@@ -121,10 +121,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   const int qrows = (S + n_qt - 1) / n_qt;
   const int q0 = qt * qrows;                 // first query row of this tile
   if (qt >= n_qt) return;   // uniform over the CTA: nothing allocated yet
-  int n_valid = 1 + lengths[seq % len_mod];
-  n_valid = n_valid < 1 ? 1 : (n_valid > S ? S : n_valid);
-  const int n_cols = (n_valid + 15) & ~15;                 // MMA N for S = Q K^T, K range of O = P V
-  const int n_boxes = (n_valid + KB_ROWS - 1) / KB_ROWS;   // 32-row key / value boxes
+  // key / value boxes of kbox rows covering the sequence's tokens (not only the valid ones,
+  // so that the loads need not wait for the lengths)
+  const int n_boxes = (S + kbox - 1) / kbox;
 
   if (threadIdx.x == 0) {
     ptx::mbar_init(bar_qk, 1);
@@ -141,17 +140,20 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       ptx::tma_prefetch_desc(&tmQ);
       ptx::tma_prefetch_desc(&tmKV);
       const int qrow = (int)row0 + q0;
-      ptx::mbar_arrive_expect_tx(bar_qk, Q_BYTES + (uint32_t)n_boxes * 2 * KB_ROWS * 128);
+      ptx::mbar_arrive_expect_tx(bar_qk, Q_BYTES + (uint32_t)(n_boxes * kbox) * 2 * 128);
       for (int hf = 0; hf < 2; ++hf) ptx::tma_load_2d(sQ + hf * (QT * 128), &tmQ, bar_qk, h * DH + hf * 64, qrow);
       for (int b = 0; b < n_boxes; ++b)
         for (int hf = 0; hf < 2; ++hf)
-          ptx::tma_load_2d(sK + (uint32_t)(hf * ka + b * KB_ROWS) * 128, &tmKV, bar_qk, D + h * DH + hf * 64,
-                           (int)row0 + b * KB_ROWS);
-      ptx::mbar_arrive_expect_tx(bar_v1, (uint32_t)n_boxes * KB_ROWS * 128);
+          ptx::tma_load_2d(sK + (uint32_t)(hf * ka + b * kbox) * 128, &tmKV, bar_qk, D + h * DH + hf * 64,
+                           (int)row0 + b * kbox);
+      ptx::mbar_arrive_expect_tx(bar_v1, (uint32_t)(n_boxes * kbox) * 128);
       for (int b = 0; b < n_boxes; ++b)
-        ptx::tma_load_2d(sV1 + (uint32_t)(b * KB_ROWS) * 128, &tmKV, bar_v1, 2 * D + h * DH + 64, (int)row0 + b * KB_ROWS);
+        ptx::tma_load_2d(sV1 + (uint32_t)(b * kbox) * 128, &tmKV, bar_v1, 2 * D + h * DH + 64, (int)row0 + b * kbox);
     }
   }
+  int n_valid = 1 + lengths[seq % len_mod];
+  n_valid = n_valid < 1 ? 1 : (n_valid > S ? S : n_valid);
+  const int n_cols = (n_valid + 15) & ~15;                 // MMA N for S = Q K^T, K range of O = P V
   if (warp == 1) {
     ptx::tmem_alloc(ptx::smem_u32(tmem_slot), tmem_cols);
     ptx::tmem_relinquish();
@@ -168,9 +170,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       // the lower value half: into the query buffer once S = Q K^T no longer reads it
       bool ok = v0q ? ptx::mbar_wait_bounded(bar_s, 0, abort, WAIT_LIMIT_NS) : true;
       if (ok) {
-        ptx::mbar_arrive_expect_tx(bar_v0, (uint32_t)n_boxes * KB_ROWS * 128);
+        ptx::mbar_arrive_expect_tx(bar_v0, (uint32_t)(n_boxes * kbox) * 128);
         for (int b = 0; b < n_boxes; ++b)
-          ptx::tma_load_2d(sV0 + (uint32_t)(b * KB_ROWS) * 128, &tmKV, bar_v0, 2 * D + h * DH, (int)row0 + b * KB_ROWS);
+          ptx::tma_load_2d(sV0 + (uint32_t)(b * kbox) * 128, &tmKV, bar_v0, 2 * D + h * DH, (int)row0 + b * kbox);
       } else if (!*abort) {
         record_timeout(err, abort);
       }
@@ -242,13 +244,32 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     if (ok && warp_rows) {
       ptx::tc_fence_after();
       // pass 1: row maximum over this half's valid keys
-      for (int c0 = c_beg; c0 < c_end; c0 += 16) {
-        float v[16];
-        ptx::tmem_ld(tmem_base + lane_addr + c0, v);
-        ptx::tmem_ld_wait();
+      for (int c0 = c_beg; c0 < c_end; c0 += 32) {
+        if (c_end - c0 >= 32) {
+          float v[32];
+          ptx::tmem_ld(tmem_base + lane_addr + c0, v);
+          ptx::tmem_ld_wait();
+          if (c0 + 32 <= n_valid) {   // all keys valid: no masks, two independent chains
+            float ma = v[0], mb = v[1];
 #pragma unroll
-        for (int j = 0; j < 16; ++j)
-          if (c0 + j < n_valid) m = fmaxf(m, v[j]);
+            for (int j = 2; j < 32; j += 2) {
+              ma = fmaxf(ma, v[j]);
+              mb = fmaxf(mb, v[j + 1]);
+            }
+            m = fmaxf(m, fmaxf(ma, mb));
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (c0 + j < n_valid) m = fmaxf(m, v[j]);
+          }
+        } else {
+          float v[16];
+          ptx::tmem_ld(tmem_base + lane_addr + c0, v);
+          ptx::tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            if (c0 + j < n_valid) m = fmaxf(m, v[j]);
+        }
       }
     }
     xmax[kh * QT + r] = m;
@@ -258,26 +279,53 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     const float msc = m * sc;
     float l = 0.f;
     if (ok && warp_rows) {
-      // pass 2: p = 2^(s sc - m sc) on valid keys, 0 elsewhere; P row r into 64-key blocks (swizzled)
-      for (int c0 = c_beg; c0 < c_end; c0 += 16) {
-        float v[16];
-        ptx::tmem_ld(tmem_base + lane_addr + c0, v);
-        ptx::tmem_ld_wait();
-        if (!row_ok) continue;
+      // pass 2: p = 2^(s sc - m sc) on valid keys, 0 elsewhere; P row r into 64-key blocks
+      // (swizzled).  The pass is bound by instruction issue: chunks of valid keys only skip
+      // the masks, and the scaling and the row sum run on pairs (f32x2 FMA and add).
+      float2 l2 = make_float2(0.f, 0.f);
+      const float2 sc2 = make_float2(sc, sc), nmsc2 = make_float2(-msc, -msc);
+      auto p_chunk = [&](const float* v, int c) {   // keys c .. c + 15
         uint32_t w[8];
+        if (c + 16 <= n_valid) {
 #pragma unroll
-        for (int j = 0; j < 16; j += 2) {
-          const float p0 = c0 + j < n_valid ? ex2_approx(fmaf(v[j], sc, -msc)) : 0.f;
-          const float p1 = c0 + j + 1 < n_valid ? ex2_approx(fmaf(v[j + 1], sc, -msc)) : 0.f;
-          l += p0 + p1;
-          w[j / 2] = bf16x2_bits(p0, p1);
+          for (int j = 0; j < 16; j += 2) {
+            const float2 x = __ffma2_rn(make_float2(v[j], v[j + 1]), sc2, nmsc2);
+            const float p0 = ex2_approx(x.x), p1 = ex2_approx(x.y);
+            l2 = __fadd2_rn(l2, make_float2(p0, p1));
+            w[j / 2] = bf16x2_bits(p0, p1);
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < 16; j += 2) {
+            const float p0 = c + j < n_valid ? ex2_approx(fmaf(v[j], sc, -msc)) : 0.f;
+            const float p1 = c + j + 1 < n_valid ? ex2_approx(fmaf(v[j + 1], sc, -msc)) : 0.f;
+            l2 = __fadd2_rn(l2, make_float2(p0, p1));
+            w[j / 2] = bf16x2_bits(p0, p1);
+          }
         }
-        // 16 keys = two 16-byte chunks of row r in block c0 / 64
-        uint8_t* blk = smem + Q_BYTES + (size_t)(c0 / 64) * (QT * 128) + (size_t)r * 128;
-        const int ch = (c0 % 64) / 8;
+        // 16 keys = two 16-byte chunks of row r in block c / 64
+        uint8_t* blk = smem + Q_BYTES + (size_t)(c / 64) * (QT * 128) + (size_t)r * 128;
+        const int ch = (c % 64) / 8;
         *reinterpret_cast<uint4*>(blk + (((ch) ^ (r & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
         *reinterpret_cast<uint4*>(blk + (((ch + 1) ^ (r & 7)) << 4)) = make_uint4(w[4], w[5], w[6], w[7]);
+      };
+      for (int c0 = c_beg; c0 < c_end; c0 += 32) {
+        if (c_end - c0 >= 32) {
+          float v[32];
+          ptx::tmem_ld(tmem_base + lane_addr + c0, v);
+          ptx::tmem_ld_wait();
+          if (!row_ok) continue;
+          p_chunk(v, c0);
+          p_chunk(v + 16, c0 + 16);
+        } else {
+          float v[16];
+          ptx::tmem_ld(tmem_base + lane_addr + c0, v);
+          ptx::tmem_ld_wait();
+          if (!row_ok) continue;
+          p_chunk(v, c0);
+        }
       }
+      l = l2.x + l2.y;
     }
     xsum[kh * QT + r] = l;
     if (ok) ok = ptx::mbar_wait_bounded(bar_v0, 0, abort, WAIT_LIMIT_NS);
@@ -353,10 +401,15 @@ cudaError_t attention_tc(const bf16* qkv, bf16* out, int M, const int* lengths, 
   if (nseq <= 0 || S <= 0 || M <= 0) return cudaSuccess;
   if (S > MAX_FRAMES + 1) return cudaErrorInvalidValue;
   CUtensorMap tq, tkv, to;
-  if (make_tmap_bf16(&tq, qkv, M, 3 * D, 3 * D, QT) || make_tmap_bf16(&tkv, qkv, M, 3 * D, 3 * D, KB_ROWS) ||
+  const int ka = ((S + KB_ROWS - 1) / KB_ROWS) * KB_ROWS;
+  // key / value rows per TMA box (a divisor of ka, so that the boxes a sequence needs never
+  // pass the ka staged rows): every issued box costs the issuing thread time, so the padded
+  // layout (every sequence S tokens) takes its keys in one box (two past 256 rows); the
+  // packed layout, whose sequences may be far shorter than S, in boxes of 32 rows
+  const int kbox = tok0 != nullptr ? KB_ROWS : (ka <= 256 ? ka : ka / 2);
+  if (make_tmap_bf16(&tq, qkv, M, 3 * D, 3 * D, QT) || make_tmap_bf16(&tkv, qkv, M, 3 * D, 3 * D, kbox) ||
       make_tmap_plain(&to, out, 2, M, D, D, 64, 32, 128))
     return cudaErrorInvalidValue;
-  const int ka = ((S + KB_ROWS - 1) / KB_ROWS) * KB_ROWS;
   // up to 256 keys S and then O share a 256-column TMEM allocation (two CTAs per SM);
   // beyond, S takes columns 0..303 and O 320..447 of 512
   const int n_cols_max = (S + 15) & ~15;
@@ -364,7 +417,7 @@ cudaError_t attention_tc(const bf16* qkv, bf16* out, int M, const int* lengths, 
   const uint32_t o_col = n_cols_max <= 256 ? 0u : 320u;
   dim3 grid(H, nseq, (S + QT - 1) / QT);
   return launch_kernel(attn_tc_kernel, grid, dim3(NUM_THREADS), smem_bytes(ka), st, tq, tkv, to, out, lengths, len_mod,
-                       S, ka, tmem_cols, o_col, tok0, err);
+                       S, ka, tmem_cols, o_col, tok0, kbox, err);
 }
 
 }  // namespace kd
