@@ -111,6 +111,23 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int h = blockIdx.x, seq = blockIdx.y, qt = blockIdx.z;
+  // set-up that reads nothing an earlier kernel writes (barriers, TMEM, descriptors) runs
+  // before the dependency wait, overlapping the previous kernel's tail
+  if (threadIdx.x == 0) {
+    ptx::mbar_init(bar_qk, 1);
+    ptx::mbar_init(bar_v1, 1);
+    ptx::mbar_init(bar_v0, 1);
+    ptx::mbar_init(bar_s, 1);
+    ptx::mbar_init(bar_p, SM_WARPS);
+    ptx::mbar_init(bar_o, 1);
+    ptx::fence_mbar_init();
+    ptx::tma_prefetch_desc(&tmQ);
+    ptx::tma_prefetch_desc(&tmKV);
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc(ptx::smem_u32(tmem_slot), tmem_cols);
+    ptx::tmem_relinquish();
+  }
   ptx::pdl_wait();
   ptx::pdl_trigger();
   const long row0 = tok0 ? tok0[seq] : (long)seq * S_pad;
@@ -120,49 +137,45 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   const int n_qt = (S + QT - 1) / QT;
   const int qrows = (S + n_qt - 1) / n_qt;
   const int q0 = qt * qrows;                 // first query row of this tile
-  if (qt >= n_qt) return;   // uniform over the CTA: nothing allocated yet
+  const bool live = qt < n_qt;               // uniform over the CTA
   // key / value boxes of kbox rows covering the sequence's tokens (not only the valid ones,
   // so that the loads need not wait for the lengths)
   const int n_boxes = (S + kbox - 1) / kbox;
 
-  if (threadIdx.x == 0) {
-    ptx::mbar_init(bar_qk, 1);
-    ptx::mbar_init(bar_v1, 1);
-    ptx::mbar_init(bar_v0, 1);
-    ptx::mbar_init(bar_s, 1);
-    ptx::mbar_init(bar_p, SM_WARPS);
-    ptx::mbar_init(bar_o, 1);
-    ptx::fence_mbar_init();
-    *abort = (err != nullptr && *reinterpret_cast<volatile int*>(&err->code) != 0) ? 1 : 0;
+  if (warp == 0) {
+    if (lane == 0) *abort = (!live || (err != nullptr && *reinterpret_cast<volatile int*>(&err->code) != 0)) ? 1 : 0;
+    __syncwarp();
     if (!*abort) {
-      // the query tile, the keys and the upper value half, issued before the TMEM allocation
-      // and the CTA barrier so that their latency overlaps the set-up
-      ptx::tma_prefetch_desc(&tmQ);
-      ptx::tma_prefetch_desc(&tmKV);
-      const int qrow = (int)row0 + q0;
-      ptx::mbar_arrive_expect_tx(bar_qk, Q_BYTES + (uint32_t)(n_boxes * kbox) * 2 * 128);
-      for (int hf = 0; hf < 2; ++hf) ptx::tma_load_2d(sQ + hf * (QT * 128), &tmQ, bar_qk, h * DH + hf * 64, qrow);
-      for (int b = 0; b < n_boxes; ++b)
-        for (int hf = 0; hf < 2; ++hf)
-          ptx::tma_load_2d(sK + (uint32_t)(hf * ka + b * kbox) * 128, &tmKV, bar_qk, D + h * DH + hf * 64,
-                           (int)row0 + b * kbox);
-      ptx::mbar_arrive_expect_tx(bar_v1, (uint32_t)(n_boxes * kbox) * 128);
-      for (int b = 0; b < n_boxes; ++b)
+      // the query tile, the keys and the upper value half, one box per lane (issue from one
+      // thread costs tens of ns per box), before the CTA barrier so that their latency
+      // overlaps it.  A box may land before its barrier's expect-tx: the phase cannot complete
+      // before that arrival.
+      if (lane == 0) {
+        ptx::mbar_arrive_expect_tx(bar_qk, Q_BYTES + (uint32_t)(n_boxes * kbox) * 2 * 128);
+        ptx::mbar_arrive_expect_tx(bar_v1, (uint32_t)(n_boxes * kbox) * 128);
+      }
+      if (lane < 2) {
+        ptx::tma_load_2d(sQ + lane * (QT * 128), &tmQ, bar_qk, h * DH + lane * 64, (int)row0 + q0);
+      } else if (lane < 2 + 2 * n_boxes) {
+        const int hf = (lane - 2) / n_boxes, b = (lane - 2) % n_boxes;
+        ptx::tma_load_2d(sK + (uint32_t)(hf * ka + b * kbox) * 128, &tmKV, bar_qk, D + h * DH + hf * 64,
+                         (int)row0 + b * kbox);
+      } else if (lane < 2 + 3 * n_boxes) {
+        const int b = lane - 2 - 2 * n_boxes;
         ptx::tma_load_2d(sV1 + (uint32_t)(b * kbox) * 128, &tmKV, bar_v1, 2 * D + h * DH + 64, (int)row0 + b * kbox);
+      }
     }
   }
-  int n_valid = 1 + lengths[seq % len_mod];
-  n_valid = n_valid < 1 ? 1 : (n_valid > S ? S : n_valid);
-  const int n_cols = (n_valid + 15) & ~15;                 // MMA N for S = Q K^T, K range of O = P V
-  if (warp == 1) {
-    ptx::tmem_alloc(ptx::smem_u32(tmem_slot), tmem_cols);
-    ptx::tmem_relinquish();
-  }
+  // read here, used after the barrier: the load's latency overlaps it
+  const int len = live ? lengths[seq % len_mod] : 0;
   ptx::tc_fence_before();
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const bool skip = *abort != 0;
+  int n_valid = 1 + len;
+  n_valid = n_valid < 1 ? 1 : (n_valid > S ? S : n_valid);
+  const int n_cols = (n_valid + 15) & ~15;                 // MMA N for S = Q K^T, K range of O = P V
 
   if (warp == 0) {
     if (lane == 0 && !skip) {
