@@ -15,9 +15,9 @@
 namespace kd {
 namespace {
 
-// Two rows per CTA and at most 56 registers a thread: 36 warps fit on an SM, so the 4832 rows
+// Four rows per CTA and at most 56 registers a thread: 36 warps fit on an SM, so the 4832 rows
 // of a 32 x 151-token batch run in a single wave (eight-warp CTAs left a short second one).
-constexpr int LN_WARPS = 2;
+constexpr int LN_WARPS = 4;
 
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
@@ -26,12 +26,21 @@ __device__ __forceinline__ float warp_sum(float v) {
 }
 
 template <typename OutT>
-__global__ void __launch_bounds__(LN_WARPS * 32, 18) layernorm_kernel(const float* y, OutT* __restrict__ out,
-                                                        const float* __restrict__ gamma,
-                                                        const float* __restrict__ beta, int M,
-                                                        float* __restrict__ stats) {
+__global__ void __launch_bounds__(LN_WARPS * 32, 9) layernorm_kernel(const float* y, OutT* __restrict__ out,
+                                                       const float* __restrict__ gamma,
+                                                       const float* __restrict__ beta, int M,
+                                                       float* __restrict__ stats) {
+  // gamma and beta are weights, which no kernel of the loop writes: they are staged in
+  // shared memory before the dependency wait, while the previous kernel drains, so that
+  // only the row itself is read after it
+  __shared__ float4 sg[D / 4], sb[D / 4];
+  for (int i = threadIdx.x; i < D / 4; i += LN_WARPS * 32) {
+    sg[i] = reinterpret_cast<const float4*>(gamma)[i];
+    sb[i] = reinterpret_cast<const float4*>(beta)[i];
+  }
   ptx::pdl_wait();
   ptx::pdl_trigger();
+  __syncthreads();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int row = blockIdx.x * LN_WARPS + warp;
   if (row >= M) return;
@@ -58,8 +67,8 @@ __global__ void __launch_bounds__(LN_WARPS * 32, 18) layernorm_kernel(const floa
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     const int c = i * 128 + lane * 4;
-    const float4 g = *reinterpret_cast<const float4*>(gamma + c);
-    const float4 b = *reinterpret_cast<const float4*>(beta + c);
+    const float4 g = sg[c / 4];
+    const float4 b = sb[c / 4];
     const float r0 = (v[4 * i] - mean) * rstd * g.x + b.x;
     const float r1 = (v[4 * i + 1] - mean) * rstd * g.y + b.y;
     const float r2 = (v[4 * i + 2] - mean) * rstd * g.z + b.z;
