@@ -44,9 +44,9 @@ struct Tc2Cfg {
   static constexpr bool RES = KIND == EPI_BIAS_RESID || KIND == EPI_BIAS_RESID_LN;
   // K columns per pipeline stage: KA swizzle atoms of 64 (one TMA box each).  Two atoms
   // halve the stage hand-offs per MMA (wait, fence, commit: measured about 200 ns on the
-  // issuing thread, more than the MMA time of a 64-column step below N = 256) and are
-  // faster once three stages fit; beside the residual tiles only two would (slower).
-  static constexpr int KA = RES ? 1 : 2;
+  // issuing thread, more than the MMA time of a 64-column step below N = 256); three such
+  // stages fit beside the epilogue staging tiles.
+  static constexpr int KA = 2;
   static constexpr uint32_t ATOM_A = BMC * 128;          // one 64-column atom of A (128-byte rows)
   static constexpr uint32_t ATOM_B = (BN / 2) * 128;
   static constexpr uint32_t A_BYTES = KA * ATOM_A;
@@ -61,7 +61,9 @@ struct Tc2Cfg {
   static constexpr int ROW_BYTES = CW * (RES ? 4 : 2);
   // staging tiles per epilogue warp: two alternating ones, or, with a residual, one per
   // chunk of the warp's tile share so the whole residual share is loaded ahead of the MMA
-  static constexpr int NBUF = RES ? PART_CH : 2;
+  // with a residual, up to four staging tiles per warp hold the residual chunks loaded ahead;
+  // a fifth chunk reuses the first tile once its store has read it
+  static constexpr int NBUF = RES ? (PART_CH < 4 ? PART_CH : 4) : 2;
   static constexpr uint32_t EPI_BYTES = EPI_WARPS * NBUF * STG_BYTES;
   static constexpr uint32_t NUM_BARS = 2 * STAGES + 5 + NBUF * EPI_WARPS;
   static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE_BYTES + EPI_BYTES + NUM_BARS * 8 + 16;
@@ -287,10 +289,10 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
       float4 ba[CW / 4], bb[CW / 4], ga[CW / 4], gb[CW / 4];
       if (nch > 0) {
         if (C::RES && lane == 0) {
-          // the whole residual share of this tile, one staging tile per chunk, loaded while
+          // the residual chunks of this tile, one staging tile each (up to NBUF), loaded while
           // the MMAs run; the previous tile's stores have read their staging tiles first
           ptx::bulk_wait_read<0>();
-          for (int k = 0; k < nch; ++k) {
+          for (int k = 0; k < nch && k < C::NBUF; ++k) {
             const int b = (cc0 + k) % C::NBUF;
             ptx::mbar_arrive_expect_tx(res_bar(ew, b), 32 * CW * 4);
             ptx::tma_load_2d(ptx::smem_u32(stage_tile(cc0 + k)), &tmR, res_bar(ew, b), gcol + k * CW, row0);
@@ -370,6 +372,13 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
         if (lane == 0) {
           ptx::tma_store_2d(&tmO, ptx::smem_u32(st), gcol + k * CW, row0);
           ptx::bulk_commit();
+          if (C::RES && k + C::NBUF < nch) {
+            // residual chunk k + NBUF into this staging tile once the store has read it
+            ptx::bulk_wait_read<0>();
+            const int b = cc % C::NBUF;
+            ptx::mbar_arrive_expect_tx(res_bar(ew, b), 32 * CW * 4);
+            ptx::tma_load_2d(ptx::smem_u32(st), &tmR, res_bar(ew, b), gcol + (k + C::NBUF) * CW, row0);
+          }
         }
         ++cc;
         return true;
