@@ -386,22 +386,25 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
       float va[CW], vb[CW];
       ptx::tmem_ld(taddr, va);
 #pragma unroll 1
+      // The accumulator is released after the last chunk's stores are issued, not before: the
+      // remote arrive takes most of a microsecond, which at the last tile of a launch would
+      // delay its last stores, while the MMAs that wait for it start a tile later anyway.
       for (int c = 0; c < nch; c += 2) {
         ptx::tmem_ld_wait();
-        if (c == nch - 1) release();
         if (c + 1 < nch) {
           ptx::tmem_ld(taddr + (c + 1) * CW, vb);
           load_bias(c + 1, bb, gb);
         }
         if (!process(va, ba, ga, c)) { failed = true; break; }
+        if (c == nch - 1) release();
         if (c + 1 >= nch) break;
         ptx::tmem_ld_wait();
-        if (c + 1 == nch - 1) release();
         if (c + 2 < nch) {
           ptx::tmem_ld(taddr + (c + 2) * CW, va);
           load_bias(c + 2, ba, ga);
         }
         if (!process(vb, bb, gb, c + 1)) { failed = true; break; }
+        if (c + 1 == nch - 1) release();
       }
       if (failed && !*abort) record_timeout(err, WHERE_GEMM_EPILOGUE, abort);
     }
