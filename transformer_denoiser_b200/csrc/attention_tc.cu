@@ -7,7 +7,8 @@
 // exact, not online:
 //   1. TMA stages the query tile (128 x 128), the keys and the upper half of the
 //      value dimensions of the sequence's rows rounded up to 32 (128-byte swizzle, no
-//      multicast); the lower value half goes into the query buffer once S is formed.
+//      multicast; a padded sequence's keys in one box per 64-dimension half, issued one
+//      box per lane); the lower value half goes into the query buffer once S is formed.
 //   2. One thread issues S = Q K^T (M = 128, N = valid keys rounded up to 16,
 //      K = 128) into TMEM.
 //   3. Eight softmax warps (two per TMEM lane quarter, one query row per thread,
@@ -42,7 +43,7 @@ constexpr int SM_WARPS = 8;                // softmax / epilogue warps
 constexpr int NUM_THREADS = 64 + 32 * SM_WARPS;
 constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;
 constexpr int KIMODO_ETIMEOUT_CODE = -5;
-constexpr int MAX_KA = ((MAX_FRAMES + 1 + KB_ROWS - 1) / KB_ROWS) * KB_ROWS;   // 304 key rows
+constexpr int MAX_KA = ((MAX_FRAMES + 1 + KB_ROWS - 1) / KB_ROWS) * KB_ROWS;   // 320 key rows
 constexpr uint32_t Q_BYTES = QT * DH * 2;  // two 64-column halves of 16 KB
 
 // Shared memory, with ka = key rows rounded up to 32 and kp = ka rounded up to 64:
