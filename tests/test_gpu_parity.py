@@ -177,8 +177,8 @@ def test_c4_full_size_sampled(gpu_bf16, oracle_refs):
     """100-step generation at B=16, T=150 (the throughput workload, as bench.py
     runs it): sequences 0 and 15 against the oracle over all 100 steps, sequence 15
     also against the same prompt sampled alone (every projection tile sums its full K
-    extent in the same order at any batch size, so the two agree bit for bit); every
-    output finite."""
+    extent in the same order at any batch size, though alone the projections run on the
+    single-CTA kernel: checked to 1e-4); every output finite."""
     emb, null, noise, L = workload_inputs(C4)
     got = gpu_bf16.ddim_sample(emb, null, noise, L, C4[3], C4[4])
     assert np.all(np.isfinite(got))
