@@ -87,7 +87,8 @@ __device__ __forceinline__ uint64_t smem_desc_sw128_mn(uint32_t saddr, uint32_t 
 __global__ void __launch_bounds__(NUM_THREADS, 2)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmKV,
                const __grid_constant__ CUtensorMap tmO, bf16* __restrict__ out, const int* __restrict__ lengths, int len_mod, int S_pad, int ka,
-               uint32_t tmem_cols, uint32_t o_col, const int* __restrict__ tok0, int kbox, DevError* err) {
+               uint32_t tmem_cols, uint32_t o_col, const int* __restrict__ tok0, int kbox, DevError* err,
+               L2Prefetch pf) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t kp = kp_of(ka);
@@ -124,6 +125,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     ptx::fence_mbar_init();
     ptx::tma_prefetch_desc(&tmQ);
     ptx::tma_prefetch_desc(&tmKV);
+    ptx::prefetch_l2_share(pf, blockIdx.x + gridDim.x * (blockIdx.y + (unsigned long long)gridDim.y * blockIdx.z),
+                           (unsigned long long)gridDim.x * gridDim.y * gridDim.z);
   }
   if (warp == 1) {
     ptx::tmem_alloc(ptx::smem_u32(tmem_slot), tmem_cols);
@@ -411,7 +414,7 @@ cudaError_t attention_tc_prepare() {
 }
 
 cudaError_t attention_tc(const bf16* qkv, bf16* out, int M, const int* lengths, int len_mod, int nseq, int S,
-                         DevError* err, cudaStream_t st, const int* tok0) {
+                         DevError* err, cudaStream_t st, const int* tok0, L2Prefetch pf) {
   if (nseq <= 0 || S <= 0 || M <= 0) return cudaSuccess;
   if (S > MAX_FRAMES + 1) return cudaErrorInvalidValue;
   CUtensorMap tq, tkv, to;
@@ -431,7 +434,7 @@ cudaError_t attention_tc(const bf16* qkv, bf16* out, int M, const int* lengths, 
   const uint32_t o_col = n_cols_max <= 256 ? 0u : 320u;
   dim3 grid(H, nseq, (S + QT - 1) / QT);
   return launch_kernel(attn_tc_kernel, grid, dim3(NUM_THREADS), smem_bytes(ka), st, tq, tkv, to, out, lengths, len_mod,
-                       S, ka, tmem_cols, o_col, tok0, kbox, err);
+                       S, ka, tmem_cols, o_col, tok0, kbox, err, pf);
 }
 
 }  // namespace kd

@@ -176,6 +176,9 @@ int launch(kimodo_ctx* c, int cls, double flops, double bytes, cudaStream_t st, 
   return KIMODO_OK;
 }
 
+// Token rows from which the layer projections run on the CTA-pair kernel.
+constexpr int PAIR_GEMM_MIN_ROWS = 1024;
+
 int pick_bn(const kimodo_ctx* c, int M, int N, int kind, bool out_f32) {
   if (N <= 16) return 16;
   if (N < 1024) return 128;
@@ -208,7 +211,7 @@ int gemm(kimodo_ctx* c, const void* A, int lda, const void* W, int ldw, int M, i
                        (double)M * N * (out_f32 ? 4.0 : (double)c->elem()) +
                        (kind == EPI_BIAS_RESID || kind == EPI_BIAS_RESID_LN ? (double)M * N * 4.0 : 0.0);
   if (c->bf16()) {
-    if (M >= 1024 && N >= 256 && gemm_tc2_supports(kind, out_f32)) {
+    if (M >= PAIR_GEMM_MIN_ROWS && N >= 256 && gemm_tc2_supports(kind, out_f32)) {
       const int bn = gemm_tc2_pick_bn(M, N, kind);
       return launch(c, cls_override >= 0 ? cls_override : CLS_GEMM_TC, flops, bytes, st, "gemm_tc2",
                     [&] { return gemm_tc2(g, bn, kind, out_f32, ep, c->derr, st); });
@@ -426,7 +429,26 @@ int run_net(kimodo_ctx* c, int net, int nseq, int T, int len_mod, const void* A_
     e.ln_b = b;
     return EPI_BIAS_RESID_LN;
   };
+  // Weights of the projections ahead, pulled into L2 by the kernels between them when the
+  // projections run on the single-CTA kernel (below 1024 tokens, where a projection's
+  // weights would otherwise come from HBM inside its K loop; the CTA-pair kernel pulls
+  // its own weights into L2 before its dependency wait, and there the extra prefetch
+  // slowed attention): attention fetches the rest of its layer (attention output, FFN1,
+  // FFN2), the second LayerNorm the next layer's QKV weights.  A layer's weights are
+  // consecutive in the arena (QKV, attention output, LayerNorm 1, FFN1, FFN2, LayerNorm 2).
+  const bool prefetch_ahead = bf && M < PAIR_GEMM_MIN_ROWS;
+  auto span = [prefetch_ahead](const void* a, const void* b) {
+    L2Prefetch p;
+    const uintptr_t ua = reinterpret_cast<uintptr_t>(a), ub = reinterpret_cast<uintptr_t>(b);
+    if (prefetch_ahead && a != nullptr && ub > ua && (ua & 15) == 0 && ((ub - ua) & 15) == 0) {
+      p.p = a;
+      p.bytes = ub - ua;
+    }
+    return p;
+  };
   for (int l = 0; l < L; ++l) {
+    const L2Prefetch pf_layer = span(n.o_W[l], l + 1 < L ? n.qkv_W[l + 1] : n.out_W);
+    const L2Prefetch pf_next = l + 1 < L ? span(n.qkv_W[l + 1], n.o_W[l + 1]) : L2Prefetch{};
     EpiParams e;
     e.bias = n.qkv_b[l]; e.out = w.qkv; e.ldo = 3 * D; e.N = 3 * D; e.M = M;
     KD_TRY(gemm(c, w.h, D, n.qkv_W[l], D, M, 3 * D, D, EPI_BIAS, act_f32, e, st));
@@ -435,7 +457,7 @@ int run_net(kimodo_ctx* c, int net, int nseq, int T, int len_mod, const void* A_
     if (bf) {
       KD_TRY(launch(c, CLS_ATTN, aflops, abytes, st, "attention_tc", [&] {
         return attention_tc(static_cast<const bf16*>(w.qkv), static_cast<bf16*>(w.attn), M, w.lengths, len_mod,
-                            nseq, S, c->derr, st, tok0);
+                            nseq, S, c->derr, st, tok0, pf_layer);
       }));
     } else {
       KD_TRY(launch(c, CLS_ATTN, aflops, abytes, st, "attention_f32", [&] {
@@ -462,7 +484,7 @@ int run_net(kimodo_ctx* c, int net, int nseq, int T, int len_mod, const void* A_
     const int kf = resid_epi(e2, 0, n.ln1_g[l], n.ln1_b[l]);
     KD_TRY(gemm(c, w.u, F, n.ff2_W[l], F, M, D, F, kf, true, e2, st));
     KD_TRY(launch(c, CLS_LN, 0, lnb, st, "layernorm", [&] {
-      return layernorm(w.y, w.h, bf, n.ln2_g[l], n.ln2_b[l], M, st, bf ? w.stats[1] : nullptr);
+      return layernorm(w.y, w.h, bf, n.ln2_g[l], n.ln2_b[l], M, st, bf ? w.stats[1] : nullptr, pf_next);
     }));
   }
   EpiParams eo;

@@ -36,6 +36,14 @@ struct DevError {
   int info;
 };
 
+// A range of weights that a kernel pulls into L2 for the projections that follow it
+// (16-byte aligned, a multiple of 16 bytes; null: none).  Weights are written only when
+// they are loaded, so the prefetch may run before the kernel's dependency wait.
+struct L2Prefetch {
+  const void* p = nullptr;
+  unsigned long long bytes = 0;
+};
+
 enum DevErrWhere : int {
   WHERE_GEMM_PRODUCER = 1,
   WHERE_GEMM_MMA = 2,

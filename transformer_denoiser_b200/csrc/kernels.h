@@ -55,9 +55,10 @@ cudaError_t attention_f32(const float* qkv, float* out, const int* lengths, int 
 
 // The same attention on the tcgen05 tensor cores (bf16 path): one CTA per (head, sequence,
 // 128-query tile), exact softmax over all keys of the sequence at once.  qkv has M
-// rows (16-byte aligned, row stride 3*D); S <= MAX_FRAMES + 1.
+// rows (16-byte aligned, row stride 3*D); S <= MAX_FRAMES + 1.  pf: weights its CTAs pull
+// into L2 for the projections that follow.
 cudaError_t attention_tc(const bf16* qkv, bf16* out, int M, const int* lengths, int len_mod, int nseq, int S,
-                         DevError* err, cudaStream_t st, const int* tok0 = nullptr);
+                         DevError* err, cudaStream_t st, const int* tok0 = nullptr, L2Prefetch pf = {});
 cudaError_t attention_tc_prepare();
 size_t attention_tc_smem(int S);
 
@@ -66,9 +67,10 @@ size_t attention_tc_smem(int S);
 cudaError_t build_token_map(const int* lengths, int len_mod, int nseq, int* tok0, int* row_seq, cudaStream_t st);
 
 // Row LayerNorm over D features: y fp32 [M, D] -> out (bf16 or fp32) [M, D], and
-// optionally the row statistics (mean, 1/std) into stats [M][2].
+// optionally the row statistics (mean, 1/std) into stats [M][2]; pf: weights its CTAs pull
+// into L2 for the projections that follow.
 cudaError_t layernorm(const float* y, void* out, bool out_bf16, const float* gamma, const float* beta, int M,
-                      cudaStream_t st, float* stats = nullptr);
+                      cudaStream_t st, float* stats = nullptr, L2Prefetch pf = {});
 
 // ---- motion / sampler kernels (element type of the activation matrices: bf16 or fp32)
 

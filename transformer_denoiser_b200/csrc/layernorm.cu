@@ -29,7 +29,7 @@ template <typename OutT>
 __global__ void __launch_bounds__(LN_WARPS * 32, 9) layernorm_kernel(const float* y, OutT* __restrict__ out,
                                                        const float* __restrict__ gamma,
                                                        const float* __restrict__ beta, int M,
-                                                       float* __restrict__ stats) {
+                                                       float* __restrict__ stats, L2Prefetch pf) {
   // gamma and beta are weights, which no kernel of the loop writes: they are staged in
   // shared memory before the dependency wait, while the previous kernel drains, so that
   // only the row itself is read after it
@@ -38,6 +38,7 @@ __global__ void __launch_bounds__(LN_WARPS * 32, 9) layernorm_kernel(const float
     sg[i] = reinterpret_cast<const float4*>(gamma)[i];
     sb[i] = reinterpret_cast<const float4*>(beta)[i];
   }
+  if (threadIdx.x == 0) ptx::prefetch_l2_share(pf, blockIdx.x, gridDim.x);
   ptx::pdl_wait();
   ptx::pdl_trigger();
   __syncthreads();
@@ -88,14 +89,14 @@ __global__ void __launch_bounds__(LN_WARPS * 32, 9) layernorm_kernel(const float
 }  // namespace
 
 cudaError_t layernorm(const float* y, void* out, bool out_bf16, const float* gamma, const float* beta, int M,
-                      cudaStream_t st, float* stats) {
+                      cudaStream_t st, float* stats, L2Prefetch pf) {
   if (M <= 0) return cudaSuccess;
   const int grid = (M + LN_WARPS - 1) / LN_WARPS;
   if (out_bf16)
     return launch_kernel(layernorm_kernel<bf16>, dim3(grid), dim3(LN_WARPS * 32), 0, st, y, static_cast<bf16*>(out), gamma, beta,
-                         M, stats);
+                         M, stats, pf);
   return launch_kernel(layernorm_kernel<float>, dim3(grid), dim3(LN_WARPS * 32), 0, st, y, static_cast<float*>(out), gamma, beta,
-                       M, stats);
+                       M, stats, pf);
 }
 
 }  // namespace kd

@@ -93,6 +93,26 @@ __device__ __forceinline__ void tma_prefetch_l2_2d(const CUtensorMap* m, int c0,
                ::"l"(reinterpret_cast<uint64_t>(m)), "r"(c0), "r"(c1) : "memory");
 }
 
+// Prefetch of `bytes` (a multiple of 16) of global memory at a 16-byte aligned address
+// into L2 (no shared memory, no completion).
+__device__ __forceinline__ void prefetch_l2_bulk(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(p)), "r"(bytes)
+               : "memory");
+}
+
+// CTA `cta` of `ncta` prefetches its equal share (16-byte multiples) of an L2 range.
+__device__ __forceinline__ void prefetch_l2_share(const L2Prefetch& pf, unsigned long long cta,
+                                                  unsigned long long ncta) {
+  if (pf.p == nullptr || pf.bytes == 0 || ncta == 0) return;
+  const unsigned long long share = ((pf.bytes + ncta - 1) / ncta + 15) & ~15ull;
+  unsigned long long off = cta * share;
+  const unsigned long long end = off + share < pf.bytes ? off + share : pf.bytes;
+  for (; off < end; off += (1ull << 30)) {
+    const unsigned long long n = end - off < (1ull << 30) ? end - off : (1ull << 30);
+    prefetch_l2_bulk(static_cast<const char*>(pf.p) + off, (uint32_t)n);
+  }
+}
+
 // ---------------------------------------------------------------- tcgen05
 __device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols) {
   asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
